@@ -1,0 +1,536 @@
+"""Benchmark: one paged decode step per iteration on the batch-256 GQA layer.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload NAME] [--partition P]
+
+A step is one pass of the whole hot path over one batch: copy_blocks (when
+the workload has copy-on-write pairs), reshape_and_cache of the step's new
+K/V, and paged decode attention (plus its split-KV merge when split).  Inputs
+are resident in HBM when the timed region starts; the KV pool (2.5 GB for the
+default workload) is larger than the 126 MB L2, so no flush is needed between
+steps.  Timing: W untimed steps, then K steps between CUDA events on the
+launching stream, bracketed by a barrier and device synchronisation; the
+maximum over ranks is reported.  Under torchrun every rank runs its own
+replica of the workload (independent sequences, no collective on the data
+path): weak scaling.
+
+value  = algorithmic bytes of the step / step time (GB/s): unique KV bytes
+         read (2 * num_kv_heads * head_size * 2 per distinct cached token, the
+         per-block formula of the KV-cache manager) + q + fp32 out + used
+         block-table entries + context lengths + the cache write (new K/V in,
+         rows out, slots) + copy-on-write bytes when present.
+roofline = the decode-attention kernel alone: its algorithmic bytes per launch
+         / its average CUDA-event duration, against the measured HBM peak.
+e2e    = the same metric through the public API with host buffers: per step
+         the step's inputs go host->device from pinned memory, the output
+         comes back device->host, all inside the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = ("paged decode attn: KV GB/s and % of HBM peak; seq-tokens/s at "
+          "batch 256")
+DEFAULT_WORKLOAD = "llama2_70b_gqa_b256"
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_dram_traffic.txt")
+KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_435_b200", "csrc", f)
+                  for f in ("pa_decode.cu", "pa_common.cuh", "pa_decode.cuh")]
+
+
+# ---------------------------------------------------------------- accounting
+def attention_bytes(case, seqs=None) -> int:
+    """Algorithmic bytes of one decode-attention call."""
+    w = case.workload
+    lens = case.lens_np if seqs is None else case.lens_np[seqs]
+    B = len(lens)
+    uniq = case.unique_tokens if seqs is None else int(lens.sum())
+    kv = uniq * 2 * w.num_kv_heads * w.head_size * 2
+    q = B * w.num_heads * w.head_size * 2
+    out = B * w.num_heads * w.head_size * 4
+    tables = int((-(-lens // w.block_size)).sum()) * 4
+    return kv + q + out + tables + B * 4
+
+
+def step_bytes(case) -> int:
+    w = case.workload
+    row = w.num_kv_heads * w.head_size * 2
+    live = int((case.slot_mapping.cpu() >= 0).sum())
+    write = 2 * live * row * 2 + case.slot_mapping.numel() * 8
+    cow = 0
+    if case.copy_pairs.shape[0]:
+        blk = w.block_size * row
+        cow = case.copy_pairs.shape[0] * (2 * blk * 2 + 16)
+    return attention_bytes(case) + write + cow
+
+
+def kernel_sha() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def read_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel source for this workload."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    kv = {}
+    with open(PROFILE_TRAFFIC) as f:
+        for line in f:
+            if "=" in line and not line.lstrip().startswith("#"):
+                k, v = line.split("=", 1)
+                kv[k.strip()] = v.strip()
+    if kv.get("kernel_sha") != kernel_sha() or kv.get("workload") != workload:
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """SM clock and throttle reasons via NVML while the timed region runs."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nvml = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        n = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
+                self.reasons |= int(n.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._nvml is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0}
+        names = [v for k, v in self.REASONS.items()
+                 if self.reasons & k and k != 0x1]
+        return {"sm_mhz": float(np.median(self.samples)),
+                "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- distributed
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        return dist
+    return None
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def max_over_ranks(dist, x: float, device) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- GPU arm
+class Step:
+    """Device buffers and the library calls of one decode step."""
+
+    def __init__(self, case, partition_size: int):
+        import paged_kv_cache_435_b200 as pa
+        self.pa = pa
+        self.case = case
+        w = case.workload
+        B, Hq, D = case.q.shape
+        self.out = torch.empty(B, Hq, D, dtype=torch.float32, device=case.q.device)
+        self.maxlen = case.max_context_len
+        self.partition = pa.pa_decode_partition_size(
+            B, Hq, w.num_kv_heads, D, w.block_size, self.maxlen, partition_size)
+        self.partition_arg = partition_size
+        nbytes = pa.pa_decode_workspace_size(B, Hq, w.num_kv_heads, D,
+                                             w.block_size, self.maxlen,
+                                             partition_size)
+        self.ws = (torch.empty(nbytes, dtype=torch.uint8, device=case.q.device)
+                   if nbytes else None)
+        self.flags = torch.zeros(1, dtype=torch.int32, device=case.q.device)
+
+    def cache_ops(self):
+        c = self.case
+        if c.copy_pairs.shape[0]:
+            self.pa.pa_copy_blocks([c.k_cache], [c.v_cache], c.copy_pairs,
+                                   error_flags=self.flags)
+        self.pa.pa_reshape_and_cache(c.new_key, c.new_value, c.k_cache,
+                                     c.v_cache, c.slot_mapping,
+                                     error_flags=self.flags)
+
+    def attention(self):
+        c = self.case
+        self.pa.pa_decode_attention(
+            self.out, c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens,
+            self.maxlen, c.scale, partition_size=self.partition_arg,
+            workspace=self.ws, error_flags=self.flags)
+
+
+def run_gpu(args):
+    import paged_kv_cache_435_b200 as pa
+    from paged_kv_cache_435_b200 import inputs
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    pa.raw()  # fail loudly if the library is missing
+
+    case = inputs.make_case(args.workload, device=dev)
+    w = case.workload
+    part = args.partition if args.partition is not None else w.partition_size
+    step = Step(case, part)
+    stream = torch.cuda.current_stream(dev)
+
+    # in-run copy bandwidth (read + write bytes of a 1 GiB device copy)
+    a = torch.empty(1 << 29, dtype=torch.bfloat16, device=dev)
+    b = torch.empty_like(a)
+    copy_best = 0.0
+    for _ in range(6):
+        e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+        e0.record(stream); b.copy_(a); e1.record(stream); e1.synchronize()
+        copy_best = max(copy_best, 2 * a.numel() * 2 / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+    del a, b
+
+    for _ in range(args.warmup):
+        step.cache_ops(); step.attention()
+    torch.cuda.synchronize(dev)
+
+    K = args.steps
+    ev_attn = [(torch.cuda.Event(True), torch.cuda.Event(True)) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    with ClockSampler(local) as clk:
+        barrier(dist)
+        torch.cuda.synchronize(dev)
+        n0 = pa.pa_launch_count()
+        t0.record(stream)
+        for i in range(K):
+            step.cache_ops()
+            ev_attn[i][0].record(stream)
+            step.attention()
+            ev_attn[i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        launches = pa.pa_launch_count() - n0
+        barrier(dist)
+    ms_total = t0.elapsed_time(t1)
+    attn_ms = sum(s.elapsed_time(e) for s, e in ev_attn) / K
+    flags = int(step.flags.item())
+
+    # e2e: host buffers through the public API
+    e2e = run_e2e(case, step, args, dist, dev)
+
+    ms_total = max_over_ranks(dist, ms_total, dev)
+    attn_ms_max = max_over_ranks(dist, attn_ms, dev)
+    sb = step_bytes(case)
+    ab = attention_bytes(case)
+    ms_step = ms_total / K
+    value = world * sb / (ms_step * 1e-3) / 1e9
+    peak, peak_kind = hbm_peak()
+    achieved = ab / (attn_ms_max * 1e-3) / 1e9
+    traffic = read_traffic(args.workload)
+
+    result = None
+    if rank == 0:
+        cpu = cpu_baseline(args) if world == 1 else None
+        clocks = clk.summary()
+        result = {
+            "metric": METRIC,
+            "value": round(value, 2),
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16, random scattered block tables)",
+            "config": {
+                "workload": w.name,
+                "description": w.description,
+                "num_seqs": w.num_seqs, "num_heads": w.num_heads,
+                "num_kv_heads": w.num_kv_heads, "head_size": w.head_size,
+                "block_size": w.block_size,
+                "num_blocks": int(case.k_cache.shape[0]),
+                "context_tokens": case.logical_tokens,
+                "unique_kv_tokens": case.unique_tokens,
+                "partition_size": step.partition,
+                "step": ("copy_blocks + " if case.copy_pairs.shape[0] else "") +
+                        "reshape_and_cache + paged_decode_attention",
+                "l2": "no flush: inputs larger than L2 (KV pool "
+                      f"{2 * case.k_cache.numel() * 2 / 1e9:.2f} GB > 126 MB)",
+                "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            },
+            "seq_tokens_per_s": round(world * w.num_seqs / (ms_step * 1e-3), 1),
+            "context_tokens_per_s": round(world * case.logical_tokens / (ms_step * 1e-3), 1),
+            "pct_hbm_peak": round(100 * value / (world * peak), 2),
+            "step_bytes": sb,
+            "in_run_copy_gbs": round(copy_best, 1),
+            "roofline": {
+                "kernel": "paged_decode_kernel" + (" + reduce" if step.partition < case.max_context_len else ""),
+                "bound": "hbm",
+                "achieved": round(achieved, 1),
+                "peak": peak,
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s",
+                "unit": "GB/s",
+                "frac": round(achieved / peak, 4),
+                "frac_of_in_run_copy": round(achieved / copy_best, 4),
+                "traffic": traffic,
+                "algorithmic_bytes_per_launch": ab,
+                "avg_launch_ms": round(attn_ms_max, 5),
+            },
+            "e2e": e2e,
+            "gpu_launches": int(launches),
+            "device_error_flags": flags,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def run_e2e(case, step, args, dist, dev):
+    """Per step: pinned host -> device copies of the step's inputs, the
+    library calls, device -> host copy of the output."""
+    c = case
+    host_in = {n: getattr(c, n).cpu().pin_memory() for n in
+               ("q", "new_key", "new_value", "slot_mapping", "block_tables",
+                "context_lens")}
+    if c.copy_pairs.shape[0]:
+        host_in["copy_pairs"] = c.copy_pairs.cpu().pin_memory()
+    host_out = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_out.numel() * host_out.element_size()
+    stream = torch.cuda.current_stream(dev)
+
+    def one():
+        for n, t in host_in.items():
+            getattr(c, n).copy_(t, non_blocking=True)
+        step.cache_ops()
+        step.attention()
+        host_out.copy_(step.out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        one()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    t0, t1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    barrier(dist)
+    t0.record(stream)
+    for _ in range(K):
+        one()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(dist, t0.elapsed_time(t1), dev) / K
+    world = dist.get_world_size() if dist is not None else 1
+    return {"value": round(world * step_bytes(case) / (ms * 1e-3) / 1e9, 2),
+            "unit": "GB/s", "ms_per_step": round(ms, 5),
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+# ---------------------------------------------------------------- CPU (oracle)
+def oracle_sample(workload: str, n_seqs: int):
+    """A bounded sample of the workload built on the host: the first n_seqs
+    sequences of its seeded length draw, same shapes, its own pool."""
+    from paged_kv_cache_435_b200 import inputs
+    w = inputs.WORKLOADS[workload]
+    if w.lengths == "shared":
+        full = inputs.make_case(workload)  # host-sized (0.3 GB pool)
+        return full, np.arange(min(n_seqs, w.num_seqs))
+    rng = np.random.default_rng(1000 + w.wid)
+    lens = inputs.draw_lengths(w.lengths, w.num_seqs, rng)[:n_seqs]
+    sub = dataclasses.replace(w, num_seqs=len(lens), name=w.name + "_sample")
+    return inputs.build_case(sub, lens, seed=4242), None
+
+
+def time_oracle(case, seqs, threads):
+    import oracle
+    q, tables, lens = case.q, case.tables_np, case.lens_np.astype(np.int32)
+    if seqs is not None:
+        q = q[torch.from_numpy(seqs)]
+        tables, lens = tables[seqs], lens[seqs]
+    t = time.perf_counter()
+    oracle.paged_decode_attention(q, case.k_cache, case.v_cache, tables, lens,
+                                  case.scale, case.workload.num_kv_heads,
+                                  threads=threads)
+    return time.perf_counter() - t
+
+
+def sample_bytes(case, seqs):
+    if seqs is None:
+        return attention_bytes(case)
+    # a shared-prefix sample: count the distinct cached tokens it reads
+    w = case.workload
+    bs = w.block_size
+    slots = set()
+    for s in seqs:
+        L = int(case.lens_np[s])
+        row = case.tables_np[s]
+        slots.update(int(row[t // bs]) * bs + t % bs for t in range(L))
+    B = len(seqs)
+    lens = case.lens_np[seqs]
+    kv = len(slots) * 2 * w.num_kv_heads * w.head_size * 2
+    tables = int((-(-lens // bs)).sum()) * 4
+    return kv + B * w.num_heads * w.head_size * 6 + tables + B * 4
+
+
+def cpu_baseline(args, budget_s: float = 10.0):
+    import oracle
+    oracle.build()
+    threads = oracle.default_threads()
+    case, seqs = oracle_sample(args.workload, 64)
+    nbytes = sample_bytes(case, seqs)
+    reps, elapsed = 0, 0.0
+    while elapsed < budget_s or reps == 0:
+        elapsed += time_oracle(case, seqs, threads)
+        reps += 1
+    n = case.workload.num_seqs if seqs is None else len(seqs)
+    return {"value": round(reps * nbytes / elapsed / 1e9, 4), "unit": "GB/s",
+            "cores": threads, "kind": "oracle",
+            "sample": f"{n} sequences of {args.workload} (same shapes and "
+                      f"length draw, host-built pool), {reps} passes, "
+                      f"{elapsed:.1f} s, fp64 C oracle on {threads} threads",
+            "seq_tokens_per_s": round(reps * n / elapsed, 2)}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: each step one bounded sample."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    import oracle
+    oracle.build()
+    threads = oracle.default_threads()
+    # size one step's sample so warm-up + timed steps take about two minutes
+    probe, pseqs = oracle_sample(args.workload, 4)
+    per_seq = time_oracle(probe, pseqs, threads) / 4
+    budget = min(2.0, 120.0 / (args.steps + args.warmup))
+    from paged_kv_cache_435_b200 import inputs
+    n = int(max(1, min(inputs.WORKLOADS[args.workload].num_seqs,
+                       round(budget / max(per_seq, 1e-6)))))
+    case, seqs = oracle_sample(args.workload, n)
+    nbytes = sample_bytes(case, seqs)
+    for _ in range(args.warmup):
+        time_oracle(case, seqs, threads)
+    t = 0.0
+    for _ in range(args.steps):
+        t += time_oracle(case, seqs, threads)
+    ms = 1e3 * t / args.steps
+    value = nbytes / (ms * 1e-3) / 1e9
+    n = case.workload.num_seqs if seqs is None else len(seqs)
+    from paged_kv_cache_435_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16, random scattered block tables)",
+        "config": {"workload": w.name, "description": w.description,
+                   "sample_seqs_per_step": n},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s",
+                         "cores": threads, "kind": "oracle",
+                         "sample": f"{n} sequences of {w.name} per step, fp64 C "
+                                   f"oracle on {threads} threads"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s",
+                "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--partition", type=int, default=None)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    res = run_reference(args) if args.impl == "reference" else run_gpu(args)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,207 @@
+/*
+ * pa.h - C ABI of libpagedattn.so: paged decode attention and its two cache
+ * companions, hand-written CUDA for NVIDIA B200 (sm_100a).
+ *
+ * The method.  The KV cache of every sequence is kept in fixed-size,
+ * non-contiguous physical blocks; a per-sequence block table maps logical
+ * block i of the sequence to a physical block id, and blocks are handed out
+ * on demand from a free pool ("vLLM: Anatomy and Mechanisms of High-Throughput
+ * LLM Inference", section "PagedAttention: The vLLM Innovation" /
+ * "Block-Level Management"; "vLLM Internals", section "The Block Manager").
+ * A decode step attends with one new query token per sequence over that
+ * sequence's cached context (first page, "Prefill vs. Decode Operations";
+ * decode is memory-bandwidth bound there and in "The Roofline Model").
+ * Sequences may share physical blocks; when a shared block diverges, only
+ * that block is copied (first page, "Memory Sharing via Copy-on-Write
+ * (CoW)").  One block of K and V occupies
+ * 2 * block_size * num_kv_heads * head_size * 2 bytes in bf16 ("Inside vLLM:
+ * Anatomy of a High-Throughput LLM Inference System", section "LLM Engine
+ * constructor", KV-cache manager).
+ *
+ * Data layout shared by every call (all device memory, row-major):
+ *   k_cache, v_cache  bf16 [num_blocks][block_size][num_kv_heads][head_size],
+ *                     contiguous, base address 16-byte aligned.  Token slot
+ *                     s = block_id * block_size + offset.
+ *   block_tables      int32 [num_seqs][max_blocks_per_seq]; entry i of row s
+ *                     is the physical block holding tokens
+ *                     [i*block_size, (i+1)*block_size) of sequence s.  Entries
+ *                     at or past ceil(context_lens[s] / block_size) are never
+ *                     read (they may hold -1).
+ *   context_lens      int32 [num_seqs]; tokens in the context of sequence s,
+ *                     INCLUDING the current token (whose K/V a prior
+ *                     pa_reshape_and_cache wrote).  0 means an empty context.
+ *   q                 bf16 [num_seqs][num_heads][head_size], contiguous.
+ *   out               fp32 [num_seqs][num_heads][head_size], contiguous.
+ *
+ * GQA grouping: query head h reads kv head h / (num_heads / num_kv_heads)
+ * (contiguous groups; the pages name num_kv_heads but not the mapping).
+ *
+ * Conventions.
+ *   - Ownership: the caller owns every buffer, including the workspace.  The
+ *     library never allocates or frees device memory and keeps no state
+ *     between calls other than a process-wide launch counter.
+ *   - Asynchrony: every call only enqueues work on `stream` (0 = the legacy
+ *     default stream) and returns; it never synchronises the host.
+ *   - Host-side validation happens before any launch; on failure nothing is
+ *     enqueued and a negative pa_status is returned.
+ *   - Device-side checks: every block id, slot and context length read from
+ *     device memory is bounds-checked in the kernel.  A violation never
+ *     touches memory outside the caller's buffers: the access is redirected
+ *     or skipped, the affected outputs are unspecified, and the matching
+ *     PA_DEVERR_* bit is OR-ed into *error_flags when error_flags is non-NULL
+ *     (a device int the caller zeroes and reads after the stream completes).
+ *   - Supported now: head_size in {64, 128}; block_size in {16, 32};
+ *     num_heads / num_kv_heads in 1..8.  Other values return
+ *     PA_ERR_UNSUPPORTED.
+ */
+#ifndef PAGEDATTN_B200_PA_H
+#define PAGEDATTN_B200_PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle; identical to cudaStream_t / CUstream. */
+typedef struct CUstream_st* pa_stream_t;
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = -1, /* null pointer, bad size, misaligned buffer */
+    PA_ERR_UNSUPPORTED = -2, /* valid but not implemented (head_size...) */
+    PA_ERR_WORKSPACE = -3,   /* workspace missing or smaller than needed */
+    PA_ERR_CUDA = -4         /* the CUDA runtime reported a launch error */
+} pa_status;
+
+/* Bits OR-ed into *error_flags by the kernels. */
+#define PA_DEVERR_BLOCK_ID 0x1    /* block-table entry outside [0,num_blocks) */
+#define PA_DEVERR_CONTEXT_LEN 0x2 /* context_lens[s] < 0 or > max_context_len */
+#define PA_DEVERR_SLOT 0x4        /* slot_mapping entry >= num_blocks*block_size */
+#define PA_DEVERR_COPY_PAIR 0x8   /* block_mapping id outside [0,num_blocks) */
+#define PA_DEVERR_TIMEOUT 0x10    /* an async-copy wait exceeded its time limit */
+
+/* Human-readable name of a pa_status value (static string, never NULL). */
+const char* pa_status_string(int status);
+
+/* ABI version: (major << 16) | minor. */
+int pa_version(void);
+
+/* Number of kernels this library has launched in this process so far
+ * (monotonic; lets a caller count the library's launches in a region). */
+uint64_t pa_launch_count(void);
+
+/*
+ * pa_reshape_and_cache - write each new token's K and V rows into its cache
+ * slot.  For token i with s = slot_mapping[i] >= 0:
+ *     k_cache[s / block_size][s % block_size][h][:] = key[i][h][:]
+ *     v_cache[s / block_size][s % block_size][h][:] = value[i][h][:]
+ * for every kv head h.  s < 0 marks a padding token and is skipped.  This is
+ * the cache write behind on-demand slot allocation ("Block-Level
+ * Management"; "Allocate, reshape and bind KV cache tensors" under "LLM
+ * Engine constructor" on the second page).  The copy is bit-exact.
+ *
+ *   key, value           bf16 [num_tokens][num_kv_heads][head_size] with a
+ *                        token stride of key_token_stride / value_token_stride
+ *                        ELEMENTS (>= num_kv_heads*head_size); heads and
+ *                        dims are contiguous within a token.
+ *   k_cache, v_cache     the pool (layout above), written in place.
+ *   slot_mapping         int64 [num_tokens], device.
+ *   num_tokens           >= 0 (0 enqueues nothing and returns PA_OK).
+ *   error_flags          nullable device int; PA_DEVERR_SLOT on a slot
+ *                        >= num_blocks*block_size (that token is skipped).
+ * Two tokens mapping to the same slot is a caller error (last writer is
+ * unspecified).  Returns PA_OK or a negative pa_status.
+ */
+int pa_reshape_and_cache(const void* key, const void* value,
+                         int64_t key_token_stride, int64_t value_token_stride,
+                         void* k_cache, void* v_cache,
+                         const int64_t* slot_mapping, int num_tokens,
+                         int num_blocks, int block_size, int num_kv_heads,
+                         int head_size, int* error_flags, pa_stream_t stream);
+
+/*
+ * pa_decode_partition_size - the KV partition width, in tokens, that
+ * pa_decode_attention uses for these arguments (resolves partition_size = 0
+ * to the library heuristic).  A result >= max_context_len means one
+ * partition per sequence (no split).  Pure host function.
+ */
+int pa_decode_partition_size(int num_seqs, int num_heads, int num_kv_heads,
+                             int head_size, int block_size,
+                             int max_context_len, int partition_size);
+
+/*
+ * pa_decode_workspace_size - bytes of device workspace pa_decode_attention
+ * needs for the same arguments (0 when no split is used).  Pure host function.
+ */
+size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                int head_size, int block_size,
+                                int max_context_len, int partition_size);
+
+/*
+ * pa_decode_attention - paged decode attention, one query token per sequence.
+ * For each sequence s with L = context_lens[s] and each query head h
+ * (kv head g = h / (num_heads/num_kv_heads)):
+ *     k_t = k_cache[block_tables[s][t / block_size]][t % block_size][g][:]
+ *     z_t = scale * dot(q[s][h][:], k_t)              for t in [0, L)
+ *     out[s][h][:] = sum_t softmax(z)_t * v_t          (fp32)
+ * and out[s][h][:] = 0 when L = 0.
+ *
+ * Work is split into one CTA per (sequence, kv head, KV partition); the CTA
+ * reads each of its blocks once for all query heads of the group.  Contexts
+ * longer than the partition width are split into partitions whose (max, sum,
+ * normalised partial output) are merged by a second kernel.
+ *
+ *   max_blocks_per_seq   row length of block_tables (>= 1).
+ *   max_context_len      host-known upper bound of context_lens
+ *                        (<= max_blocks_per_seq*block_size); sizes the split.
+ *   scale                logit scale (e.g. 1/sqrt(head_size)).
+ *   partition_size       0: library heuristic; otherwise the partition width
+ *                        in tokens, a positive multiple of block_size.
+ *   workspace            device buffer of at least
+ *                        pa_decode_workspace_size(...) bytes, 256-byte
+ *                        aligned (may be NULL when that size is 0).  Its
+ *                        contents need no initialisation and are scratch.
+ *   error_flags          nullable device int (PA_DEVERR_BLOCK_ID,
+ *                        PA_DEVERR_CONTEXT_LEN, PA_DEVERR_TIMEOUT).
+ * Returns PA_OK or a negative pa_status.  Run-to-run results are bitwise
+ * deterministic for identical arguments.
+ */
+int pa_decode_attention(float* out, const void* q, const void* k_cache,
+                        const void* v_cache, const int32_t* block_tables,
+                        int max_blocks_per_seq, const int32_t* context_lens,
+                        int max_context_len, int num_seqs, int num_heads,
+                        int num_kv_heads, int head_size, int block_size,
+                        int num_blocks, float scale, int partition_size,
+                        void* workspace, size_t workspace_bytes,
+                        int* error_flags, pa_stream_t stream);
+
+/*
+ * pa_copy_blocks - copy-on-write block copies ("Memory Sharing via
+ * Copy-on-Write (CoW)": when sequences sharing a block diverge, only that
+ * block is copied).  For each pair p and each layer l:
+ *     k_caches[l][dst] = k_caches[l][src],  v_caches[l][dst] = v_caches[l][src]
+ * with (src, dst) = (block_mapping[2p], block_mapping[2p+1]); whole blocks,
+ * bit-exact.
+ *
+ *   k_caches, v_caches   HOST arrays of num_layers device pointers, each a
+ *                        pool with the layout above (same shape per layer).
+ *   block_mapping        int64 [num_pairs][2], device.
+ *   num_pairs            >= 0 (0 enqueues nothing).
+ *   error_flags          nullable device int; PA_DEVERR_COPY_PAIR on an id
+ *                        outside [0, num_blocks) (that pair is skipped).
+ * Pairs run concurrently, so no dst may equal another pair's src or dst
+ * (src == dst is a no-op); a mapping that breaks this has an unspecified
+ * result.  Returns PA_OK or a negative pa_status.
+ */
+int pa_copy_blocks(void* const* k_caches, void* const* v_caches,
+                   int num_layers, const int64_t* block_mapping, int num_pairs,
+                   int num_blocks, int block_size, int num_kv_heads,
+                   int head_size, int* error_flags, pa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_B200_PA_H */

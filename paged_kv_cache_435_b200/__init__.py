@@ -1,0 +1,22 @@
+"""Paged decode attention for NVIDIA B200 (sm_100a).
+
+The product is ``libpagedattn.so`` (C ABI in ``include/pa.h``) with three
+entry points, bound here under the same names:
+
+* ``pa_reshape_and_cache``: write each new token's K/V into its paged-cache
+  slot;
+* ``pa_decode_attention``: one-query-token-per-sequence attention over the
+  paged K/V pool through per-sequence block tables (GQA folded, split-KV for
+  long contexts);
+* ``pa_copy_blocks``: copy-on-write block copies.
+
+``inputs`` builds seeded synthetic workloads.  The library is loaded lazily on
+first use and its absence raises; nothing here computes on the CPU.
+"""
+from ._native import (  # noqa: F401
+    PA_DEVERR_BLOCK_ID, PA_DEVERR_CONTEXT_LEN, PA_DEVERR_COPY_PAIR,
+    PA_DEVERR_SLOT, PA_DEVERR_TIMEOUT, PA_ERR_CUDA, PA_ERR_INVALID_ARG,
+    PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_OK, PAError, library_path,
+    pa_copy_blocks, pa_decode_attention, pa_decode_partition_size,
+    pa_decode_workspace_size, pa_launch_count, pa_reshape_and_cache, raw,
+    status_string)

@@ -1,0 +1,244 @@
+// C ABI of libpagedattn.so: argument validation, the split-KV plan and the
+// dispatch to the kernels.  Every check here runs on the host before any
+// launch; a failed check enqueues nothing.
+#include <atomic>
+#include <cmath>
+#include <cstddef>
+#include <cstdint>
+
+#include "pa.h"
+#include "pa_cache_ops.cuh"
+#include "pa_common.cuh"
+#include "pa_decode.cuh"
+
+namespace pa {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+namespace {
+
+constexpr int kNumSMs = 148;           // B200
+constexpr int kAutoPartition = 512;    // tokens per partition when splitting
+constexpr int kMaxGridYZ = 65535;
+
+bool aligned16(const void* p) {
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+int round_up(int x, int m) { return ((x + m - 1) / m) * m; }
+
+bool decode_shape_supported(int num_heads, int num_kv_heads, int head_size,
+                            int block_size) {
+    const int G = num_heads / num_kv_heads;
+    return (head_size == 64 || head_size == 128) &&
+           (block_size == 16 || block_size == 32) && G >= 1 && G <= 8;
+}
+
+// Partition width in tokens (>= max_context_len means one partition).
+// Split only when (sequence, kv head) units alone cannot fill the GPU with a
+// few CTAs per SM; then 512-token partitions spread long contexts.
+int plan_partition(int num_seqs, int num_kv_heads, int block_size,
+                   int max_context_len, int partition_size) {
+    if (partition_size > 0) return partition_size;
+    const int whole = round_up(max_context_len > 0 ? max_context_len : 1,
+                               block_size);
+    if (max_context_len <= kAutoPartition) return whole;
+    const long long units = (long long)num_seqs * num_kv_heads;
+    if (units >= 4LL * kNumSMs) return whole;
+    int part = round_up(kAutoPartition, block_size);
+    while ((max_context_len + part - 1) / part > kMaxGridYZ) part *= 2;
+    return part;
+}
+
+int num_partitions(int max_context_len, int part) {
+    const int n = (max_context_len + part - 1) / part;
+    return n < 1 ? 1 : n;
+}
+
+size_t workspace_bytes_for(int num_seqs, int num_heads, int head_size,
+                           int max_partitions) {
+    if (max_partitions <= 1) return 0;
+    const size_t rows = (size_t)num_seqs * num_heads * max_partitions;
+    size_t bytes = rows * (size_t)head_size * 4;  // tmp_o
+    bytes = (bytes + 255) & ~(size_t)255;
+    bytes += ((rows * 4 + 255) & ~(size_t)255) * 2;  // tmp_m, tmp_l
+    return bytes;
+}
+
+}  // namespace
+}  // namespace pa
+
+extern "C" {
+
+const char* pa_status_string(int status) {
+    switch (status) {
+        case PA_OK: return "PA_OK";
+        case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
+        case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+        case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE";
+        case PA_ERR_CUDA: return "PA_ERR_CUDA";
+        default: return "PA_UNKNOWN_STATUS";
+    }
+}
+
+int pa_version(void) { return (1 << 16) | 0; }
+
+uint64_t pa_launch_count(void) {
+    return pa::g_launches.load(std::memory_order_relaxed);
+}
+
+int pa_reshape_and_cache(const void* key, const void* value,
+                         int64_t key_token_stride, int64_t value_token_stride,
+                         void* k_cache, void* v_cache,
+                         const int64_t* slot_mapping, int num_tokens,
+                         int num_blocks, int block_size, int num_kv_heads,
+                         int head_size, int* error_flags, pa_stream_t stream) {
+    if (num_tokens < 0 || num_blocks <= 0 || block_size <= 0 ||
+        num_kv_heads <= 0 || head_size <= 0)
+        return PA_ERR_INVALID_ARG;
+    const int64_t row = (int64_t)num_kv_heads * head_size;
+    if (key_token_stride < row || value_token_stride < row)
+        return PA_ERR_INVALID_ARG;
+    if (!k_cache || !v_cache) return PA_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PA_OK;
+    if (!key || !value || !slot_mapping) return PA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(key) | reinterpret_cast<uintptr_t>(value) |
+         reinterpret_cast<uintptr_t>(k_cache) |
+         reinterpret_cast<uintptr_t>(v_cache)) & 1u)
+        return PA_ERR_INVALID_ARG;  // bf16 needs 2-byte alignment
+    if ((reinterpret_cast<uintptr_t>(slot_mapping) & 7u) != 0)
+        return PA_ERR_INVALID_ARG;
+    cudaError_t e = pa::launch_reshape_and_cache(
+        key, value, key_token_stride, value_token_stride, k_cache, v_cache,
+        slot_mapping, num_tokens, num_blocks, block_size, num_kv_heads,
+        head_size, error_flags, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_decode_partition_size(int num_seqs, int num_heads, int num_kv_heads,
+                             int head_size, int block_size,
+                             int max_context_len, int partition_size) {
+    (void)num_heads;
+    (void)head_size;
+    if (num_seqs < 0 || num_kv_heads <= 0 || block_size <= 0 ||
+        max_context_len < 0 || partition_size < 0)
+        return PA_ERR_INVALID_ARG;
+    if (partition_size > 0 && partition_size % block_size != 0)
+        return PA_ERR_INVALID_ARG;
+    return pa::plan_partition(num_seqs, num_kv_heads, block_size,
+                              max_context_len, partition_size);
+}
+
+size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                int head_size, int block_size,
+                                int max_context_len, int partition_size) {
+    const int part = pa_decode_partition_size(num_seqs, num_heads, num_kv_heads,
+                                              head_size, block_size,
+                                              max_context_len, partition_size);
+    if (part <= 0 || num_heads <= 0 || head_size <= 0) return 0;
+    return pa::workspace_bytes_for(num_seqs, num_heads, head_size,
+                                   pa::num_partitions(max_context_len, part));
+}
+
+int pa_decode_attention(float* out, const void* q, const void* k_cache,
+                        const void* v_cache, const int32_t* block_tables,
+                        int max_blocks_per_seq, const int32_t* context_lens,
+                        int max_context_len, int num_seqs, int num_heads,
+                        int num_kv_heads, int head_size, int block_size,
+                        int num_blocks, float scale, int partition_size,
+                        void* workspace, size_t workspace_bytes,
+                        int* error_flags, pa_stream_t stream) {
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 ||
+        head_size <= 0 || block_size <= 0 || num_blocks <= 0 ||
+        max_blocks_per_seq <= 0 || max_context_len < 0 || partition_size < 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    if ((long long)max_context_len > (long long)max_blocks_per_seq * block_size)
+        return PA_ERR_INVALID_ARG;
+    if (partition_size > 0 && partition_size % block_size != 0)
+        return PA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+    if (!pa::decode_shape_supported(num_heads, num_kv_heads, head_size,
+                                       block_size))
+        return PA_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PA_OK;
+    if (num_seqs > pa::kMaxGridYZ) return PA_ERR_UNSUPPORTED;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+        return PA_ERR_INVALID_ARG;
+    if (!pa::aligned16(out) || !pa::aligned16(q) || !pa::aligned16(k_cache) ||
+        !pa::aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+        (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+        return PA_ERR_INVALID_ARG;
+
+    const int part = pa::plan_partition(num_seqs, num_kv_heads, block_size,
+                                        max_context_len, partition_size);
+    const int np = pa::num_partitions(max_context_len, part);
+    if (np > pa::kMaxGridYZ) return PA_ERR_INVALID_ARG;
+    const size_t need =
+        pa::workspace_bytes_for(num_seqs, num_heads, head_size, np);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need) return PA_ERR_WORKSPACE;
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+            return PA_ERR_INVALID_ARG;
+    }
+
+    pa::DecodeParams p{};
+    p.out = out;
+    p.q = static_cast<const uint16_t*>(q);
+    p.k_cache = static_cast<const uint16_t*>(k_cache);
+    p.v_cache = static_cast<const uint16_t*>(v_cache);
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    if (need > 0) {
+        const size_t rows = (size_t)num_seqs * num_heads * np;
+        unsigned char* ws = static_cast<unsigned char*>(workspace);
+        const size_t o_bytes = (rows * head_size * 4 + 255) & ~(size_t)255;
+        const size_t s_bytes = (rows * 4 + 255) & ~(size_t)255;
+        p.tmp_o = reinterpret_cast<float*>(ws);
+        p.tmp_m = reinterpret_cast<float*>(ws + o_bytes);
+        p.tmp_l = reinterpret_cast<float*>(ws + o_bytes + s_bytes);
+    }
+    p.error_flags = error_flags;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.max_context_len = max_context_len;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.num_blocks = num_blocks;
+    p.group = num_heads / num_kv_heads;
+    p.partition_size = part;
+    p.max_partitions = np;
+    p.scale_log2 = pa::log2e_scale(scale);
+    cudaError_t e = pa::launch_paged_decode(
+        p, num_seqs, head_size, block_size,
+        reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_copy_blocks(void* const* k_caches, void* const* v_caches,
+                   int num_layers, const int64_t* block_mapping, int num_pairs,
+                   int num_blocks, int block_size, int num_kv_heads,
+                   int head_size, int* error_flags, pa_stream_t stream) {
+    if (num_layers <= 0 || num_pairs < 0 || num_blocks <= 0 ||
+        block_size <= 0 || num_kv_heads <= 0 || head_size <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (!k_caches || !v_caches) return PA_ERR_INVALID_ARG;
+    for (int l = 0; l < num_layers; ++l) {
+        if (!k_caches[l] || !v_caches[l]) return PA_ERR_INVALID_ARG;
+        if (!pa::aligned16(k_caches[l]) || !pa::aligned16(v_caches[l]))
+            return PA_ERR_INVALID_ARG;
+    }
+    if (((long long)block_size * num_kv_heads * head_size * 2) % 16 != 0)
+        return PA_ERR_UNSUPPORTED;
+    if (num_pairs == 0) return PA_OK;
+    if (!block_mapping || (reinterpret_cast<uintptr_t>(block_mapping) & 7u))
+        return PA_ERR_INVALID_ARG;
+    cudaError_t e = pa::launch_copy_blocks(
+        k_caches, v_caches, num_layers, block_mapping, num_pairs, num_blocks,
+        block_size, num_kv_heads, head_size, error_flags,
+        reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,40 @@
+// Internal interface between the C ABI (pa_api.cu) and the decode kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace pa {
+
+struct DecodeParams {
+    float* out;                  // fp32 [B][Hq][D]
+    const uint16_t* q;           // bf16 [B][Hq][D]
+    const uint16_t* k_cache;     // bf16 [NB][bs][Hkv][D]
+    const uint16_t* v_cache;
+    const int32_t* block_tables; // int32 [B][max_blocks_per_seq]
+    const int32_t* context_lens; // int32 [B]
+    float* tmp_o;                // fp32 [B][Hq][max_partitions][D]
+    float* tmp_m;                // fp32 [B][Hq][max_partitions] (log2 domain)
+    float* tmp_l;                // fp32 [B][Hq][max_partitions]
+    int* error_flags;            // nullable
+    int max_blocks_per_seq;
+    int max_context_len;
+    int num_heads;
+    int num_kv_heads;
+    int num_blocks;
+    int group;                   // num_heads / num_kv_heads (1..8)
+    int partition_size;          // tokens, multiple of block_size
+    int max_partitions;          // ceil(max_context_len / partition_size)
+    float scale_log2;            // scale * log2(e)
+};
+
+// scale * log2(e): logits are kept in the log2 domain (exp2f).
+float log2e_scale(float scale);
+
+// Enqueue the partition kernel (and the merge kernel when
+// max_partitions > 1).  head_size in {64,128}, block_size in {16,32}.
+cudaError_t launch_paged_decode(const DecodeParams& p, int num_seqs,
+                                int head_size, int block_size,
+                                cudaStream_t stream);
+
+}  // namespace pa

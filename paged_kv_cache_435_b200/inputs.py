@@ -110,9 +110,12 @@ class DecodeCase:
     tables_np: np.ndarray        # int32 [B, MB] (host copy, after CoW remap)
     unique_tokens: int           # distinct (block, offset) positions read
     logical_tokens: int          # sum of context lengths
+    scale_override: Optional[float] = None
 
     @property
     def scale(self) -> float:
+        if self.scale_override is not None:
+            return self.scale_override
         return self.workload.scale
 
     @property
