@@ -250,21 +250,24 @@ def run_gpu(args):
     dist = init_dist(world, "nccl")
     pa.raw()  # fail loudly if the library is missing
 
-    case = inputs.make_case(args.workload, device=dev)
+    case = inputs.make_case(args.workload, device=dev, num_seqs=args.seqs)
     w = case.workload
     part = args.partition if args.partition is not None else w.partition_size
     step = Step(case, part)
     stream = torch.cuda.current_stream(dev)
 
     # in-run copy bandwidth (read + write bytes of a 1 GiB device copy)
-    a = torch.empty(1 << 29, dtype=torch.bfloat16, device=dev)
-    b = torch.empty_like(a)
-    copy_best = 0.0
-    for _ in range(6):
-        e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
-        e0.record(stream); b.copy_(a); e1.record(stream); e1.synchronize()
-        copy_best = max(copy_best, 2 * a.numel() * 2 / (e0.elapsed_time(e1) * 1e-3) / 1e9)
-    del a, b
+    copy_best = None
+    if not args.kernel_only:
+        a = torch.empty(1 << 29, dtype=torch.bfloat16, device=dev)
+        b = torch.empty_like(a)
+        copy_best = 0.0
+        for _ in range(6):
+            e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+            e0.record(stream); b.copy_(a); e1.record(stream); e1.synchronize()
+            copy_best = max(copy_best, 2 * a.numel() * 2 /
+                            (e0.elapsed_time(e1) * 1e-3) / 1e9)
+        del a, b
 
     for _ in range(args.warmup):
         step.cache_ops(); step.attention()
@@ -292,7 +295,7 @@ def run_gpu(args):
     flags = int(step.flags.item())
 
     # e2e: host buffers through the public API
-    e2e = run_e2e(case, step, args, dist, dev)
+    e2e = None if args.kernel_only else run_e2e(case, step, args, dist, dev)
 
     ms_total = max_over_ranks(dist, ms_total, dev)
     attn_ms_max = max_over_ranks(dist, attn_ms, dev)
@@ -306,7 +309,7 @@ def run_gpu(args):
 
     result = None
     if rank == 0:
-        cpu = cpu_baseline(args) if world == 1 else None
+        cpu = cpu_baseline(args) if world == 1 and not args.kernel_only else None
         clocks = clk.summary()
         result = {
             "metric": METRIC,
@@ -341,7 +344,7 @@ def run_gpu(args):
             "context_tokens_per_s": round(world * case.logical_tokens / (ms_step * 1e-3), 1),
             "pct_hbm_peak": round(100 * value / (world * peak), 2),
             "step_bytes": sb,
-            "in_run_copy_gbs": round(copy_best, 1),
+            "in_run_copy_gbs": None if copy_best is None else round(copy_best, 1),
             "roofline": {
                 "kernel": "paged_decode_kernel" + (" + reduce" if step.partition < case.max_context_len else ""),
                 "bound": "hbm",
@@ -350,7 +353,8 @@ def run_gpu(args):
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s",
                 "unit": "GB/s",
                 "frac": round(achieved / peak, 4),
-                "frac_of_in_run_copy": round(achieved / copy_best, 4),
+                "frac_of_in_run_copy": (None if copy_best is None
+                                        else round(achieved / copy_best, 4)),
                 "traffic": traffic,
                 "algorithmic_bytes_per_launch": ab,
                 "avg_launch_ms": round(attn_ms_max, 5),
@@ -524,6 +528,11 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--partition", type=int, default=None)
+    ap.add_argument("--seqs", type=int, default=None,
+                    help="keep only the first N sequences of the workload")
+    ap.add_argument("--kernel-only", action="store_true",
+                    help="time the device step only: no e2e leg, no in-run "
+                         "copy peak, no CPU baseline (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -262,14 +262,22 @@ def _finish(w: Workload, lens, tables, NB, pairs, device, vseed, pool_device,
     )
 
 
-def make_case(name: str, device="cpu", pool_device=None) -> DecodeCase:
-    """The named workload with its fixed seeds."""
+def make_case(name: str, device="cpu", pool_device=None,
+              num_seqs: Optional[int] = None) -> DecodeCase:
+    """The named workload with its fixed seeds.  ``num_seqs`` keeps only the
+    first sequences of its length draw (same shapes; a smaller case)."""
     w = WORKLOADS[name]
     if w.lengths == "shared":
+        if num_seqs is not None and num_seqs != w.num_seqs:
+            raise ValueError("the shared-prefix workload cannot be truncated")
         return build_shared_prefix_case(w, device=device,
                                         pool_device=pool_device)
     rng = np.random.default_rng(1000 + w.wid)
     lens = draw_lengths(w.lengths, w.num_seqs, rng)
+    if num_seqs is not None and num_seqs != w.num_seqs:
+        lens = lens[:num_seqs]
+        w = dataclasses.replace(w, num_seqs=len(lens),
+                                name=f"{w.name}_first{len(lens)}")
     return build_case(w, lens, device=device, pool_device=pool_device,
                       seed=None, rng=rng)
 
