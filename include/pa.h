@@ -177,6 +177,49 @@ int pa_decode_attention(float* out, const void* q, const void* k_cache,
                         void* workspace, size_t workspace_bytes,
                         int* error_flags, pa_stream_t stream);
 
+/* Capacity, in bytes, of the workspace built into the library for
+ * pa_decode_attention_static_ws (32 MiB per GPU that uses the library). */
+#define PA_STATIC_WORKSPACE_BYTES (32u << 20)
+
+/*
+ * pa_decode_attention_static_ws - pa_decode_attention for callers that cannot
+ * allocate device memory.  The pages have no counterpart of this call: it is
+ * an interface addition of this library.
+ *
+ * Some callers are given only their inputs and outputs and may not allocate
+ * on the device themselves (plugin hooks of inference runtimes, processes
+ * whose device memory another allocator reserved at start-up, C code without
+ * a device allocator).  This call takes the same arguments as
+ * pa_decode_attention minus the workspace, and uses as split-KV scratch a
+ * fixed array of PA_STATIC_WORKSPACE_BYTES compiled into the library (held on
+ * every GPU that uses the library until the process exits).  It never calls
+ * cudaMalloc, cudaFree or any allocating routine.
+ *
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - If pa_decode_workspace_size(...) for these arguments exceeds
+ *     PA_STATIC_WORKSPACE_BYTES the call returns PA_ERR_WORKSPACE and
+ *     enqueues nothing (use a larger partition_size, or pa_decode_attention
+ *     with your own workspace).
+ *   - Every call shares the one array, which keeps the last call's contents;
+ *     the kernels write each scratch value before reading it, so nothing needs
+ *     clearing.  Calls that overlap on the GPU (several streams, several host
+ *     threads) race on the array: serialise them.
+ * Other arguments, results and errors are those of pa_decode_attention.
+ */
+int pa_decode_attention_static_ws(float* out, const void* q,
+                                  const void* k_cache, const void* v_cache,
+                                  const int32_t* block_tables,
+                                  int max_blocks_per_seq,
+                                  const int32_t* context_lens,
+                                  int max_context_len, int num_seqs,
+                                  int num_heads, int num_kv_heads,
+                                  int head_size, int block_size,
+                                  int num_blocks, float scale,
+                                  int partition_size, int* error_flags,
+                                  pa_stream_t stream);
+
 /*
  * pa_copy_blocks - copy-on-write block copies ("Memory Sharing via
  * Copy-on-Write (CoW)": when sequences sharing a block diverge, only that

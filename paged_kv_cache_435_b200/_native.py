@@ -218,3 +218,39 @@ def pa_copy_blocks(k_caches: Sequence, v_caches: Sequence, block_mapping,
                               _ptr(block_mapping), block_mapping.shape[0], NB,
                               bs, Hkv, D, _ptr(error_flags), _stream(stream))
     return _check(rc, "pa_copy_blocks")
+
+
+def pa_decode_attention_static_ws(out, q, k_cache, v_cache, block_tables,
+                                  context_lens, max_context_len: int,
+                                  scale: float, partition_size: int = 0,
+                                  error_flags=None, stream=None) -> int:
+    """pa_decode_attention with the library's built-in workspace, for callers
+    that cannot allocate device memory (see include/pa.h)."""
+    import torch
+    lib = raw()
+    f = lib.pa_decode_attention_static_ws
+    p, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    f.argtypes = [p, p, p, p, p, i32, p, i32, i32, i32, i32, i32, i32, i32,
+                  f32, i32, p, p]
+    f.restype = i32
+    bf = torch.bfloat16
+    _cuda(out, "out", torch.float32, 3); _cuda(q, "q", bf, 3)
+    _cuda(k_cache, "k_cache", bf, 4); _cuda(v_cache, "v_cache", bf, 4)
+    _cuda(block_tables, "block_tables", torch.int32, 2)
+    _cuda(context_lens, "context_lens", torch.int32, 1)
+    for name, t in (("out", out), ("q", q), ("k_cache", k_cache),
+                    ("v_cache", v_cache), ("block_tables", block_tables),
+                    ("context_lens", context_lens)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    B, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_cache.shape
+    if out.shape != q.shape or D2 != D or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch between q, out and the pools")
+    if block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise ValueError("block_tables / context_lens must have B rows")
+    rc = f(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+           block_tables.shape[1], _ptr(context_lens), int(max_context_len), B,
+           Hq, Hkv, D, bs, NB, float(scale), int(partition_size),
+           _ptr(error_flags), _stream(stream))
+    return _check(rc, "pa_decode_attention_static_ws")
