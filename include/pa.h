@@ -50,9 +50,10 @@
  *     or skipped, the affected outputs are unspecified, and the matching
  *     PA_DEVERR_* bit is OR-ed into *error_flags when error_flags is non-NULL
  *     (a device int the caller zeroes and reads after the stream completes).
- *   - Supported now: head_size in {64, 128}; block_size in {16, 32};
- *     num_heads / num_kv_heads in 1..8.  Other values return
- *     PA_ERR_UNSUPPORTED.
+ *   - pa_decode_attention supports head_size in {64, 128}, block_size in
+ *     {16, 32}, num_heads / num_kv_heads in 1..8 and
+ *     num_blocks * block_size < 2^31; other values return PA_ERR_UNSUPPORTED.
+ *     The cache ops accept any positive sizes.
  */
 #ifndef PAGEDATTN_B200_PA_H
 #define PAGEDATTN_B200_PA_H
@@ -81,6 +82,7 @@ typedef enum {
 #define PA_DEVERR_SLOT 0x4        /* slot_mapping entry >= num_blocks*block_size */
 #define PA_DEVERR_COPY_PAIR 0x8   /* block_mapping id outside [0,num_blocks) */
 #define PA_DEVERR_TIMEOUT 0x10    /* an async-copy wait exceeded its time limit */
+#define PA_DEVERR_INTERNAL 0x20   /* shared memory not 1024-byte aligned (no work done) */
 
 /* Human-readable name of a pa_status value (static string, never NULL). */
 const char* pa_status_string(int status);

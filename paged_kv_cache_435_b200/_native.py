@@ -26,6 +26,7 @@ PA_DEVERR_CONTEXT_LEN = 0x2
 PA_DEVERR_SLOT = 0x4
 PA_DEVERR_COPY_PAIR = 0x8
 PA_DEVERR_TIMEOUT = 0x10
+PA_DEVERR_INTERNAL = 0x20
 
 _lock = threading.Lock()
 _lib = None

@@ -162,6 +162,8 @@ int pa_decode_attention(float* out, const void* q, const void* k_cache,
     if (!pa::decode_shape_supported(num_heads, num_kv_heads, head_size,
                                        block_size))
         return PA_ERR_UNSUPPORTED;
+    if ((long long)num_blocks * block_size > 0x7fffffffLL)
+        return PA_ERR_UNSUPPORTED;  // token slots are 32-bit TMA coordinates
     if (num_seqs == 0) return PA_OK;
     if (num_seqs > pa::kMaxGridYZ) return PA_ERR_UNSUPPORTED;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
@@ -201,6 +203,7 @@ int pa_decode_attention(float* out, const void* q, const void* k_cache,
         p.tmp_l = reinterpret_cast<float*>(ws + o_bytes + s_bytes);
     }
     p.error_flags = error_flags;
+    p.num_seqs = num_seqs;
     p.max_blocks_per_seq = max_blocks_per_seq;
     p.max_context_len = max_context_len;
     p.num_heads = num_heads;
@@ -211,8 +214,7 @@ int pa_decode_attention(float* out, const void* q, const void* k_cache,
     p.max_partitions = np;
     p.scale_log2 = pa::log2e_scale(scale);
     cudaError_t e = pa::launch_paged_decode(
-        p, num_seqs, head_size, block_size,
-        reinterpret_cast<cudaStream_t>(stream));
+        p, head_size, block_size, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

@@ -9,25 +9,35 @@
 // Operations" and "The Roofline Model"), so the design goal is to read every
 // needed KV byte exactly once at close to HBM speed.
 //
-// Kernel structure (one CTA per (kv head, KV partition, sequence)):
-//  * 4 warps; warp w owns 16-token chunks w, w+4, w+8, ... of the partition
-//    and runs its own ring of shared-memory stages, each guarded by an
-//    mbarrier with a transaction count.  A chunk is 16 K rows + 16 V rows of
-//    head_size bf16 each; every lane issues one bulk asynchronous copy
-//    (cp.async.bulk, executed by the TMA unit) per row, so one warp
-//    instruction puts a whole chunk in flight.  Rows land at a padded stride
-//    (head_size*2 + 16 bytes) so ldmatrix reads are bank-conflict free.
-//  * All G = num_heads/num_kv_heads query heads of the kv head are folded
-//    into one pass: S = Q K^T and O += P V run on the bf16 tensor cores with
-//    mma.m16n8k16, rows 0..7 of the 16-row M tile holding the G heads.  The
-//    spare rows 8..15 carry the low-order bf16 part of P (P = P_hi + P_lo),
-//    so the PV product keeps ~16 bits of P instead of bf16's 8.
-//  * fp32 online softmax in the log2 domain (exp2f), per-warp running max
-//    and sum; the warps merge through shared memory at the end.
-//  * Contexts longer than the partition are split; each partition writes its
-//    max, sum and normalised output, and pa_decode_reduce_kernel merges them.
+// Work unit ("item"): one (sequence, KV partition) for one kv head.  A CTA of
+// 4 warps processes items; warp w owns 16-token chunks w, w+4, w+8, ... of
+// each item.
+//  * Loads: every warp runs its own ring of shared-memory stages guarded by
+//    mbarriers with transaction counts.  Lane 0 fills a stage with 2 * D/64
+//    TMA tensor copies (cp.async.bulk.tensor, 128-byte swizzle): 16 rows of
+//    K and of V for this kv head, 8 KB at D=128.  The producer side of the
+//    ring runs ahead across item boundaries, so copies stay in flight while
+//    an item is being merged.  Block ids for the next 32 chunks are
+//    prefetched into one register per lane.
+//  * Math: the G = num_heads/num_kv_heads query heads of the kv head share the
+//    pass.  S = Q K^T and O += P V run on the bf16 tensor cores with
+//    mma.m16n8k16: rows 0..7 of the 16-row M tile hold the G heads, and the
+//    spare rows 8..15 carry the low-order bf16 part of P (P = P_hi + P_lo), so
+//    the PV product keeps ~16 bits of P.  fp32 online softmax in the log2
+//    domain; O is rescaled only when a row's running max grows.
+//  * Item end: warps 1..3 post (max, sum, O) to shared memory and continue;
+//    warp 0 merges and writes either the output or, when the sequence is
+//    split, the partition's (max, sum, normalised O) for the merge kernel.
+//  * Grids: without a split, one CTA per (kv head, sequence) item, scheduled
+//    by the hardware.  With a split, a persistent grid of ~2 CTAs per SM; each
+//    CTA builds the prefix sum of partitions per sequence in shared memory
+//    and walks a compact item list, so no CTA is spent on partitions past a
+//    sequence's end.
+#include <cuda.h>
+
 #include <cfloat>
 #include <cstdint>
+#include <mutex>
 
 #include "pa_common.cuh"
 #include "pa_decode.cuh"
@@ -37,58 +47,165 @@ namespace {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
-constexpr int kChunk = 16;  // tokens per pipeline stage (one M/K tile)
+constexpr int kChunk = 16;          // tokens per pipeline stage
 constexpr int kMaxGroup = 8;
+constexpr int kMaxPersistSeqs = 768;
+constexpr int kTargetCtasPerSM = 2;
+constexpr int kNumSMs = 148;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct Cfg {
-    static constexpr int kRowBytes = D * 2 + 16;
-    static constexpr int kStageBytes = 2 * kChunk * kRowBytes;
-    static constexpr int kStagesRaw = 26112 / kStageBytes;
-    static constexpr int kStages = kStagesRaw < 2 ? 2 : kStagesRaw;
-    static constexpr int kBarBytes = (kWarps * kStages * 8 + 127) / 128 * 128;
+    static constexpr int kHalves = D / 64;                  // 128-byte column tiles
+    static constexpr int kHalfBytes = kChunk * 128;         // 16 rows x 128 B
+    static constexpr int kKVBytes = kHalves * kHalfBytes;   // K (or V) of a chunk
+    static constexpr int kStageBytes = 2 * kKVBytes;
+    static constexpr int kStages = D == 128 ? 3 : 5;
     static constexpr int kRingBytes = kWarps * kStages * kStageBytes;
-    static constexpr int kMergeBytes = kWarps * kMaxGroup * (D + 2) * 4;
-    static constexpr int kSmemBytes =
-        kBarBytes + (kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes);
-    static_assert(kWarps * kStages * 8 <= kBarBytes, "barrier area");
+    static constexpr int kRedStride = D + 8;                // floats per row
+    static constexpr int kRedOBytes = (kWarps - 1) * kMaxGroup * kRedStride * 4;
+    static constexpr int kRedMLBytes = kWarps * kMaxGroup * 2 * 4;
+    static constexpr int kRedOff = kRingBytes;
+    static constexpr int kBarOff = kRedOff + kRedOBytes + kRedMLBytes;
+    static constexpr int kBarBytes = (kWarps * kStages * 8 + 127) / 128 * 128;
+    static constexpr int kPrefixOff = kBarOff + kBarBytes;
+    static constexpr int kSmemGrid = kPrefixOff;
+    static constexpr int kSmemPersist = kPrefixOff + (kMaxPersistSeqs + 1) * 4;
+    static_assert(kRingBytes % 1024 == 0, "ring tiles must stay 1024-aligned");
+    static_assert(kSmemPersist + 1024 <= 232448 / kTargetCtasPerSM,
+                  "two CTAs per SM must fit");
 };
 
-template <int D, int BS>
-__global__ void __launch_bounds__(kThreads, 2)
-paged_decode_kernel(const DecodeParams p) {
-    using C = Cfg<D>;
-    extern __shared__ __align__(128) unsigned char smem[];
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-    unsigned char* ring = smem + C::kBarBytes;
+struct Item {
+    int s;       // sequence; -1 = no item
+    int part;    // partition index
+    int L;       // context length (clamped)
+    int tok0;    // first token of the partition
+    int tok1;    // one past its last token
+    int nparts;  // partitions of this sequence
+};
 
-    const int g = blockIdx.x;     // kv head
-    const int part = blockIdx.y;  // KV partition
-    const int s = blockIdx.z;     // sequence
+__device__ __forceinline__ int clamped_len(const DecodeParams& p, int s) {
+    int L = p.context_lens[s];
+    if (L < 0 || L > p.max_context_len) {
+        if ((threadIdx.x & 31) == 0) report(p.error_flags, PA_DEVERR_CONTEXT_LEN);
+        L = L < 0 ? 0 : p.max_context_len;
+    }
+    return L;
+}
+
+__device__ __forceinline__ int parts_of(int L, int P) {
+    return L <= 0 ? 1 : (L + P - 1) / P;  // an empty context still owns one item
+}
+
+// Item k of this CTA (k = 0, 1, ...).
+template <bool kPersist>
+__device__ __forceinline__ Item get_item(const DecodeParams& p,
+                                         const int* prefix, int k) {
+    Item it;
+    it.s = -1;
+    int s, part;
+    if (kPersist) {
+        const int j = blockIdx.y + k * gridDim.y;
+        if (j >= prefix[p.num_seqs]) return it;
+        int lo = 0, hi = p.num_seqs - 1;  // largest s with prefix[s] <= j
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (prefix[mid] <= j) lo = mid; else hi = mid - 1;
+        }
+        s = lo;
+        part = j - prefix[s];
+    } else {
+        if (k > 0) return it;
+        s = blockIdx.z;
+        part = blockIdx.y;
+    }
+    const int L = clamped_len(p, s);
+    const int np = parts_of(L, p.partition_size);
+    if (part >= np) return it;
+    it.s = s;
+    it.part = part;
+    it.L = L;
+    it.nparts = np;
+    it.tok0 = part * p.partition_size;
+    it.tok1 = min(L, it.tok0 + p.partition_size);
+    return it;
+}
+
+// Chunks of `it` that warp w owns.
+__device__ __forceinline__ int warp_chunks(const Item& it, int warp) {
+    if (it.s < 0) return 0;
+    const int n = (it.tok1 - it.tok0 + kChunk - 1) / kChunk;
+    return n > warp ? (n - warp + kWarps - 1) / kWarps : 0;
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map,
+                                            int c0, int c1, int c2,
+                                            uint64_t* bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::"
+        "complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2),
+        "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kThreads) : "memory");
+}
+__device__ __forceinline__ void named_bar_arrive(int id) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(kThreads) : "memory");
+}
+
+template <int D, int BS, bool kPersist>
+__global__ void __launch_bounds__(kThreads, kTargetCtasPerSM)
+paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const DecodeParams p) {
+    using C = Cfg<D>;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    unsigned char* ring = smem;
+    float* red_o = reinterpret_cast<float*>(smem + C::kRedOff);
+    float* red_m = red_o + (kWarps - 1) * kMaxGroup * C::kRedStride;
+    float* red_l = red_m + kWarps * kMaxGroup;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+    int* prefix = reinterpret_cast<int*>(smem + C::kPrefixOff);
+
+    const int g = blockIdx.x;  // kv head
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int G = p.group;
     const int Hq = p.num_heads;
 
-    int L = p.context_lens[s];
-    if (L < 0 || L > p.max_context_len) {
-        if (threadIdx.x == 0 && g == 0 && part == 0)
-            report(p.error_flags, PA_DEVERR_CONTEXT_LEN);
-        L = L < 0 ? 0 : p.max_context_len;
-    }
-    const int tok0 = part * p.partition_size;
-    if (L == 0) {  // empty context: zeros, written once per (seq, kv head)
-        if (part == 0)
-            for (int i = threadIdx.x; i < G * D; i += kThreads)
-                p.out[((int64_t)s * Hq + g * G + i / D) * D + i % D] = 0.f;
+    // The 128-byte swizzle of the TMA tiles is tied to 1024-byte alignment.
+    if (smem_u32(ring) & 1023u) {
+        if (threadIdx.x == 0) report(p.error_flags, PA_DEVERR_INTERNAL);
         return;
     }
-    if (tok0 >= L) return;  // partition past this sequence's end
-    const int num_parts = (L + p.partition_size - 1) / p.partition_size;
-    const int tok1 = min(L, tok0 + p.partition_size);
-    const int nchunks = (tok1 - tok0 + kChunk - 1) / kChunk;
-    const int my_n = nchunks > warp ? (nchunks - warp + kWarps - 1) / kWarps : 0;
+
+    if (kPersist) {
+        // prefix[s] = partitions of sequences 0..s-1 (block-wide scan).  The
+        // merge area is free until the first item ends; it holds the warp sums.
+        int* warp_tot = reinterpret_cast<int*>(red_l);
+        int running = 0;
+        if (threadIdx.x == 0) prefix[0] = 0;
+        for (int base = 0; base < p.num_seqs; base += kThreads) {
+            const int s = base + threadIdx.x;
+            int v = s < p.num_seqs ? parts_of(clamped_len(p, s), p.partition_size) : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += t;
+            }
+            if (lane == 31) warp_tot[warp] = v;
+            __syncthreads();
+            int before = running;
+            for (int w = 0; w < warp; ++w) before += warp_tot[w];
+            if (s < p.num_seqs) prefix[s + 1] = before + v;
+            for (int w = 0; w < kWarps; ++w) running += warp_tot[w];
+            __syncthreads();
+        }
+    }
 
     uint64_t* my_bars = bars + warp * C::kStages;
     unsigned char* my_ring = ring + warp * C::kStages * C::kStageBytes;
@@ -96,217 +213,290 @@ paged_decode_kernel(const DecodeParams p) {
         for (int i = 0; i < C::kStages; ++i) mbar_init(&my_bars[i], 1);
         mbar_init_fence();
     }
-    __syncwarp();
+    __syncthreads();  // barriers initialised, prefix visible
 
-    // Q fragments (A operand, rows = heads of the group, rows >= G zero).
+    // Q fragments (A operand): rows = heads of the group, rows >= G zero.
+    // Reloaded per item because items of a persistent CTA differ in sequence.
     const int qr = lane >> 2;       // fragment row owned by this lane
     const int qc = (lane & 3) * 2;  // fragment column pair
-    uint32_t qa[D / 16][2];
-    {
-        const bool live = qr < G;
-        const uint16_t* qp = p.q + ((int64_t)s * Hq + g * G + (live ? qr : 0)) * D;
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-            qa[ks][0] = live ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + qc) : 0u;
-            qa[ks][1] = live ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8 + qc) : 0u;
-        }
-    }
+    const int xr = lane & 7;        // swizzle phase of this lane's ldmatrix row
+    const int mi = lane >> 3;       // ldmatrix sub-matrix this lane addresses
 
     const uint64_t pol = l2_policy_evict_first();
-    const int64_t tok_stride = (int64_t)p.num_kv_heads * D;  // elements
-    const uint16_t* kbase = p.k_cache + (int64_t)g * D;
-    const uint16_t* vbase = p.v_cache + (int64_t)g * D;
-    const int32_t* bt = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
+    const int32_t* tables = p.block_tables;
+    const float sl2 = p.scale_log2;
 
-    // Lane j keeps the physical block of this warp's chunk (32*k + j).
-    int ids = 0;
-    auto load_ids = [&](int j0) {
-        const int j = j0 + lane;
-        int id = 0;
-        if (j < my_n) {
-            const int ctok = tok0 + (warp + kWarps * j) * kChunk;
-            id = bt[ctok / BS];
+    // ---------------- producer state (this warp's chunk stream) ----------
+    int prod_k = 0;        // item of the next chunk to look up
+    int prod_i = 0;        // warp-chunk index within that item
+    int prod_count = 0;    // chunks issued so far
+    int ids_base = 0;      // prod_count at the last refill
+    int ids = -1;          // lane l: slot coordinate of chunk ids_base + l
+    bool prod_done = false;
+
+    // Lane l finds the (ids_base + l)-th chunk of the stream and its slot.
+    auto refill = [&]() {
+        int k = prod_k, i = prod_i, n = lane;
+        Item it = get_item<kPersist>(p, prefix, k);
+        for (;;) {
+            if (it.s < 0) break;
+            const int rem = warp_chunks(it, warp) - i;
+            if (rem > n) break;
+            n -= rem > 0 ? rem : 0;
+            ++k;
+            i = 0;
+            it = get_item<kPersist>(p, prefix, k);
+        }
+        int slot = -1;
+        if (it.s >= 0) {
+            i += n;
+            const int ctok = it.tok0 + (warp + kWarps * i) * kChunk;
+            int id = tables[(int64_t)it.s * p.max_blocks_per_seq + ctok / BS];
             if (id < 0 || id >= p.num_blocks) {
                 report(p.error_flags, PA_DEVERR_BLOCK_ID);
                 id = 0;
             }
+            slot = id * BS + ctok % BS;
+            ++i;  // position after this lane's chunk
         }
-        ids = id;
+        ids = slot;
+        ids_base = prod_count;
+        prod_k = __shfl_sync(0xffffffffu, k, 31);
+        prod_i = __shfl_sync(0xffffffffu, i, 31);
+        prod_done = __shfl_sync(0xffffffffu, slot, 31) < 0;
     };
 
-    // Put chunk j of this warp in flight (warp-uniform call).
-    auto issue = [&](int j) {
-        if ((j & 31) == 0) load_ids(j);
-        const int phys = __shfl_sync(0xffffffffu, ids, j & 31);
-        const int ctok = tok0 + (warp + kWarps * j) * kChunk;  // first token
-        const int valid = min(kChunk, tok1 - ctok);
-        const int off = ctok % BS;                             // row in block
-        unsigned char* st = my_ring + (j % C::kStages) * C::kStageBytes;
-        uint64_t* bar = &my_bars[j % C::kStages];
+    // Issue the next chunk of the stream into its stage; false when none.
+    auto issue = [&]() -> bool {
+        if (prod_count == ids_base + 32 || prod_count == 0) {
+            if (prod_count == 0 || !prod_done) refill();
+        }
+        const int slot = __shfl_sync(0xffffffffu, ids, (prod_count - ids_base) & 31);
+        if (slot < 0 || prod_count - ids_base >= 32) return false;
+        const int stage = prod_count % C::kStages;
+        const uint32_t dst = smem_u32(my_ring + stage * C::kStageBytes);
+        uint64_t* bar = &my_bars[stage];
         fence_proxy_async_smem();
-        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(2 * valid * D * 2));
         __syncwarp();
-        const bool is_v = lane >= kChunk;
-        const int t = lane & (kChunk - 1);
-        unsigned char* dst = st + lane * C::kRowBytes;
-        if (t < valid) {
-            const uint16_t* src = (is_v ? vbase : kbase) +
-                                  ((int64_t)phys * BS + off + t) * tok_stride;
-            bulk_g2s(dst, src, D * 2, bar, pol);
-        } else if (is_v) {
-            // Rows past the context: V must be finite (P is 0 there).
-            uint4* z = reinterpret_cast<uint4*>(dst);
+        if (lane == 0) {
+            mbar_arrive_expect_tx(bar, C::kStageBytes);
 #pragma unroll
-            for (int c = 0; c < D * 2 / 16; ++c) z[c] = make_uint4(0, 0, 0, 0);
+            for (int h = 0; h < C::kHalves; ++h) {
+                tma_load_3d(dst + h * C::kHalfBytes, &tm_k, 0, g * C::kHalves + h,
+                            slot, bar, pol);
+                tma_load_3d(dst + C::kKVBytes + h * C::kHalfBytes, &tm_v, 0,
+                            g * C::kHalves + h, slot, bar, pol);
+            }
         }
-        __syncwarp();
+        ++prod_count;
+        return true;
     };
 
-    float o[D / 8][4];
-#pragma unroll
-    for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-    float m_run = -INFINITY;  // running max of scaled logits (log2 domain)
-    float l_run = 0.f;        // this lane's share of the running sum
-    const float sl2 = p.scale_log2;
+    for (int j = 0; j < C::kStages; ++j)
+        if (!issue()) break;
 
-    const int pre = my_n < C::kStages ? my_n : C::kStages;
-    for (int j = 0; j < pre; ++j) issue(j);
-
-    int consumed = 0;
+    // ---------------- consumer ----------------
+    int cons_count = 0;
     bool aborted = false;
-    for (int j = 0; j < my_n; ++j) {
-        const int stage = j % C::kStages;
-        const bool ok = mbar_wait_bounded(&my_bars[stage], (j / C::kStages) & 1);
-        if (!__all_sync(0xffffffffu, ok)) {
-            aborted = true;
-            break;
-        }
-        consumed = j + 1;
-        const int ctok = tok0 + (warp + kWarps * j) * kChunk;
-        const uint32_t kaddr = smem_u32(my_ring + stage * C::kStageBytes);
-        const uint32_t vaddr = kaddr + kChunk * C::kRowBytes;
+    int drain_from = 0;  // first chunk whose wait gave up
+    int k = 0;
+    for (;; ++k) {
+        const Item it = get_item<kPersist>(p, prefix, k);
+        if (it.s < 0) break;
+        const int my_n = warp_chunks(it, warp);
 
-        // S (16 rows x 16 tokens) = Q K^T, as two n8 tiles of tokens.
-        float sacc[2][4];
+        uint32_t qa[D / 16][2];
+        {
+            const bool live = qr < G && it.L > 0;
+            const uint16_t* qp =
+                p.q + ((int64_t)it.s * Hq + g * G + (qr < G ? qr : 0)) * D;
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
-            const uint32_t row = kaddr + (nt * 8 + (lane & 7)) * C::kRowBytes +
-                                 (lane >> 3) * 16;
+            for (int ks = 0; ks < D / 16; ++ks) {
+                qa[ks][0] = live ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + qc) : 0u;
+                qa[ks][1] = live ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8 + qc) : 0u;
+            }
+        }
+
+        float o[D / 8][4];
 #pragma unroll
-            for (int kk = 0; kk < D / 32; ++kk) {
+        for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+        float m_run = -INFINITY;
+        float l_run = 0.f;
+
+        for (int i = 0; i < my_n; ++i) {
+            const int stage = cons_count % C::kStages;
+            if (!aborted) {
+                const bool ok = mbar_wait_bounded(&my_bars[stage],
+                                                  (cons_count / C::kStages) & 1);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    aborted = true;
+                    drain_from = cons_count;
+                    if (lane == 0) report(p.error_flags, PA_DEVERR_TIMEOUT);
+                }
+            }
+            ++cons_count;
+            if (aborted) continue;
+
+            const int ctok = it.tok0 + (warp + kWarps * i) * kChunk;
+            const int valid = min(kChunk, it.tok1 - ctok);
+            const uint32_t kaddr = smem_u32(my_ring + stage * C::kStageBytes);
+            const uint32_t vaddr = kaddr + C::kKVBytes;
+
+            if (valid < kChunk) {
+                // Rows past the context hold whatever the block holds; V must
+                // be finite there because P is zero.
+                const int rows = kChunk - valid;
+                for (int e = lane; e < rows * C::kHalves * 8; e += 32) {
+                    const int r = valid + e / (C::kHalves * 8);
+                    const int h = (e / 8) % C::kHalves;
+                    const int c = e & 7;
+                    const uint32_t a = vaddr + h * C::kHalfBytes + r * 128 + c * 16;
+                    asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(a), "r"(0)
+                                 : "memory");
+                }
+                __syncwarp();
+            }
+
+            // S (16 rows x 16 tokens) = Q K^T: two n8 tiles, two k chains each.
+            float sacc[2][2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+                for (int ch = 0; ch < 2; ++ch)
+                    sacc[nt][ch][0] = sacc[nt][ch][1] = sacc[nt][ch][2] = sacc[nt][ch][3] = 0.f;
+                const uint32_t row = kaddr + (nt * 8 + xr) * 128;
+#pragma unroll
+                for (int kk = 0; kk < D / 32; ++kk) {
+                    const int cidx = ((kk & 1) << 2) + mi;
+                    const uint32_t a = row + (kk >> 1) * C::kHalfBytes + ((cidx ^ xr) << 4);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(b0, b1, b2, b3, a);
+                    mma_bf16_16816(sacc[nt][kk & 1], qa[2 * kk][0], 0u, qa[2 * kk][1], 0u, b0, b1);
+                    mma_bf16_16816(sacc[nt][kk & 1], qa[2 * kk + 1][0], 0u, qa[2 * kk + 1][1], 0u, b2, b3);
+                }
+            }
+
+            float sv[4];
+            if (valid == kChunk) {
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e)
+                        sv[nt * 2 + e] = (sacc[nt][0][e] + sacc[nt][1][e]) * sl2;
+            } else {
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e)
+                        sv[nt * 2 + e] = (nt * 8 + qc + e < valid)
+                                             ? (sacc[nt][0][e] + sacc[nt][1][e]) * sl2
+                                             : -INFINITY;
+            }
+            float mx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            if (__any_sync(0xffffffffu, mx > m_run)) {
+                const float m_new = fmaxf(m_run, mx);
+                const float alpha = exp2f(m_run - m_new);
+                m_run = m_new;
+                l_run *= alpha;
+#pragma unroll
+                for (int j2 = 0; j2 < D / 8; ++j2) {
+                    o[j2][0] *= alpha; o[j2][1] *= alpha;
+                    o[j2][2] *= alpha; o[j2][3] *= alpha;
+                }
+            }
+            float pv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) pv[e] = exp2f(sv[e] - m_run);
+            l_run += (pv[0] + pv[1]) + (pv[2] + pv[3]);
+
+            // P as the A operand: rows 0..7 = bf16(P), rows 8..15 = bf16(P - bf16(P)).
+            const float h0 = bf16_round(pv[0]), h1 = bf16_round(pv[1]);
+            const float h2 = bf16_round(pv[2]), h3 = bf16_round(pv[3]);
+            const uint32_t a0 = pack_bf16x2(h0, h1);
+            const uint32_t a2 = pack_bf16x2(h2, h3);
+            const uint32_t a1 = pack_bf16x2(pv[0] - h0, pv[1] - h1);
+            const uint32_t a3 = pack_bf16x2(pv[2] - h2, pv[3] - h3);
+
+            // O (16 x D) += P (16 x 16 tokens) V (16 tokens x D).
+            const uint32_t vrow = vaddr + (((mi & 1) << 3) + xr) * 128;
+#pragma unroll
+            for (int dp = 0; dp < D / 16; ++dp) {
+                const int cidx = ((dp & 3) << 1) + (mi >> 1);
+                const uint32_t a = vrow + (dp >> 2) * C::kHalfBytes + ((cidx ^ xr) << 4);
                 uint32_t b0, b1, b2, b3;
-                ldsm_x4(b0, b1, b2, b3, row + kk * 64);
-                mma_bf16_16816(sacc[nt], qa[2 * kk][0], 0u, qa[2 * kk][1], 0u, b0, b1);
-                mma_bf16_16816(sacc[nt], qa[2 * kk + 1][0], 0u, qa[2 * kk + 1][1], 0u, b2, b3);
+                ldsm_x4_trans(b0, b1, b2, b3, a);
+                mma_bf16_16816(o[2 * dp], a0, a1, a2, a3, b0, b1);
+                mma_bf16_16816(o[2 * dp + 1], a0, a1, a2, a3, b2, b3);
             }
+            __syncwarp();
+            if (!prod_done || prod_count < ids_base + 32) issue();
         }
 
-        // Online softmax over this chunk for row qr (quad = 16 tokens).
-        float sv[4];
+        // ---------------- item end: merge the four warps ----------------
+        l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+        l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+        if (warp != 0) {
+            if (k > 0) named_bar_sync(2);  // warp 0 has read the previous item
+            float* dst = red_o + ((warp - 1) * kMaxGroup + qr) * C::kRedStride + qc;
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int tok = ctok + nt * 8 + qc + e;
-                sv[nt * 2 + e] = tok < tok1 ? sacc[nt][e] * sl2 : -INFINITY;
+            for (int j = 0; j < D / 8; ++j)
+                *reinterpret_cast<float2*>(dst + 8 * j) =
+                    make_float2(o[j][0] + o[j][2], o[j][1] + o[j][3]);
+            if ((lane & 3) == 0) {
+                red_m[warp * kMaxGroup + qr] = m_run;
+                red_l[warp * kMaxGroup + qr] = l_run;
             }
-        float mx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float m_new = fmaxf(m_run, mx);
-        const float alpha = exp2f(m_run - m_new);
-        m_run = m_new;
-        float pv[4];
+            named_bar_arrive(1);
+        } else {
+            named_bar_sync(1);
+            float sc[kWarps], M = m_run;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) pv[e] = exp2f(sv[e] - m_new);
-        l_run = l_run * alpha + ((pv[0] + pv[1]) + (pv[2] + pv[3]));
+            for (int w = 1; w < kWarps; ++w) M = fmaxf(M, red_m[w * kMaxGroup + qr]);
+            float den = 0.f;
 #pragma unroll
-        for (int j2 = 0; j2 < D / 8; ++j2) {
-            o[j2][0] *= alpha; o[j2][1] *= alpha;
-            o[j2][2] *= alpha; o[j2][3] *= alpha;
+            for (int w = 0; w < kWarps; ++w) {
+                const float mw = w == 0 ? m_run : red_m[w * kMaxGroup + qr];
+                const float lw = w == 0 ? l_run : red_l[w * kMaxGroup + qr];
+                sc[w] = mw == -INFINITY ? 0.f : exp2f(mw - M);
+                den += sc[w] * lw;
+            }
+            if (qr < G) {
+                const int h = g * G + qr;
+                const bool direct = it.nparts == 1;
+                const int64_t row = (int64_t)it.s * Hq + h;
+                const int64_t idx = row * p.max_partitions + it.part;
+                float* dst = direct ? p.out + row * D : p.tmp_o + idx * D;
+#pragma unroll
+                for (int j = 0; j < D / 8; ++j) {
+                    float v[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        float acc = sc[0] * (o[j][e] + o[j][e + 2]);
+#pragma unroll
+                        for (int w = 1; w < kWarps; ++w)
+                            acc += sc[w] * red_o[((w - 1) * kMaxGroup + qr) * C::kRedStride + 8 * j + qc + e];
+                        v[e] = it.L > 0 ? acc / den : 0.f;
+                    }
+                    *reinterpret_cast<float2*>(dst + 8 * j + qc) = make_float2(v[0], v[1]);
+                }
+                if (!direct && (lane & 3) == 0) {
+                    p.tmp_m[idx] = M;
+                    p.tmp_l[idx] = den;
+                }
+            }
+            named_bar_arrive(2);
         }
-
-        // P as the A operand: rows 0..7 = bf16(P), rows 8..15 = bf16(P - bf16(P)).
-        const float h0 = bf16_round(pv[0]), h1 = bf16_round(pv[1]);
-        const float h2 = bf16_round(pv[2]), h3 = bf16_round(pv[3]);
-        const uint32_t a0 = pack_bf16x2(h0, h1);
-        const uint32_t a2 = pack_bf16x2(h2, h3);
-        const uint32_t a1 = pack_bf16x2(pv[0] - h0, pv[1] - h1);
-        const uint32_t a3 = pack_bf16x2(pv[2] - h2, pv[3] - h3);
-
-        // O (16 x D) += P (16 x 16 tokens) V (16 tokens x D).
-        const uint32_t vrow = vaddr +
-                              ((lane & 7) + ((lane >> 3) & 1) * 8) * C::kRowBytes +
-                              (lane >> 4) * 16;
-#pragma unroll
-        for (int dp = 0; dp < D / 16; ++dp) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_trans(b0, b1, b2, b3, vrow + dp * 32);
-            mma_bf16_16816(o[2 * dp], a0, a1, a2, a3, b0, b1);
-            mma_bf16_16816(o[2 * dp + 1], a0, a1, a2, a3, b2, b3);
-        }
-        __syncwarp();
-        if (j + C::kStages < my_n) issue(j + C::kStages);
     }
+    // Consume warp 0's last "merged" arrival so no barrier is left pending.
+    if (warp != 0 && k > 0) named_bar_sync(2);
 
     if (aborted) {
-        // Report, then drain this warp's copies still in flight (bounded)
-        // before the CTA may exit or reuse the ring.
-        if (lane == 0) report(p.error_flags, PA_DEVERR_TIMEOUT);
-        const int issued = min(my_n, consumed + C::kStages);
-        for (int j = consumed; j < issued; ++j)
-            (void)mbar_wait_bounded(&my_bars[j % C::kStages], (j / C::kStages) & 1);
-        m_run = -INFINITY;
-        l_run = 0.f;
-    }
-
-    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
-
-    // Merge the warps through shared memory (the ring is free now).
-    __syncthreads();
-    float* red_o = reinterpret_cast<float*>(ring);           // [warps][8][D]
-    float* red_m = red_o + kWarps * kMaxGroup * D;             // [warps][8]
-    float* red_l = red_m + kWarps * kMaxGroup;                 // [warps][8]
-#pragma unroll
-    for (int j = 0; j < D / 8; ++j) {
-        float* dst = red_o + (warp * kMaxGroup + qr) * D + 8 * j + qc;
-        dst[0] = o[j][0] + o[j][2];
-        dst[1] = o[j][1] + o[j][3];
-    }
-    if ((lane & 3) == 0) {
-        red_m[warp * kMaxGroup + qr] = m_run;
-        red_l[warp * kMaxGroup + qr] = l_run;
-    }
-    __syncthreads();
-
-    for (int i = threadIdx.x; i < G * D; i += kThreads) {
-        const int r = i / D;
-        const int d = i - r * D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, red_m[w * kMaxGroup + r]);
-        float acc = 0.f, den = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            const float mw = red_m[w * kMaxGroup + r];
-            const float sc = mw == -INFINITY ? 0.f : exp2f(mw - M);
-            acc += sc * red_o[(w * kMaxGroup + r) * D + d];
-            den += sc * red_l[w * kMaxGroup + r];
-        }
-        const int h = g * G + r;
-        const float val = acc / den;
-        if (num_parts == 1) {
-            p.out[((int64_t)s * Hq + h) * D + d] = val;
-        } else {
-            const int64_t idx = ((int64_t)s * Hq + h) * p.max_partitions + part;
-            p.tmp_o[idx * D + d] = val;
-            if (d == 0) {
-                p.tmp_m[idx] = M;
-                p.tmp_l[idx] = den;
-            }
-        }
+        // Drain copies still in flight on this warp's ring (bounded) before
+        // the CTA exits.
+        for (int c = drain_from; c < prod_count; ++c)
+            (void)mbar_wait_bounded(&my_bars[c % C::kStages], (c / C::kStages) & 1);
     }
 }
 
@@ -344,29 +534,90 @@ paged_decode_reduce_kernel(const DecodeParams p) {
     p.out[((int64_t)s * p.num_heads + h) * D + d] = acc / den;
 }
 
-template <int D, int BS>
-cudaError_t launch_typed(const DecodeParams& p, int num_seqs,
-                         cudaStream_t stream) {
-    using C = Cfg<D>;
-    static int configured[64] = {0};
+// ------------------------------------------------------------ host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
+                                   void*, const cuuint64_t*, const cuuint64_t*,
+                                   const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr,
+                                    cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// Pool [NB*bs][Hkv][D] viewed as 3-D {64 elements, Hkv*D/64 column tiles,
+// NB*bs token slots}; box = one 128-byte column tile of 16 slots.
+bool encode_pool_map(CUtensorMap* map, const void* pool, int num_blocks,
+                     int block_size, int num_kv_heads, int head_size) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {64, (cuuint64_t)num_kv_heads * head_size / 64,
+                                (cuuint64_t)num_blocks * block_size};
+    const cuuint64_t strides[2] = {128, (cuuint64_t)num_kv_heads * head_size * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)kChunk};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(pool),
+              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename Kernel>
+cudaError_t set_smem(Kernel kernel, int bytes, int* flags) {
     int dev = 0;
-    cudaGetDevice(&dev);
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!__atomic_load_n(&configured[dev], __ATOMIC_ACQUIRE)) {
-        cudaError_t e = cudaFuncSetAttribute(
-            paged_decode_kernel<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-            C::kSmemBytes);
+    if (!__atomic_load_n(&flags[dev], __ATOMIC_ACQUIRE)) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
         if (e != cudaSuccess) return e;
-        __atomic_store_n(&configured[dev], 1, __ATOMIC_RELEASE);
+        __atomic_store_n(&flags[dev], 1, __ATOMIC_RELEASE);
     }
-    dim3 grid((unsigned)p.num_kv_heads, (unsigned)p.max_partitions,
-              (unsigned)num_seqs);
-    paged_decode_kernel<D, BS><<<grid, kThreads, C::kSmemBytes, stream>>>(p);
+    return cudaSuccess;
+}
+
+template <int D, int BS>
+cudaError_t launch_typed(const DecodeParams& p, cudaStream_t stream) {
+    using C = Cfg<D>;
+    static int grid_ready[64] = {0};
+    static int persist_ready[64] = {0};
+    CUtensorMap tmk, tmv;
+    if (!encode_pool_map(&tmk, p.k_cache, p.num_blocks, BS, p.num_kv_heads, D) ||
+        !encode_pool_map(&tmv, p.v_cache, p.num_blocks, BS, p.num_kv_heads, D))
+        return cudaErrorInvalidValue;
+    const bool persist = p.max_partitions > 1 && p.num_seqs <= kMaxPersistSeqs;
+    cudaError_t e;
+    if (persist) {
+        e = set_smem(paged_decode_kernel<D, BS, true>, C::kSmemPersist, persist_ready);
+        if (e != cudaSuccess) return e;
+        long long per_head = (kTargetCtasPerSM * kNumSMs + p.num_kv_heads - 1) / p.num_kv_heads;
+        const long long items = (long long)p.num_seqs * p.max_partitions;
+        if (per_head > items) per_head = items;
+        if (per_head < 1) per_head = 1;
+        dim3 grid((unsigned)p.num_kv_heads, (unsigned)per_head, 1);
+        paged_decode_kernel<D, BS, true><<<grid, kThreads, C::kSmemPersist, stream>>>(tmk, tmv, p);
+    } else {
+        e = set_smem(paged_decode_kernel<D, BS, false>, C::kSmemGrid, grid_ready);
+        if (e != cudaSuccess) return e;
+        dim3 grid((unsigned)p.num_kv_heads, (unsigned)p.max_partitions,
+                  (unsigned)p.num_seqs);
+        paged_decode_kernel<D, BS, false><<<grid, kThreads, C::kSmemGrid, stream>>>(tmk, tmv, p);
+    }
     count_launch();
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (p.max_partitions > 1) {
-        dim3 rgrid((unsigned)p.num_heads, (unsigned)num_seqs);
+        dim3 rgrid((unsigned)p.num_heads, (unsigned)p.num_seqs);
         paged_decode_reduce_kernel<D><<<rgrid, D, 0, stream>>>(p);
         count_launch();
         e = cudaGetLastError();
@@ -378,13 +629,12 @@ cudaError_t launch_typed(const DecodeParams& p, int num_seqs,
 
 float log2e_scale(float scale) { return scale * kLog2e; }
 
-cudaError_t launch_paged_decode(const DecodeParams& p, int num_seqs,
-                                int head_size, int block_size,
-                                cudaStream_t stream) {
-    if (head_size == 128 && block_size == 16) return launch_typed<128, 16>(p, num_seqs, stream);
-    if (head_size == 128 && block_size == 32) return launch_typed<128, 32>(p, num_seqs, stream);
-    if (head_size == 64 && block_size == 16) return launch_typed<64, 16>(p, num_seqs, stream);
-    if (head_size == 64 && block_size == 32) return launch_typed<64, 32>(p, num_seqs, stream);
+cudaError_t launch_paged_decode(const DecodeParams& p, int head_size,
+                                int block_size, cudaStream_t stream) {
+    if (head_size == 128 && block_size == 16) return launch_typed<128, 16>(p, stream);
+    if (head_size == 128 && block_size == 32) return launch_typed<128, 32>(p, stream);
+    if (head_size == 64 && block_size == 16) return launch_typed<64, 16>(p, stream);
+    if (head_size == 64 && block_size == 32) return launch_typed<64, 32>(p, stream);
     return cudaErrorInvalidValue;
 }
 

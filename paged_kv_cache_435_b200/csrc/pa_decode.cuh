@@ -17,6 +17,7 @@ struct DecodeParams {
     float* tmp_m;                // fp32 [B][Hq][max_partitions] (log2 domain)
     float* tmp_l;                // fp32 [B][Hq][max_partitions]
     int* error_flags;            // nullable
+    int num_seqs;
     int max_blocks_per_seq;
     int max_context_len;
     int num_heads;
@@ -32,9 +33,9 @@ struct DecodeParams {
 float log2e_scale(float scale);
 
 // Enqueue the partition kernel (and the merge kernel when
-// max_partitions > 1).  head_size in {64,128}, block_size in {16,32}.
-cudaError_t launch_paged_decode(const DecodeParams& p, int num_seqs,
-                                int head_size, int block_size,
-                                cudaStream_t stream);
+// max_partitions > 1).  head_size in {64,128}, block_size in {16,32};
+// num_blocks * block_size < 2^31.
+cudaError_t launch_paged_decode(const DecodeParams& p, int head_size,
+                                int block_size, cudaStream_t stream);
 
 }  // namespace pa
