@@ -30,6 +30,7 @@ reshape_and_cache_kernel(const uint16_t* __restrict__ key,
                          const int64_t* __restrict__ slot_mapping,
                          int num_tokens, int64_t num_slots, int block_size,
                          int num_kv_heads, int head_size, int* error_flags) {
+    pdl_launch_dependents();  // a following decode launch may get scheduled
     const int chunk_elems = kVec ? 8 : 1;
     const int chunks = head_size / chunk_elems;
     const int64_t per_token = (int64_t)num_kv_heads * chunks;
@@ -71,6 +72,7 @@ reshape_and_cache_kernel(const uint16_t* __restrict__ key,
 __global__ void __launch_bounds__(256)
 copy_blocks_kernel(CopyLayerPtrs ptrs, const int64_t* __restrict__ mapping,
                    int64_t num_blocks, int64_t block_vecs, int* error_flags) {
+    pdl_launch_dependents();
     const int p = blockIdx.x;
     const int layer = blockIdx.y;
     const int64_t src = mapping[2 * (int64_t)p];

@@ -110,6 +110,19 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     return pol;
 }
 
+// ------------------------------------------- programmatic dependent launch
+// Wait until the grids this launch depends on have completed and their
+// memory is visible (no-op when the launch carries no programmatic edge).
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Allow the next launch in the stream, if it opted in, to be scheduled now;
+// it still waits for this grid's completion before touching memory.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------ tensor core
 __device__ __forceinline__ void ldsm_x4(uint32_t& r0, uint32_t& r1,
                                         uint32_t& r2, uint32_t& r3,

@@ -38,6 +38,7 @@
 #include <cfloat>
 #include <cstdint>
 #include <mutex>
+#include <utility>
 
 #include "pa_common.cuh"
 #include "pa_decode.cuh"
@@ -182,6 +183,10 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         if (threadIdx.x == 0) report(p.error_flags, PA_DEVERR_INTERNAL);
         return;
     }
+    // Launched behind the cache write: nothing global is read before the
+    // preceding grid has completed.
+    pdl_wait();
+    pdl_launch_dependents();
 
     if (kPersist) {
         // prefix[s] = partitions of sequences 0..s-1 (block-wide scan).  The
@@ -215,8 +220,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
     }
     __syncthreads();  // barriers initialised, prefix visible
 
-    // Q fragments (A operand): rows = heads of the group, rows >= G zero.
-    // Reloaded per item because items of a persistent CTA differ in sequence.
     const int qr = lane >> 2;       // fragment row owned by this lane
     const int qc = (lane & 3) * 2;  // fragment column pair
     const int xr = lane & 7;        // swizzle phase of this lane's ldmatrix row
@@ -300,22 +303,33 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
     bool aborted = false;
     int drain_from = 0;  // first chunk whose wait gave up
     int k = 0;
+    // Q fragments of an item (A operand): rows = heads of the group, rows >= G
+    // zero.  The next item's are fetched while the current one streams.
+    auto load_q = [&](const Item& it, uint32_t (&dst)[D / 16][2]) {
+        const bool live = it.s >= 0 && qr < G && it.L > 0;
+        const uint16_t* qp =
+            p.q + ((int64_t)(it.s < 0 ? 0 : it.s) * Hq + g * G + (qr < G ? qr : 0)) * D;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            dst[ks][0] = live ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + qc) : 0u;
+            dst[ks][1] = live ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8 + qc) : 0u;
+        }
+    };
+    Item next_it = get_item<kPersist>(p, prefix, 0);
+    uint32_t qnext[D / 16][2];
+    load_q(next_it, qnext);
     for (;; ++k) {
-        const Item it = get_item<kPersist>(p, prefix, k);
+        const Item it = next_it;
         if (it.s < 0) break;
         const int my_n = warp_chunks(it, warp);
-
         uint32_t qa[D / 16][2];
-        {
-            const bool live = qr < G && it.L > 0;
-            const uint16_t* qp =
-                p.q + ((int64_t)it.s * Hq + g * G + (qr < G ? qr : 0)) * D;
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-                qa[ks][0] = live ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + qc) : 0u;
-                qa[ks][1] = live ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8 + qc) : 0u;
-            }
+        for (int ks = 0; ks < D / 16; ++ks) {
+            qa[ks][0] = qnext[ks][0];
+            qa[ks][1] = qnext[ks][1];
         }
+        next_it = get_item<kPersist>(p, prefix, k + 1);
+        load_q(next_it, qnext);
 
         float o[D / 8][4];
 #pragma unroll
@@ -501,37 +515,90 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
 }
 
 // Merge of the per-partition results: out = sum_p w_p o_p / sum_p w_p with
-// w_p = l_p * 2^(m_p - max_p m_p).  One CTA per (query head, sequence).
+// w_p = l_p * 2^(m_p - max_p m_p).  One CTA of 8 warps per (query head,
+// sequence); warp w takes partitions w, w+8, ... with 8 partitions' rows in
+// flight per round, each lane holding D/32 consecutive columns.
+constexpr int kReduceWarps = 8;
+constexpr int kReduceUnroll = 8;
+
 template <int D>
-__global__ void __launch_bounds__(D)
+__global__ void __launch_bounds__(kReduceWarps * 32)
 paged_decode_reduce_kernel(const DecodeParams p) {
+    constexpr int V = D / 32;  // columns per lane
     const int h = blockIdx.x;
     const int s = blockIdx.y;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    pdl_wait();  // the partials come from the grid launched just before
     int L = p.context_lens[s];
     L = L < 0 ? 0 : (L > p.max_context_len ? p.max_context_len : L);
     const int np = (L + p.partition_size - 1) / p.partition_size;
     if (np <= 1) return;  // written directly by the partition kernel
     const int64_t base = ((int64_t)s * p.num_heads + h) * p.max_partitions;
 
-    __shared__ float warp_max[D / 32];
+    __shared__ float warp_max[kReduceWarps];
+    __shared__ float part_acc[kReduceWarps][D];
+    __shared__ float part_den[kReduceWarps];
+
     float M = -INFINITY;
-    for (int i = threadIdx.x; i < np; i += D) M = fmaxf(M, p.tmp_m[base + i]);
+    for (int i = threadIdx.x; i < np; i += kReduceWarps * 32)
+        M = fmaxf(M, p.tmp_m[base + i]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = M;
+    if (lane == 0) warp_max[warp] = M;
     __syncthreads();
     M = warp_max[0];
 #pragma unroll
-    for (int w = 1; w < D / 32; ++w) M = fmaxf(M, warp_max[w]);
+    for (int w = 1; w < kReduceWarps; ++w) M = fmaxf(M, warp_max[w]);
 
-    const int d = threadIdx.x;
-    float acc = 0.f, den = 0.f;
-    for (int i = 0; i < np; ++i) {
-        const float w = p.tmp_l[base + i] * exp2f(p.tmp_m[base + i] - M);
-        acc += w * p.tmp_o[(base + i) * D + d];
-        den += w;
+    float acc[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) acc[v] = 0.f;
+    float den = 0.f;
+    for (int i0 = warp; i0 < np; i0 += kReduceWarps * kReduceUnroll) {
+        float wts[kReduceUnroll];
+        float vals[kReduceUnroll][V];
+        float lv[kReduceUnroll], mv[kReduceUnroll];
+#pragma unroll
+        for (int u = 0; u < kReduceUnroll; ++u) {
+            // Rows past np re-read the last row with weight 0, so every load
+            // of the round is unconditional and in flight together.
+            const int i = min(i0 + u * kReduceWarps, np - 1);
+            lv[u] = p.tmp_l[base + i];
+            mv[u] = p.tmp_m[base + i];
+            const float* row = p.tmp_o + (base + i) * D + lane * V;
+            if (V == 4) {
+                const float4 t = *reinterpret_cast<const float4*>(row);
+                vals[u][0] = t.x; vals[u][V > 1 ? 1 : 0] = t.y;
+                vals[u][V > 2 ? 2 : 0] = t.z; vals[u][V > 3 ? 3 : 0] = t.w;
+            } else {
+                const float2 t = *reinterpret_cast<const float2*>(row);
+                vals[u][0] = t.x; vals[u][V > 1 ? 1 : 0] = t.y;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kReduceUnroll; ++u)
+            wts[u] = i0 + u * kReduceWarps < np ? lv[u] * exp2f(mv[u] - M) : 0.f;
+#pragma unroll
+        for (int u = 0; u < kReduceUnroll; ++u) {
+            den += wts[u];
+#pragma unroll
+            for (int v = 0; v < V; ++v) acc[v] += wts[u] * vals[u][v];
+        }
     }
-    p.out[((int64_t)s * p.num_heads + h) * D + d] = acc / den;
+#pragma unroll
+    for (int v = 0; v < V; ++v) part_acc[warp][lane * V + v] = acc[v];
+    if (lane == 0) part_den[warp] = den;
+    __syncthreads();
+    for (int d = threadIdx.x; d < D; d += kReduceWarps * 32) {
+        float a = 0.f, dn = 0.f;
+#pragma unroll
+        for (int w = 0; w < kReduceWarps; ++w) {
+            a += part_acc[w][d];
+            dn += part_den[w];
+        }
+        p.out[((int64_t)s * p.num_heads + h) * D + d] = a / dn;
+    }
 }
 
 // ------------------------------------------------------------ host side
@@ -572,6 +639,24 @@ bool encode_pool_map(CUtensorMap* map, const void* pool, int num_blocks,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Launch with a programmatic edge to the previous kernel in the stream: this
+// grid may be scheduled while that one finishes and waits for it in-kernel.
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block,
+                       size_t smem, cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <typename Kernel>
 cudaError_t set_smem(Kernel kernel, int bytes, int* flags) {
     int dev = 0;
@@ -605,22 +690,23 @@ cudaError_t launch_typed(const DecodeParams& p, cudaStream_t stream) {
         if (per_head > items) per_head = items;
         if (per_head < 1) per_head = 1;
         dim3 grid((unsigned)p.num_kv_heads, (unsigned)per_head, 1);
-        paged_decode_kernel<D, BS, true><<<grid, kThreads, C::kSmemPersist, stream>>>(tmk, tmv, p);
+        e = launch_pdl(paged_decode_kernel<D, BS, true>, grid, dim3(kThreads),
+                       C::kSmemPersist, stream, tmk, tmv, p);
     } else {
         e = set_smem(paged_decode_kernel<D, BS, false>, C::kSmemGrid, grid_ready);
         if (e != cudaSuccess) return e;
         dim3 grid((unsigned)p.num_kv_heads, (unsigned)p.max_partitions,
                   (unsigned)p.num_seqs);
-        paged_decode_kernel<D, BS, false><<<grid, kThreads, C::kSmemGrid, stream>>>(tmk, tmv, p);
+        e = launch_pdl(paged_decode_kernel<D, BS, false>, grid, dim3(kThreads),
+                       C::kSmemGrid, stream, tmk, tmv, p);
     }
     count_launch();
-    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (p.max_partitions > 1) {
         dim3 rgrid((unsigned)p.num_heads, (unsigned)p.num_seqs);
-        paged_decode_reduce_kernel<D><<<rgrid, D, 0, stream>>>(p);
+        e = launch_pdl(paged_decode_reduce_kernel<D>, rgrid,
+                       dim3(kReduceWarps * 32), 0, stream, p);
         count_launch();
-        e = cudaGetLastError();
     }
     return e;
 }
