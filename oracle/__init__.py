@@ -75,6 +75,10 @@ def _load():
             lib.oracle_paged_decode_attention.argtypes = [
                 p, p, p, p, p, i32, p, i32, i32, i32, i32, i32, i32, dbl, i32]
             lib.oracle_paged_decode_attention.restype = i32
+            lib.oracle_paged_multi_query_attention.argtypes = [
+                p, p, p, p, p, i32, p, p, i32, i32, i32, i32, i32, i32, dbl,
+                i32]
+            lib.oracle_paged_multi_query_attention.restype = i32
             _lib = lib
     return _lib
 
@@ -135,6 +139,37 @@ def paged_decode_attention(q, k_cache, v_cache, block_tables, context_lens,
         _ptr(cl), B, Hq, Hkv, D, bs, NB, float(scale),
         threads if threads is not None else default_threads())
     _check(rc, "paged_decode_attention")
+    return out
+
+
+def paged_multi_query_attention(q, k_cache, v_cache, block_tables,
+                                context_lens, query_start_loc, scale: float,
+                                num_kv_heads: int,
+                                threads: int | None = None) -> np.ndarray:
+    """fp64 causal attention of k new query tokens per sequence.
+
+    q: bf16 [T, Hq, D] (T = query_start_loc[-1]); query_start_loc: int32
+    [B+1]; the last k_s = qsl[s+1]-qsl[s] of sequence s's context_lens[s]
+    tokens are its queries.  Returns float64 [T, Hq, D].
+    """
+    lib = _load()
+    qb, kb, vb = _bits16(q), _bits16(k_cache), _bits16(v_cache)
+    bt = _arr(block_tables, np.int32)
+    cl = _arr(context_lens, np.int32)
+    qsl = _arr(query_start_loc, np.int32)
+    T, Hq, D = qb.shape
+    NB, bs, Hkv, D2 = kb.shape
+    B = cl.shape[0]
+    if D2 != D or Hkv != num_kv_heads or vb.shape != kb.shape:
+        raise ValueError("shape mismatch")
+    if qsl.shape != (B + 1,) or int(qsl[-1]) != T or bt.shape[0] != B:
+        raise ValueError("query_start_loc / block_tables shape mismatch")
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    rc = lib.oracle_paged_multi_query_attention(
+        _ptr(out), _ptr(qb), _ptr(kb), _ptr(vb), _ptr(bt), bt.shape[1],
+        _ptr(cl), _ptr(qsl), B, Hq, Hkv, D, bs, NB, float(scale),
+        threads if threads is not None else default_threads())
+    _check(rc, "paged_multi_query_attention")
     return out
 
 

@@ -263,3 +263,147 @@ int oracle_paged_decode_attention(
     pthread_mutex_destroy(&job.lock);
     return job.status;
 }
+
+/* ------------------------------------------------------------------------ */
+/* multi-query paged attention (chunked prefill / speculative verification)  */
+/* ------------------------------------------------------------------------ */
+/* Sequence s holds L = context_lens[s] cached tokens, of which the last
+ * k = query_start_loc[s+1] - query_start_loc[s] are the new query tokens
+ * (their K/V already written).  Query token j (0 <= j < k) sits at logical
+ * position L - k + j and attends causally to tokens t <= L - k + j
+ * ("vLLM: Anatomy and Mechanisms of High-Throughput LLM Inference",
+ * "Chunked Prefill" and "Speculative Decoding": the large model verifies all
+ * k proposed tokens in one forward pass).  q and out are indexed by the
+ * global query token query_start_loc[s] + j.  Output double
+ * out[num_q_tokens][num_heads][head_size]. */
+typedef struct {
+    double* out;
+    const uint16_t* q;
+    const uint16_t* k_cache;
+    const uint16_t* v_cache;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    const int32_t* query_start_loc;
+    int max_blocks_per_seq, num_seqs, num_heads, num_kv_heads, head_size;
+    int block_size, num_blocks;
+    double scale;
+    int next_item;
+    pthread_mutex_t lock;
+    int status;
+} mq_job;
+
+static int mq_attend_one(mq_job* job, int s, int h) {
+    const int D = job->head_size;
+    const int G = job->num_heads / job->num_kv_heads;
+    const int kv = h / G;
+    const int L = job->context_lens[s];
+    const int q0 = job->query_start_loc[s];
+    const int k = job->query_start_loc[s + 1] - q0;
+    if (k < 0 || k > L || L > job->max_blocks_per_seq * job->block_size)
+        return ORACLE_ERR_RANGE;
+    double* z = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+    if (!z) return ORACLE_ERR_NOMEM;
+    for (int j = 0; j < k; ++j) {
+        const int last = L - k + j; /* last visible logical position */
+        const uint16_t* qv = job->q + ((int64_t)(q0 + j) * job->num_heads + h) * D;
+        double* o = job->out + ((int64_t)(q0 + j) * job->num_heads + h) * D;
+        for (int d = 0; d < D; ++d) o[d] = 0.0;
+        for (int t = 0; t <= last; ++t) {
+            int32_t phys = job->block_tables[(int64_t)s * job->max_blocks_per_seq +
+                                             t / job->block_size];
+            if (phys < 0 || phys >= job->num_blocks) {
+                free(z);
+                return ORACLE_ERR_RANGE;
+            }
+            double dot = 0.0;
+            for (int d = 0; d < D; ++d)
+                dot += bf16_bits_to_double(qv[d]) *
+                       bf16_bits_to_double(job->k_cache[pool_index(
+                           phys, t % job->block_size, kv, d, job->block_size,
+                           job->num_kv_heads, D)]);
+            z[t] = job->scale * dot;
+        }
+        double zmax = z[0];
+        for (int t = 1; t <= last; ++t)
+            if (z[t] > zmax) zmax = z[t];
+        double wsum = 0.0;
+        for (int t = 0; t <= last; ++t) {
+            z[t] = exp(z[t] - zmax);
+            wsum += z[t];
+        }
+        for (int t = 0; t <= last; ++t) {
+            int32_t phys = job->block_tables[(int64_t)s * job->max_blocks_per_seq +
+                                             t / job->block_size];
+            for (int d = 0; d < D; ++d)
+                o[d] += z[t] * bf16_bits_to_double(job->v_cache[pool_index(
+                                   phys, t % job->block_size, kv, d,
+                                   job->block_size, job->num_kv_heads, D)]);
+        }
+        for (int d = 0; d < D; ++d) o[d] /= wsum;
+    }
+    free(z);
+    return ORACLE_OK;
+}
+
+static void* mq_worker(void* arg) {
+    mq_job* job = (mq_job*)arg;
+    const int total = job->num_seqs * job->num_heads;
+    for (;;) {
+        pthread_mutex_lock(&job->lock);
+        int item = job->next_item++;
+        int failed = job->status != ORACLE_OK;
+        pthread_mutex_unlock(&job->lock);
+        if (item >= total || failed) break;
+        int rc = mq_attend_one(job, item / job->num_heads, item % job->num_heads);
+        if (rc != ORACLE_OK) {
+            pthread_mutex_lock(&job->lock);
+            if (job->status == ORACLE_OK) job->status = rc;
+            pthread_mutex_unlock(&job->lock);
+        }
+    }
+    return NULL;
+}
+
+int oracle_paged_multi_query_attention(
+    double* out, const uint16_t* q, const uint16_t* k_cache,
+    const uint16_t* v_cache, const int32_t* block_tables,
+    int max_blocks_per_seq, const int32_t* context_lens,
+    const int32_t* query_start_loc, int num_seqs, int num_heads,
+    int num_kv_heads, int head_size, int block_size, int num_blocks,
+    double scale, int num_threads) {
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 ||
+        head_size <= 0 || block_size <= 0 || num_blocks <= 0 ||
+        max_blocks_per_seq <= 0 || num_heads % num_kv_heads != 0)
+        return ORACLE_ERR_ARG;
+    mq_job job;
+    job.out = out;
+    job.q = q;
+    job.k_cache = k_cache;
+    job.v_cache = v_cache;
+    job.block_tables = block_tables;
+    job.context_lens = context_lens;
+    job.query_start_loc = query_start_loc;
+    job.max_blocks_per_seq = max_blocks_per_seq;
+    job.num_seqs = num_seqs;
+    job.num_heads = num_heads;
+    job.num_kv_heads = num_kv_heads;
+    job.head_size = head_size;
+    job.block_size = block_size;
+    job.num_blocks = num_blocks;
+    job.scale = scale;
+    job.next_item = 0;
+    job.status = ORACLE_OK;
+    pthread_mutex_init(&job.lock, NULL);
+    if (num_threads < 1) num_threads = 1;
+    if (num_threads > 256) num_threads = 256;
+    pthread_t tids[256];
+    int started = 0;
+    for (int i = 1; i < num_threads; ++i) {
+        if (pthread_create(&tids[started], NULL, mq_worker, &job) != 0) break;
+        ++started;
+    }
+    mq_worker(&job);
+    for (int i = 0; i < started; ++i) pthread_join(tids[i], NULL);
+    pthread_mutex_destroy(&job.lock);
+    return job.status;
+}

@@ -111,6 +111,10 @@ class DecodeCase:
     unique_tokens: int           # distinct (block, offset) positions read
     logical_tokens: int          # sum of context lengths
     scale_override: Optional[float] = None
+    # multi-query cases: the last k_s context tokens of sequence s are its
+    # queries; q / new_key / new_value / slot_mapping then have sum(k_s) rows
+    query_start_loc: Optional[torch.Tensor] = None   # int32 [B+1]
+    query_lens_np: Optional[np.ndarray] = None        # int64 [B]
 
     @property
     def scale(self) -> float:
@@ -291,3 +295,37 @@ def custom_case(num_seqs: int, num_heads: int, num_kv_heads: int,
     lens = np.asarray(lens, dtype=np.int64)
     return build_case(w, lens, device=device, seed=seed,
                       num_blocks=num_blocks)
+
+
+def multi_query_case(num_seqs: int, num_heads: int, num_kv_heads: int,
+                     head_size: int, block_size: int, lens, query_lens,
+                     seed: int, device="cpu", pool_device=None,
+                     name: str = "multi_query") -> DecodeCase:
+    """k_s new query tokens per sequence (chunked prefill or speculative
+    verification): they occupy logical positions L_s - k_s .. L_s - 1, and
+    their K/V rows are the step's new tokens with slots from the tables."""
+    lens = np.asarray(lens, dtype=np.int64)
+    qlens = np.asarray(query_lens, dtype=np.int64)
+    assert lens.shape == qlens.shape == (num_seqs,) and np.all(qlens <= lens)
+    w = Workload(name, 0, num_seqs, num_heads, num_kv_heads, head_size,
+                 block_size, "fixed")
+    base = build_case(w, lens, device=device, seed=seed,
+                      pool_device=pool_device)
+    T = int(qlens.sum())
+    g = _generator("cpu", seed + 3)
+    q = _randn_bf16((T, num_heads, head_size), g, "cpu")
+    nk = _randn_bf16((T, num_kv_heads, head_size), g, "cpu")
+    nv = _randn_bf16((T, num_kv_heads, head_size), g, "cpu")
+    qsl = np.zeros(num_seqs + 1, dtype=np.int32)
+    qsl[1:] = np.cumsum(qlens)
+    slots = np.empty(T, dtype=np.int64)
+    for s in range(num_seqs):
+        for j in range(int(qlens[s])):
+            pos = int(lens[s] - qlens[s] + j)
+            slots[qsl[s] + j] = int(base.tables_np[s, pos // block_size]) * \
+                block_size + pos % block_size
+    dev = torch.device(device)
+    return dataclasses.replace(
+        base, q=q.to(dev), new_key=nk.to(dev), new_value=nv.to(dev),
+        slot_mapping=torch.from_numpy(slots).to(dev),
+        query_start_loc=torch.from_numpy(qsl).to(dev), query_lens_np=qlens)

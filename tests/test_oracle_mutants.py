@@ -1,5 +1,5 @@
 """Plant plausible mistakes in the oracle's C source and check that the pins in
-tests/test_oracle.py catch every one.
+tests/test_oracle.py and tests/test_oracle_multi_query.py catch every one.
 
 Each mutant is one textual edit of oracle/pa_oracle.c (a wrong head mapping, a
 dropped scale, a transposed pool layout, ...).  It is compiled with gcc into a
@@ -43,6 +43,13 @@ MUTANTS = {
         "k_cache[dst] = value[(int64_t)i * value_token_stride +"),
     "padding_rule_includes_slot_zero": ("if (slot < 0) continue;",
                                         "if (slot <= 0) continue;"),
+    "causal_limit_off_by_one": ("const int last = L - k + j;",
+                                "const int last = L - k + j - 1;"),
+    "query_row_not_advanced": (
+        "const uint16_t* qv = job->q + ((int64_t)(q0 + j) * job->num_heads + h) * D;",
+        "const uint16_t* qv = job->q + ((int64_t)(q0) * job->num_heads + h) * D;"),
+    "query_count_off_by_one": ("const int k = job->query_start_loc[s + 1] - q0;",
+                               "const int k = job->query_start_loc[s + 1] - q0 - 1;"),
     "copy_direction_swapped": (
         "int64_t src = block_mapping[2 * p];\n        int64_t dst = block_mapping[2 * p + 1];",
         "int64_t src = block_mapping[2 * p + 1];\n        int64_t dst = block_mapping[2 * p];"),
@@ -63,7 +70,8 @@ def _run_pins(lib_path: str) -> int:
     env = dict(os.environ, PA_ORACLE_LIB=lib_path)
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q",
                         "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle.py")],
+                        os.path.join(ROOT, "tests", "test_oracle.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_multi_query.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True,
                        timeout=600)
     return r.returncode
