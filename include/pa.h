@@ -83,6 +83,7 @@ typedef enum {
 #define PA_DEVERR_COPY_PAIR 0x8   /* block_mapping id outside [0,num_blocks) */
 #define PA_DEVERR_TIMEOUT 0x10    /* an async-copy wait exceeded its time limit */
 #define PA_DEVERR_INTERNAL 0x20   /* shared memory not 1024-byte aligned (no work done) */
+#define PA_DEVERR_QUERY_LEN 0x40  /* query count < 0, > context length or > max_query_len */
 
 /* Human-readable name of a pa_status value (static string, never NULL). */
 const char* pa_status_string(int status);
@@ -178,6 +179,43 @@ int pa_decode_attention(float* out, const void* q, const void* k_cache,
                         int num_blocks, float scale, int partition_size,
                         void* workspace, size_t workspace_bytes,
                         int* error_flags, pa_stream_t stream);
+
+/*
+ * pa_multi_query_attention - paged attention of k new query tokens per
+ * sequence, causal within the chunk: the attention of a chunked-prefill chunk
+ * or of speculative-decoding verification, where all k proposed tokens are
+ * checked in one pass ("vLLM: Anatomy and Mechanisms of High-Throughput LLM
+ * Inference", sections "Chunked Prefill" and "Speculative Decoding"; "Inside
+ * vLLM: Anatomy of a High-Throughput LLM Inference System", "Scheduler").
+ *
+ * Sequence s has L = context_lens[s] cached tokens, the last
+ * k = query_start_loc[s+1] - query_start_loc[s] of which are its queries
+ * (their K/V already written, e.g. by pa_reshape_and_cache).  Query token j
+ * of s is row t = query_start_loc[s] + j of q / out; it sits at position
+ * L - k + j and, for each query head h (kv head g = h / (num_heads /
+ * num_kv_heads)), computes
+ *     out[t][h][:] = sum_{u <= L-k+j} softmax_u(scale * q[t][h].k_u) v_u.
+ * k = 1 for every sequence is decode attention.
+ *
+ *   q                   bf16 [T][num_heads][head_size], T = query_start_loc[num_seqs]
+ *   out                 fp32 [T][num_heads][head_size]
+ *   query_start_loc     int32 [num_seqs + 1], device, non-decreasing, [0] = 0
+ *   max_query_len       host-known upper bound of k (<= max_context_len)
+ *   other arguments     as for pa_decode_attention (no workspace: no split)
+ *   error_flags         nullable; PA_DEVERR_BLOCK_ID, PA_DEVERR_CONTEXT_LEN,
+ *                       PA_DEVERR_QUERY_LEN, PA_DEVERR_TIMEOUT
+ * Supports head_size in {64, 128}, block_size in {16, 32},
+ * num_heads / num_kv_heads in 1..64.  Returns PA_OK or a negative pa_status.
+ */
+int pa_multi_query_attention(float* out, const void* q, const void* k_cache,
+                             const void* v_cache, const int32_t* block_tables,
+                             int max_blocks_per_seq,
+                             const int32_t* context_lens, int max_context_len,
+                             const int32_t* query_start_loc, int max_query_len,
+                             int num_seqs, int num_heads, int num_kv_heads,
+                             int head_size, int block_size, int num_blocks,
+                             float scale, int* error_flags,
+                             pa_stream_t stream);
 
 /* Capacity, in bytes, of the workspace built into the library for
  * pa_decode_attention_static_ws (32 MiB per GPU that uses the library). */

@@ -8,7 +8,9 @@ entry points, bound here under the same names:
 * ``pa_decode_attention``: one-query-token-per-sequence attention over the
   paged K/V pool through per-sequence block tables (GQA folded, split-KV for
   long contexts);
-* ``pa_copy_blocks``: copy-on-write block copies.
+* ``pa_copy_blocks``: copy-on-write block copies;
+* ``pa_multi_query_attention``: k causal query tokens per sequence (chunked
+  prefill chunks, speculative-decoding verification).
 
 ``inputs`` builds seeded synthetic workloads.  The library is loaded lazily on
 first use and its absence raises; nothing here computes on the CPU.
@@ -16,7 +18,8 @@ first use and its absence raises; nothing here computes on the CPU.
 from ._native import (  # noqa: F401
     PA_DEVERR_BLOCK_ID, PA_DEVERR_CONTEXT_LEN, PA_DEVERR_COPY_PAIR,
     PA_DEVERR_SLOT, PA_DEVERR_TIMEOUT, PA_ERR_CUDA, PA_ERR_INVALID_ARG,
-    PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_OK, PAError, library_path,
+    PA_DEVERR_QUERY_LEN, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_OK, PAError,
+    library_path,
     pa_copy_blocks, pa_decode_attention, pa_decode_partition_size,
-    pa_decode_workspace_size, pa_launch_count, pa_reshape_and_cache, raw,
-    status_string)
+    pa_decode_workspace_size, pa_launch_count, pa_multi_query_attention,
+    pa_reshape_and_cache, raw, status_string)

@@ -27,6 +27,7 @@ PA_DEVERR_SLOT = 0x4
 PA_DEVERR_COPY_PAIR = 0x8
 PA_DEVERR_TIMEOUT = 0x10
 PA_DEVERR_INTERNAL = 0x20
+PA_DEVERR_QUERY_LEN = 0x40
 
 _lock = threading.Lock()
 _lib = None
@@ -72,6 +73,10 @@ def raw():
             p, p, p, p, p, i32, p, i32, i32, i32, i32, i32, i32, i32, f32, i32,
             p, sz, p, p]
         lib.pa_decode_attention.restype = i32
+        lib.pa_multi_query_attention.argtypes = [
+            p, p, p, p, p, i32, p, i32, p, i32, i32, i32, i32, i32, i32, i32,
+            f32, p, p]
+        lib.pa_multi_query_attention.restype = i32
         lib.pa_copy_blocks.argtypes = [p, p, i32, p, i32, i32, i32, i32, i32,
                                        p, p]
         lib.pa_copy_blocks.restype = i32
@@ -193,6 +198,40 @@ def pa_decode_attention(out, q, k_cache, v_cache, block_tables, context_lens,
         Hkv, D, bs, NB, float(scale), int(partition_size), _ptr(workspace),
         ws_bytes, _ptr(error_flags), _stream(stream))
     return _check(rc, "pa_decode_attention")
+
+
+def pa_multi_query_attention(out, q, k_cache, v_cache, block_tables,
+                             context_lens, query_start_loc, max_context_len: int,
+                             max_query_len: int, scale: float,
+                             error_flags=None, stream=None) -> int:
+    """out fp32 [T,Hq,D] = causal paged attention of the last k_s context
+    tokens of each sequence (q bf16 [T,Hq,D], query_start_loc int32 [B+1])."""
+    import torch
+    bf = torch.bfloat16
+    _cuda(out, "out", torch.float32, 3); _cuda(q, "q", bf, 3)
+    _cuda(k_cache, "k_cache", bf, 4); _cuda(v_cache, "v_cache", bf, 4)
+    _cuda(block_tables, "block_tables", torch.int32, 2)
+    _cuda(context_lens, "context_lens", torch.int32, 1)
+    _cuda(query_start_loc, "query_start_loc", torch.int32, 1)
+    for name, t in (("out", out), ("q", q), ("k_cache", k_cache),
+                    ("v_cache", v_cache), ("block_tables", block_tables),
+                    ("context_lens", context_lens),
+                    ("query_start_loc", query_start_loc)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    T, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_cache.shape
+    B = context_lens.shape[0]
+    if out.shape != q.shape or D2 != D or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch between q, out and the pools")
+    if block_tables.shape[0] != B or query_start_loc.shape[0] != B + 1:
+        raise ValueError("block_tables / query_start_loc must match B")
+    rc = raw().pa_multi_query_attention(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), int(max_context_len),
+        _ptr(query_start_loc), int(max_query_len), B, Hq, Hkv, D, bs, NB,
+        float(scale), _ptr(error_flags), _stream(stream))
+    return _check(rc, "pa_multi_query_attention")
 
 
 def pa_copy_blocks(k_caches: Sequence, v_caches: Sequence, block_mapping,

@@ -10,6 +10,7 @@
 #include "pa_cache_ops.cuh"
 #include "pa_common.cuh"
 #include "pa_decode.cuh"
+#include "pa_multi_query.cuh"
 
 namespace pa {
 
@@ -214,6 +215,65 @@ int pa_decode_attention(float* out, const void* q, const void* k_cache,
     p.max_partitions = np;
     p.scale_log2 = pa::log2e_scale(scale);
     cudaError_t e = pa::launch_paged_decode(
+        p, head_size, block_size, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_multi_query_attention(float* out, const void* q, const void* k_cache,
+                             const void* v_cache, const int32_t* block_tables,
+                             int max_blocks_per_seq,
+                             const int32_t* context_lens, int max_context_len,
+                             const int32_t* query_start_loc, int max_query_len,
+                             int num_seqs, int num_heads, int num_kv_heads,
+                             int head_size, int block_size, int num_blocks,
+                             float scale, int* error_flags,
+                             pa_stream_t stream) {
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 ||
+        head_size <= 0 || block_size <= 0 || num_blocks <= 0 ||
+        max_blocks_per_seq <= 0 || max_context_len < 0 || max_query_len < 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    if ((long long)max_context_len > (long long)max_blocks_per_seq * block_size)
+        return PA_ERR_INVALID_ARG;
+    if (max_query_len > max_context_len) return PA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+    const int G = num_heads / num_kv_heads;
+    if (!((head_size == 64 || head_size == 128) &&
+          (block_size == 16 || block_size == 32) && G >= 1 && G <= 64))
+        return PA_ERR_UNSUPPORTED;
+    if ((long long)num_blocks * block_size > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+    if (num_seqs == 0 || max_query_len == 0) return PA_OK;
+    if (num_seqs > pa::kMaxGridYZ) return PA_ERR_UNSUPPORTED;
+    if ((long long)max_query_len * G > 16LL * 4 * pa::kMaxGridYZ)
+        return PA_ERR_UNSUPPORTED;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens ||
+        !query_start_loc)
+        return PA_ERR_INVALID_ARG;
+    if (!pa::aligned16(out) || !pa::aligned16(q) || !pa::aligned16(k_cache) ||
+        !pa::aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+        (reinterpret_cast<uintptr_t>(context_lens) & 3u) ||
+        (reinterpret_cast<uintptr_t>(query_start_loc) & 3u))
+        return PA_ERR_INVALID_ARG;
+    pa::MultiQueryParams p{};
+    p.out = out;
+    p.q = static_cast<const uint16_t*>(q);
+    p.k_cache = static_cast<const uint16_t*>(k_cache);
+    p.v_cache = static_cast<const uint16_t*>(v_cache);
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.query_start_loc = query_start_loc;
+    p.error_flags = error_flags;
+    p.num_seqs = num_seqs;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.max_context_len = max_context_len;
+    p.max_query_len = max_query_len;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.num_blocks = num_blocks;
+    p.group = G;
+    p.scale_log2 = pa::mq_log2e_scale(scale);
+    cudaError_t e = pa::launch_paged_multi_query(
         p, head_size, block_size, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

@@ -1,0 +1,121 @@
+"""pa_multi_query_attention on the GPU through the C ABI against the fp64
+oracle: k causal query tokens per sequence (speculative verification,
+chunked-prefill chunks, whole-prompt prefill), the step's K/V written first
+with pa_reshape_and_cache.  Tolerance as for decode: max-abs <= 4e-3 and
+relative L2 <= 1e-3; cache writes bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_435_b200 as pa
+from paged_kv_cache_435_b200 import inputs
+from tests.helpers import assert_attn_close, bits
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _need_gpu():
+    assert torch.cuda.is_available(), "GPU test run without a CUDA device"
+
+
+def gpu_mq(case, flags=None, write=True):
+    if write:
+        pa.pa_reshape_and_cache(case.new_key, case.new_value, case.k_cache,
+                                case.v_cache, case.slot_mapping,
+                                error_flags=flags)
+    out = torch.empty(case.q.shape, dtype=torch.float32, device="cuda")
+    pa.pa_multi_query_attention(out, case.q, case.k_cache, case.v_cache,
+                                case.block_tables, case.context_lens,
+                                case.query_start_loc, case.max_context_len,
+                                int(case.query_lens_np.max(initial=0)),
+                                case.scale, error_flags=flags)
+    return out
+
+
+def check(case, rows=None):
+    ek, ev = bits(case.k_cache), bits(case.v_cache)
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = gpu_mq(case, flags)
+    torch.cuda.synchronize()
+    assert int(flags.item()) == 0
+    oracle.reshape_and_cache(case.new_key.cpu(), case.new_value.cpu(), ek, ev,
+                             case.slot_mapping.cpu().numpy())
+    np.testing.assert_array_equal(bits(case.k_cache), ek)
+    ref = oracle.paged_multi_query_attention(
+        case.q.cpu(), ek, ev, case.tables_np, case.lens_np.astype(np.int32),
+        case.query_start_loc.cpu().numpy(), case.scale,
+        case.workload.num_kv_heads)
+    if rows is not None:
+        return assert_attn_close(out[torch.as_tensor(rows).cuda()], ref[rows],
+                                 case.workload.name), out
+    return assert_attn_close(out, ref, case.workload.name), out
+
+
+@pytest.mark.parametrize("Hq,Hkv,D,bs,lens,qlens", [
+    (64, 8, 128, 16, [300, 1000, 17, 4096], [4, 4, 4, 4]),     # spec verify
+    (32, 8, 128, 32, [700, 64, 129], [5, 3, 8]),
+    (16, 16, 128, 16, [257, 40, 90], [2, 1, 7]),                # MHA
+    (8, 2, 64, 16, [600, 33, 512, 5], [128, 33, 100, 0]),       # chunks
+    (28, 4, 64, 32, [100, 70], [100, 19]),                       # G=7, k=L
+    (4, 4, 128, 16, [1, 2, 3], [1, 2, 3]),
+    (32, 2, 128, 16, [2048, 300], [200, 64]),                    # G=16
+])
+def test_multi_query_shapes(Hq, Hkv, D, bs, lens, qlens):
+    case = inputs.multi_query_case(len(lens), Hq, Hkv, D, bs, lens, qlens,
+                                   seed=sum(lens) + Hq, device="cuda")
+    check(case)
+
+
+def test_single_query_matches_decode_kernel():
+    lens = [1, 15, 16, 17, 100, 1000, 3000]
+    case = inputs.multi_query_case(len(lens), 32, 8, 128, 16, lens,
+                                   [1] * len(lens), seed=2, device="cuda")
+    (_, _), mq = check(case)
+    B, Hq, D = case.q.shape
+    dec = torch.empty(B, Hq, D, dtype=torch.float32, device="cuda")
+    nbytes = pa.pa_decode_workspace_size(B, Hq, 8, D, 16, case.max_context_len)
+    ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device="cuda")
+    pa.pa_decode_attention(dec, case.q, case.k_cache, case.v_cache,
+                           case.block_tables, case.context_lens,
+                           case.max_context_len, case.scale, workspace=ws)
+    torch.cuda.synchronize()
+    assert (mq - dec).abs().max().item() <= 2e-5
+
+
+def test_speculative_verify_batch256_sampled():
+    """Batch-256 GQA layer (64q/8kv, D=128, L~U[256,4096]) verifying 4 draft
+    tokens per sequence; 16 sequences' rows compared."""
+    rng = np.random.default_rng(1003)
+    lens = rng.integers(256, 4097, size=256)
+    case = inputs.multi_query_case(256, 64, 8, 128, 16, lens, [4] * 256,
+                                   seed=77, device="cuda")
+    seqs = np.concatenate([[int(np.argmax(lens)), int(np.argmin(lens))],
+                           np.arange(0, 256, 19)])
+    rows = np.concatenate([np.arange(4 * s, 4 * s + 4) for s in np.unique(seqs)])
+    check(case, rows=rows)
+
+
+def test_run_to_run_determinism():
+    case = inputs.multi_query_case(3, 32, 4, 128, 16, [500, 90, 2000],
+                                   [40, 9, 6], seed=5, device="cuda")
+    a = gpu_mq(case, write=False)
+    b = gpu_mq(case, write=False)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_query_count_above_context_sets_flag():
+    case = inputs.multi_query_case(2, 8, 2, 64, 16, [20, 30], [4, 4], seed=9,
+                                   device="cuda")
+    case.query_start_loc[2] = 40          # seq 1 claims 36 queries > 30 tokens
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.empty(40, 8, 64, dtype=torch.float32, device="cuda")
+    q = torch.zeros(40, 8, 64, dtype=torch.bfloat16, device="cuda")
+    pa.pa_multi_query_attention(out, q, case.k_cache, case.v_cache,
+                                case.block_tables, case.context_lens,
+                                case.query_start_loc, 30, 30, case.scale,
+                                error_flags=flags)
+    torch.cuda.synchronize()
+    assert int(flags.item()) & pa.PA_DEVERR_QUERY_LEN
