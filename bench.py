@@ -60,10 +60,24 @@ def attention_bytes(case, seqs=None) -> int:
     B = len(lens)
     uniq = case.unique_tokens if seqs is None else int(lens.sum())
     kv = uniq * 2 * w.num_kv_heads * w.head_size * 2
-    q = B * w.num_heads * w.head_size * 2
-    out = B * w.num_heads * w.head_size * 4
+    nq = B if case.query_lens_np is None else int(
+        (case.query_lens_np if seqs is None else case.query_lens_np[seqs]).sum())
+    q = nq * w.num_heads * w.head_size * 2
+    out = nq * w.num_heads * w.head_size * 4
     tables = int((-(-lens // w.block_size)).sum()) * 4
     return kv + q + out + tables + B * 4
+
+
+def attention_flops(case) -> int:
+    """Dense flops of the attention: 4 * Hq * D per (query, visible token)
+    pair (QK^T and PV multiply-adds)."""
+    w = case.workload
+    if case.query_lens_np is None:
+        pairs = int(case.lens_np.sum())
+    else:
+        L, k = case.lens_np, case.query_lens_np
+        pairs = int((k * (L - k) + k * (k + 1) // 2).sum())
+    return pairs * 4 * w.num_heads * w.head_size
 
 
 def step_bytes(case) -> int:
@@ -112,6 +126,19 @@ def hbm_peak():
             return float(json.load(f)["hbm_gbs"]), "measured"
     except (OSError, KeyError, ValueError):
         return FALLBACK_HBM_GBS, "fallback"
+
+
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
+
+
+def tensor_peak():
+    """Dense bf16 TFLOP/s for a kernel timed inside a long loop (sustained)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback"
 
 
 # ---------------------------------------------------------------- clocks
@@ -210,8 +237,10 @@ class Step:
         self.pa = pa
         self.case = case
         w = case.workload
-        B, Hq, D = case.q.shape
-        self.out = torch.empty(B, Hq, D, dtype=torch.float32, device=case.q.device)
+        B = w.num_seqs
+        _, Hq, D = case.q.shape
+        self.out = torch.empty(case.q.shape, dtype=torch.float32,
+                               device=case.q.device)
         self.maxlen = case.max_context_len
         self.partition = pa.pa_decode_partition_size(
             B, Hq, w.num_kv_heads, D, w.block_size, self.maxlen, partition_size)
@@ -234,6 +263,12 @@ class Step:
 
     def attention(self):
         c = self.case
+        if c.query_start_loc is not None:
+            self.pa.pa_multi_query_attention(
+                self.out, c.q, c.k_cache, c.v_cache, c.block_tables,
+                c.context_lens, c.query_start_loc, self.maxlen,
+                int(c.query_lens_np.max()), c.scale, error_flags=self.flags)
+            return
         self.pa.pa_decode_attention(
             self.out, c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens,
             self.maxlen, c.scale, partition_size=self.partition_arg,
@@ -297,6 +332,7 @@ def run_gpu(args):
     # e2e: host buffers through the public API
     e2e = None if args.kernel_only else run_e2e(case, step, args, dist, dev)
 
+
     ms_total = max_over_ranks(dist, ms_total, dev)
     attn_ms_max = max_over_ranks(dist, attn_ms, dev)
     sb = step_bytes(case)
@@ -304,12 +340,31 @@ def run_gpu(args):
     ms_step = ms_total / K
     value = world * sb / (ms_step * 1e-3) / 1e9
     peak, peak_kind = hbm_peak()
+    tpeak, tpeak_kind = tensor_peak()
+    flops = attention_flops(case)
+    ridge = tpeak * 1e12 / (peak * 1e9)          # flop per byte
+    tensor_bound = flops / ab > ridge
     achieved = ab / (attn_ms_max * 1e-3) / 1e9
+    achieved_tflops = flops / (attn_ms_max * 1e-3) / 1e12
     traffic = read_traffic(args.workload)
+    if tensor_bound:
+        roof = {"bound": "tensor", "achieved": round(achieved_tflops, 1),
+                "peak": tpeak,
+                "peak_source": f"{tpeak_kind} (MEASURED_PEAKS.json bf16_tflops_sustained)",
+                "unit": "TFLOP/s", "frac": round(achieved_tflops / tpeak, 4)}
+    else:
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+                               if peak_kind == "measured" else "fallback 6.65 TB/s",
+                "unit": "GB/s", "frac": round(achieved / peak, 4)}
+    kernel_name = ("paged_multi_query_kernel" if case.query_start_loc is not None
+                   else "paged_decode_kernel" +
+                   (" + reduce" if step.partition < case.max_context_len else ""))
 
     result = None
     if rank == 0:
-        cpu = cpu_baseline(args) if world == 1 and not args.kernel_only else None
+        cpu = (cpu_baseline(args) if world == 1 and not args.kernel_only
+               and case.query_start_loc is None else None)
         clocks = clk.summary()
         result = {
             "metric": METRIC,
@@ -335,30 +390,30 @@ def run_gpu(args):
                 "unique_kv_tokens": case.unique_tokens,
                 "partition_size": step.partition,
                 "step": ("copy_blocks + " if case.copy_pairs.shape[0] else "") +
-                        "reshape_and_cache + paged_decode_attention",
+                        "reshape_and_cache + " +
+                        ("paged_multi_query_attention" if case.query_start_loc is not None
+                         else "paged_decode_attention"),
+                "query_tokens_per_seq": (1 if case.query_lens_np is None
+                                         else w.query_len),
                 "l2": "no flush: inputs larger than L2 (KV pool "
                       f"{2 * case.k_cache.numel() * 2 / 1e9:.2f} GB > 126 MB)",
                 "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             },
-            "seq_tokens_per_s": round(world * w.num_seqs / (ms_step * 1e-3), 1),
+            "seq_tokens_per_s": round(world * (w.num_seqs if case.query_lens_np is None else int(case.query_lens_np.sum())) / (ms_step * 1e-3), 1),
             "context_tokens_per_s": round(world * case.logical_tokens / (ms_step * 1e-3), 1),
             "pct_hbm_peak": round(100 * value / (world * peak), 2),
             "step_bytes": sb,
             "in_run_copy_gbs": None if copy_best is None else round(copy_best, 1),
-            "roofline": {
-                "kernel": "paged_decode_kernel" + (" + reduce" if step.partition < case.max_context_len else ""),
-                "bound": "hbm",
-                "achieved": round(achieved, 1),
-                "peak": peak,
-                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s",
-                "unit": "GB/s",
-                "frac": round(achieved / peak, 4),
-                "frac_of_in_run_copy": (None if copy_best is None
-                                        else round(achieved / copy_best, 4)),
-                "traffic": traffic,
-                "algorithmic_bytes_per_launch": ab,
-                "avg_launch_ms": round(attn_ms_max, 5),
-            },
+            "roofline": dict(
+                kernel=kernel_name, **roof,
+                frac_of_in_run_copy=(None if copy_best is None or tensor_bound
+                                     else round(achieved / copy_best, 4)),
+                traffic=traffic,
+                algorithmic_bytes_per_launch=ab,
+                flops_per_launch=flops,
+                achieved_gbs=round(achieved, 1),
+                achieved_tflops=round(achieved_tflops, 2),
+                avg_launch_ms=round(attn_ms_max, 5)),
             "e2e": e2e,
             "gpu_launches": int(launches),
             "device_error_flags": flags,
@@ -381,7 +436,8 @@ def run_e2e(case, step, args, dist, dev):
     import paged_kv_cache_435_b200 as pa
     c = case
     names = ["q", "new_key", "new_value", "slot_mapping", "block_tables",
-             "context_lens"] + (["copy_pairs"] if c.copy_pairs.shape[0] else [])
+             "context_lens"] + (["copy_pairs"] if c.copy_pairs.shape[0] else []) \
+        + (["query_start_loc"] if c.query_start_loc is not None else [])
     host_in = {n: getattr(c, n).cpu().pin_memory() for n in names}
     dev_in = [{n: torch.empty_like(getattr(c, n)) for n in names} for _ in range(2)]
     outs = [torch.empty_like(step.out) for _ in range(2)]
@@ -416,12 +472,19 @@ def run_e2e(case, step, args, dist, dev):
         pa.pa_reshape_and_cache(d["new_key"], d["new_value"], c.k_cache,
                                 c.v_cache, d["slot_mapping"],
                                 error_flags=step.flags, stream=comp)
-        pa.pa_decode_attention(outs[b], d["q"], c.k_cache, c.v_cache,
-                               d["block_tables"], d["context_lens"],
-                               step.maxlen, c.scale,
-                               partition_size=step.partition_arg,
-                               workspace=step.ws, error_flags=step.flags,
-                               stream=comp)
+        if c.query_start_loc is not None:
+            pa.pa_multi_query_attention(
+                outs[b], d["q"], c.k_cache, c.v_cache, d["block_tables"],
+                d["context_lens"], d["query_start_loc"], step.maxlen,
+                int(c.query_lens_np.max()), c.scale, error_flags=step.flags,
+                stream=comp)
+        else:
+            pa.pa_decode_attention(outs[b], d["q"], c.k_cache, c.v_cache,
+                                   d["block_tables"], d["context_lens"],
+                                   step.maxlen, c.scale,
+                                   partition_size=step.partition_arg,
+                                   workspace=step.ws, error_flags=step.flags,
+                                   stream=comp)
         in_free[b].record(comp)
         out_ready[b].record(comp)
 

@@ -56,6 +56,9 @@ class Workload:
     samples: int = 0
     prefix_tokens: int = 0
     tail_max: int = 0
+    # multi-query workloads: the last query_len tokens of each context are
+    # the step's queries (0: decode, one query per sequence)
+    query_len: int = 0
     description: str = ""
 
     @property
@@ -90,6 +93,17 @@ WORKLOADS = {
         "long_skew_bs32", 5, 32, 32, 8, 128, 32, "skew:131072;64,1024",
         partition_size=512,
         description="as long_skew_bs16 with bs=32"),
+    "spec_verify_70b_b256": Workload(
+        "spec_verify_70b_b256", 6, 256, 64, 8, 128, 16, "uniform:256,4096",
+        query_len=4,
+        description="speculative verification of 4 draft tokens per sequence "
+                    "on the batch-256 GQA layer (64q/8kv, D=128, bs=16, "
+                    "L~U[256,4096])"),
+    "chunked_prefill_70b": Workload(
+        "chunked_prefill_70b", 7, 16, 64, 8, 128, 16, "uniform:1024,4096",
+        query_len=512,
+        description="512-token prefill chunks of 16 sequences (64q/8kv, "
+                    "D=128, bs=16, L~U[1024,4096] including the chunk)"),
 }
 
 
@@ -282,6 +296,13 @@ def make_case(name: str, device="cpu", pool_device=None,
         lens = lens[:num_seqs]
         w = dataclasses.replace(w, num_seqs=len(lens),
                                 name=f"{w.name}_first{len(lens)}")
+    if w.query_len > 0:
+        qlens = np.minimum(lens, w.query_len)
+        case = multi_query_case(w.num_seqs, w.num_heads, w.num_kv_heads,
+                                w.head_size, w.block_size, lens, qlens,
+                                seed=2000 + w.wid, device=device,
+                                pool_device=pool_device, name=w.name)
+        return dataclasses.replace(case, workload=w)
     return build_case(w, lens, device=device, pool_device=pool_device,
                       seed=None, rng=rng)
 
