@@ -632,6 +632,52 @@ def run_reference(args):
     }
 
 
+def run_swap(args):
+    """swap_blocks bandwidth: 4096 blocks of the batch-256 GQA pool shape
+    (K and V, 32 KB each) to pinned host memory and back, against a plain
+    pinned-memory copy of the same bytes in each direction."""
+    import paged_kv_cache_435_b200 as pa
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    nb_gpu, n, shape = 8192, 4096, (16, 8, 128)
+    gen = torch.Generator(device=dev).manual_seed(5)
+    gpu = [torch.randn(nb_gpu, *shape, device=dev, generator=gen).to(torch.bfloat16)
+           for _ in range(2)]
+    cpu = [torch.empty(n, *shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    rng = np.random.default_rng(9)
+    src = rng.permutation(nb_gpu)[:n]
+    out_pairs = torch.from_numpy(np.stack([src, np.arange(n)], 1).astype(np.int64)).to(dev)
+    in_pairs = torch.from_numpy(np.stack([np.arange(n), src], 1).astype(np.int64)).to(dev)
+    nbytes = 2 * n * gpu[0][0].numel() * 2
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / args.steps
+
+    ms_out = timed(lambda: pa.pa_swap_blocks(gpu, cpu, out_pairs))
+    ms_in = timed(lambda: pa.pa_swap_blocks(cpu, gpu, in_pairs))
+    flat_g = torch.empty(nbytes // 2, dtype=torch.bfloat16, device=dev)
+    flat_h = torch.empty(nbytes // 2, dtype=torch.bfloat16).pin_memory()
+    ms_d2h = timed(lambda: flat_h.copy_(flat_g, non_blocking=True))
+    ms_h2d = timed(lambda: flat_g.copy_(flat_h, non_blocking=True))
+    gbs = lambda ms: round(nbytes / (ms * 1e-3) / 1e9, 1)  # noqa: E731
+    return {"metric": "swap_blocks GB/s (GPU <-> pinned host)",
+            "blocks": n, "bytes_per_direction": nbytes,
+            "swap_out_gbs": gbs(ms_out), "swap_in_gbs": gbs(ms_in),
+            "pinned_copy_d2h_gbs": gbs(ms_d2h), "pinned_copy_h2d_gbs": gbs(ms_h2d),
+            "frac_out": round(ms_d2h / ms_out, 4), "frac_in": round(ms_h2d / ms_in, 4),
+            "steps": args.steps, "warmup": args.warmup}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -642,13 +688,18 @@ def main():
     ap.add_argument("--partition", type=int, default=None)
     ap.add_argument("--seqs", type=int, default=None,
                     help="keep only the first N sequences of the workload")
+    ap.add_argument("--swap", action="store_true",
+                    help="measure swap_blocks bandwidth instead (own JSON line)")
     ap.add_argument("--kernel-only", action="store_true",
                     help="time the device step only: no e2e leg, no in-run "
                          "copy peak, no CPU baseline (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    res = run_reference(args) if args.impl == "reference" else run_gpu(args)
+    if args.swap:
+        res = run_swap(args)
+    else:
+        res = run_reference(args) if args.impl == "reference" else run_gpu(args)
     if res is not None:
         print(json.dumps(res), flush=True)
 

@@ -217,6 +217,36 @@ int pa_multi_query_attention(float* out, const void* q, const void* k_cache,
                              float scale, int* error_flags,
                              pa_stream_t stream);
 
+/*
+ * pa_swap_blocks - move whole KV blocks between pools in different memories:
+ * the swapping form of preemption, where evicted blocks go to CPU RAM and
+ * come back when the request resumes ("vLLM: Anatomy and Mechanisms of
+ * High-Throughput LLM Inference", "Preemption and Recovery"; "vLLM
+ * Internals", "The Block Manager").  For each pair p and cache c:
+ *     dst_caches[c][dst] = src_caches[c][src],  (src, dst) = block_mapping[p]
+ * each block block_bytes bytes (2 * block_size * num_kv_heads * head_size for
+ * one K or V pool of bf16), bit-exact.  One kernel serves both directions:
+ * every pointer may be device memory or pinned (page-locked, registered) host
+ * memory, which the GPU reads and writes directly.
+ *
+ *   src_caches, dst_caches  HOST arrays of num_caches pointers (e.g. the K and
+ *                           V pools of every layer), 16-byte aligned;
+ *                           source pools hold src_num_blocks blocks,
+ *                           destination pools dst_num_blocks.
+ *   block_mapping           int64 [num_pairs][2], device or pinned host.
+ *   block_bytes             multiple of 16.
+ *   error_flags             nullable; PA_DEVERR_COPY_PAIR on an id out of
+ *                           range (that pair is skipped).
+ * Pageable (unregistered) host memory is rejected with PA_ERR_INVALID_ARG.
+ * No destination block may appear twice.  Returns PA_OK or a negative
+ * pa_status.
+ */
+int pa_swap_blocks(const void* const* src_caches, void* const* dst_caches,
+                   int num_caches, const int64_t* block_mapping, int num_pairs,
+                   int64_t block_bytes, int64_t src_num_blocks,
+                   int64_t dst_num_blocks, int* error_flags,
+                   pa_stream_t stream);
+
 /* Capacity, in bytes, of the workspace built into the library for
  * pa_decode_attention_static_ws (32 MiB per GPU that uses the library). */
 #define PA_STATIC_WORKSPACE_BYTES (32u << 20)

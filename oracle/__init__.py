@@ -79,6 +79,8 @@ def _load():
                 p, p, p, p, p, i32, p, p, i32, i32, i32, i32, i32, i32, dbl,
                 i32]
             lib.oracle_paged_multi_query_attention.restype = i32
+            lib.oracle_swap_blocks.argtypes = [p, p, i32, p, i32, i64, i64, i64]
+            lib.oracle_swap_blocks.restype = i32
             _lib = lib
     return _lib
 
@@ -214,3 +216,25 @@ def copy_blocks(k_caches_bits: list, v_caches_bits: list,
                                 ctypes.cast(varr, ctypes.c_void_p), L,
                                 _ptr(bm), bm.shape[0], NB, bs, Hkv, D)
     _check(rc, "copy_blocks")
+
+
+def swap_blocks(src_caches: list, dst_caches: list, block_mapping) -> None:
+    """In-place whole-block copies src_caches[c][src] -> dst_caches[c][dst]
+    for each (src, dst) pair; each cache a C-contiguous array whose first
+    dimension is the block index (pools may differ in block count)."""
+    lib = _load()
+    n = len(src_caches)
+    if n == 0 or len(dst_caches) != n:
+        raise ValueError("need matching, non-empty source and destination lists")
+    block_bytes = src_caches[0][0].nbytes
+    for a in list(src_caches) + list(dst_caches):
+        if not a.flags.c_contiguous or a[0].nbytes != block_bytes:
+            raise ValueError("every cache must be C-contiguous with equal blocks")
+    bm = _arr(block_mapping, np.int64).reshape(-1, 2)
+    sarr = (ctypes.c_void_p * n)(*[a.ctypes.data for a in src_caches])
+    darr = (ctypes.c_void_p * n)(*[a.ctypes.data for a in dst_caches])
+    rc = lib.oracle_swap_blocks(ctypes.cast(sarr, ctypes.c_void_p),
+                                ctypes.cast(darr, ctypes.c_void_p), n, _ptr(bm),
+                                bm.shape[0], block_bytes, src_caches[0].shape[0],
+                                dst_caches[0].shape[0])
+    _check(rc, "swap_blocks")

@@ -407,3 +407,28 @@ int oracle_paged_multi_query_attention(
     pthread_mutex_destroy(&job.lock);
     return job.status;
 }
+
+/* ------------------------------------------------------------------------ */
+/* swap_blocks                                                                */
+/* ------------------------------------------------------------------------ */
+/* Preemption by swapping: evicted KV blocks are moved to CPU RAM and brought
+ * back when the request is rescheduled ("vLLM: Anatomy and Mechanisms of
+ * High-Throughput LLM Inference", "Preemption and Recovery"; "vLLM
+ * Internals", "The Block Manager").  For each pair (src, dst) and each cache
+ * c: dst_caches[c] block dst = src_caches[c] block src, block_bytes bytes. */
+int oracle_swap_blocks(const uint8_t* const* src_caches, uint8_t* const* dst_caches,
+                       int num_caches, const int64_t* block_mapping, int num_pairs,
+                       int64_t block_bytes, int64_t src_num_blocks,
+                       int64_t dst_num_blocks) {
+    if (num_caches <= 0 || num_pairs < 0 || block_bytes <= 0) return ORACLE_ERR_ARG;
+    for (int p = 0; p < num_pairs; ++p) {
+        int64_t src = block_mapping[2 * p];
+        int64_t dst = block_mapping[2 * p + 1];
+        if (src < 0 || src >= src_num_blocks || dst < 0 || dst >= dst_num_blocks)
+            return ORACLE_ERR_RANGE;
+        for (int c = 0; c < num_caches; ++c)
+            memcpy(dst_caches[c] + dst * block_bytes,
+                   src_caches[c] + src * block_bytes, (size_t)block_bytes);
+    }
+    return ORACLE_OK;
+}

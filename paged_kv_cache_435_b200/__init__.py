@@ -10,7 +10,9 @@ entry points, bound here under the same names:
   long contexts);
 * ``pa_copy_blocks``: copy-on-write block copies;
 * ``pa_multi_query_attention``: k causal query tokens per sequence (chunked
-  prefill chunks, speculative-decoding verification).
+  prefill chunks, speculative-decoding verification);
+* ``pa_swap_blocks``: whole-block moves between GPU and pinned CPU pools
+  (preemption by swapping).
 
 ``inputs`` builds seeded synthetic workloads.  The library is loaded lazily on
 first use and its absence raises; nothing here computes on the CPU.
@@ -22,4 +24,4 @@ from ._native import (  # noqa: F401
     library_path,
     pa_copy_blocks, pa_decode_attention, pa_decode_partition_size,
     pa_decode_workspace_size, pa_launch_count, pa_multi_query_attention,
-    pa_reshape_and_cache, raw, status_string)
+    pa_reshape_and_cache, pa_swap_blocks, raw, status_string)

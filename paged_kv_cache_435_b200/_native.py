@@ -77,6 +77,8 @@ def raw():
             p, p, p, p, p, i32, p, i32, p, i32, i32, i32, i32, i32, i32, i32,
             f32, p, p]
         lib.pa_multi_query_attention.restype = i32
+        lib.pa_swap_blocks.argtypes = [p, p, i32, p, i32, i64, i64, i64, p, p]
+        lib.pa_swap_blocks.restype = i32
         lib.pa_copy_blocks.argtypes = [p, p, i32, p, i32, i32, i32, i32, i32,
                                        p, p]
         lib.pa_copy_blocks.restype = i32
@@ -232,6 +234,40 @@ def pa_multi_query_attention(out, q, k_cache, v_cache, block_tables,
         _ptr(query_start_loc), int(max_query_len), B, Hq, Hkv, D, bs, NB,
         float(scale), _ptr(error_flags), _stream(stream))
     return _check(rc, "pa_multi_query_attention")
+
+
+def pa_swap_blocks(src_caches: Sequence, dst_caches: Sequence, block_mapping,
+                   error_flags=None, stream=None) -> int:
+    """Move whole blocks src_caches[c][src] -> dst_caches[c][dst] for each
+    (src, dst) row of block_mapping (int64 [N,2]).  Each cache is a
+    contiguous tensor whose first dimension is the block index, on the GPU or
+    in pinned host memory (pin_memory()); block_mapping likewise."""
+    import torch
+    n = len(src_caches)
+    if n == 0 or len(dst_caches) != n:
+        raise ValueError("need matching, non-empty source and destination lists")
+    block_bytes = src_caches[0][0].numel() * src_caches[0].element_size()
+    for t in list(src_caches) + list(dst_caches):
+        if not isinstance(t, torch.Tensor) or not t.is_contiguous():
+            raise ValueError("caches must be contiguous tensors")
+        if not (t.is_cuda or t.is_pinned()):
+            raise ValueError("host caches must be pinned (pin_memory())")
+        if t[0].numel() * t.element_size() != block_bytes:
+            raise ValueError("every cache must have the same block size")
+    if block_mapping.dtype != torch.int64 or block_mapping.dim() != 2 or \
+            block_mapping.shape[1] != 2 or not block_mapping.is_contiguous():
+        raise ValueError("block_mapping must be a contiguous int64 [N,2] tensor")
+    if not (block_mapping.is_cuda or block_mapping.is_pinned()):
+        raise ValueError("block_mapping must be on the GPU or pinned")
+    sarr = (ctypes.c_void_p * n)(*[t.data_ptr() for t in src_caches])
+    darr = (ctypes.c_void_p * n)(*[t.data_ptr() for t in dst_caches])
+    rc = raw().pa_swap_blocks(ctypes.cast(sarr, ctypes.c_void_p),
+                              ctypes.cast(darr, ctypes.c_void_p), n,
+                              _ptr(block_mapping), block_mapping.shape[0],
+                              block_bytes, src_caches[0].shape[0],
+                              dst_caches[0].shape[0], _ptr(error_flags),
+                              _stream(stream))
+    return _check(rc, "pa_swap_blocks")
 
 
 def pa_copy_blocks(k_caches: Sequence, v_caches: Sequence, block_mapping,

@@ -17,9 +17,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpagedattn.so")
 SOURCES = ["pa_api.cu", "pa_decode.cu", "pa_multi_query.cu", "pa_cache_ops.cu",
-           "pa_static_ws.cu"]
+           "pa_swap.cu", "pa_static_ws.cu"]
 HEADERS = ["pa_common.cuh", "pa_decode.cuh", "pa_multi_query.cuh",
-           "pa_cache_ops.cuh"]
+           "pa_cache_ops.cuh", "pa_swap.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

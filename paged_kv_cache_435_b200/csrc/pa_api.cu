@@ -11,6 +11,7 @@
 #include "pa_common.cuh"
 #include "pa_decode.cuh"
 #include "pa_multi_query.cuh"
+#include "pa_swap.cuh"
 
 namespace pa {
 
@@ -25,6 +26,17 @@ constexpr int kMaxGridYZ = 65535;
 
 bool aligned16(const void* p) {
     return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+// True when the GPU can address `p` (device, pinned host or managed memory).
+bool device_accessible(const void* p) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeHost ||
+           a.type == cudaMemoryTypeManaged;
 }
 
 int round_up(int x, int m) { return ((x + m - 1) / m) * m; }
@@ -275,6 +287,34 @@ int pa_multi_query_attention(float* out, const void* q, const void* k_cache,
     p.scale_log2 = pa::mq_log2e_scale(scale);
     cudaError_t e = pa::launch_paged_multi_query(
         p, head_size, block_size, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_swap_blocks(const void* const* src_caches, void* const* dst_caches,
+                   int num_caches, const int64_t* block_mapping, int num_pairs,
+                   int64_t block_bytes, int64_t src_num_blocks,
+                   int64_t dst_num_blocks, int* error_flags,
+                   pa_stream_t stream) {
+    if (num_caches <= 0 || num_pairs < 0 || block_bytes <= 0 ||
+        block_bytes % 16 != 0 || src_num_blocks <= 0 || dst_num_blocks <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (!src_caches || !dst_caches) return PA_ERR_INVALID_ARG;
+    if (num_pairs == 0) return PA_OK;
+    if (!block_mapping || (reinterpret_cast<uintptr_t>(block_mapping) & 7u) ||
+        !pa::device_accessible(block_mapping))
+        return PA_ERR_INVALID_ARG;
+    for (int c = 0; c < num_caches; ++c) {
+        if (!src_caches[c] || !dst_caches[c]) return PA_ERR_INVALID_ARG;
+        if (!pa::aligned16(src_caches[c]) || !pa::aligned16(dst_caches[c]))
+            return PA_ERR_INVALID_ARG;
+        if (!pa::device_accessible(src_caches[c]) ||
+            !pa::device_accessible(dst_caches[c]))
+            return PA_ERR_INVALID_ARG;
+    }
+    cudaError_t e = pa::launch_swap_blocks(
+        src_caches, dst_caches, num_caches, block_mapping, num_pairs,
+        block_bytes, src_num_blocks, dst_num_blocks, error_flags,
+        reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

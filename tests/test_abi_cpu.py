@@ -160,3 +160,32 @@ def test_product_package_does_not_reach_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text
                 assert "pa_oracle" not in text, f
+
+
+def test_swap_blocks_host_validation(lib):
+    arr = (ctypes.c_void_p * 1)(FAKE)
+    a = ctypes.cast(arr, ctypes.c_void_p)
+    f = lib.pa_swap_blocks
+    assert f(a, a, 0, FAKE, 1, 4096, 4, 4, None, None) == nat.PA_ERR_INVALID_ARG
+    assert f(a, a, 1, FAKE, 1, 4100, 4, 4, None, None) == nat.PA_ERR_INVALID_ARG
+    assert f(a, a, 1, FAKE, -1, 4096, 4, 4, None, None) == nat.PA_ERR_INVALID_ARG
+    assert f(a, a, 1, FAKE, 1, 4096, 0, 4, None, None) == nat.PA_ERR_INVALID_ARG
+    assert f(a, a, 1, None, 0, 4096, 4, 4, None, None) == nat.PA_OK
+    assert f(None, a, 1, FAKE, 1, 4096, 4, 4, None, None) == nat.PA_ERR_INVALID_ARG
+
+
+def test_multi_query_host_validation(lib):
+    f = lib.pa_multi_query_attention
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, 8, FAKE, 100, FAKE, 4, 2, 8, 2, 128,
+            16, 64, 0.1, None, None]
+    def call(**kw):
+        a = list(args)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return f(*a)
+    assert call(a12=4, a11=6) == nat.PA_ERR_INVALID_ARG        # Hq % Hkv
+    assert call(a9=101) == nat.PA_ERR_INVALID_ARG              # mq > max len
+    assert call(a7=129) == nat.PA_ERR_INVALID_ARG              # > MB*bs
+    assert call(a13=96) == nat.PA_ERR_UNSUPPORTED
+    assert call(a8=None) == nat.PA_ERR_INVALID_ARG
+    assert call(a9=0) == nat.PA_OK

@@ -344,6 +344,36 @@ def test_copy_blocks_rejects_out_of_range():
 
 
 # --------------------------------------------------------------------------
+# swap_blocks
+# --------------------------------------------------------------------------
+def test_swap_blocks_matches_numpy_and_round_trips():
+    rng = np.random.default_rng(11)
+    gpu = [rng.integers(0, 65535, (12, 16, 2, 8), dtype=np.uint16) for _ in range(4)]
+    cpu = [np.zeros((5, 16, 2, 8), dtype=np.uint16) for _ in range(4)]
+    out_pairs = np.array([[3, 0], [7, 4], [11, 2]], dtype=np.int64)
+    expect = [c.copy() for c in cpu]
+    for e, g in zip(expect, gpu):
+        e[out_pairs[:, 1]] = g[out_pairs[:, 0]]
+    oracle.swap_blocks(gpu, cpu, out_pairs)                    # swap out
+    for a, b in zip(cpu, expect):
+        np.testing.assert_array_equal(a, b)
+    back = [np.zeros_like(g) for g in gpu]
+    in_pairs = out_pairs[:, ::-1].copy()
+    in_pairs[:, 1] = [1, 5, 9]                                 # new block ids
+    oracle.swap_blocks(cpu, back, in_pairs)                    # swap in
+    for b, g in zip(back, gpu):
+        np.testing.assert_array_equal(b[[1, 5, 9]], g[[3, 7, 11]])
+        assert not b[[0, 2, 3]].any()
+
+
+def test_swap_blocks_rejects_out_of_range():
+    a = [np.zeros((4, 16), np.uint16)]
+    b = [np.zeros((2, 16), np.uint16)]
+    with pytest.raises(ValueError):
+        oracle.swap_blocks(a, b, np.array([[3, 2]], np.int64))
+
+
+# --------------------------------------------------------------------------
 # numbers the pages print
 # --------------------------------------------------------------------------
 def _golden_rows(name):

@@ -50,6 +50,9 @@ MUTANTS = {
         "const uint16_t* qv = job->q + ((int64_t)(q0) * job->num_heads + h) * D;"),
     "query_count_off_by_one": ("const int k = job->query_start_loc[s + 1] - q0;",
                                "const int k = job->query_start_loc[s + 1] - q0 - 1;"),
+    "swap_direction_reversed": (
+        "memcpy(dst_caches[c] + dst * block_bytes,\n                   src_caches[c] + src * block_bytes, (size_t)block_bytes);",
+        "memcpy(dst_caches[c] + src * block_bytes,\n                   src_caches[c] + dst * block_bytes, (size_t)block_bytes);"),
     "copy_direction_swapped": (
         "int64_t src = block_mapping[2 * p];\n        int64_t dst = block_mapping[2 * p + 1];",
         "int64_t src = block_mapping[2 * p + 1];\n        int64_t dst = block_mapping[2 * p];"),
