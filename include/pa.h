@@ -73,7 +73,8 @@ typedef enum {
     PA_ERR_INVALID_ARG = -1, /* null pointer, bad size, misaligned buffer */
     PA_ERR_UNSUPPORTED = -2, /* valid but not implemented (head_size...) */
     PA_ERR_WORKSPACE = -3,   /* workspace missing or smaller than needed */
-    PA_ERR_CUDA = -4         /* the CUDA runtime reported a launch error */
+    PA_ERR_CUDA = -4,        /* the CUDA runtime reported a launch error */
+    PA_ERR_NO_BLOCKS = -5    /* the block manager has too few free blocks */
 } pa_status;
 
 /* Bits OR-ed into *error_flags by the kernels. */
@@ -246,6 +247,93 @@ int pa_swap_blocks(const void* const* src_caches, void* const* dst_caches,
                    int64_t block_bytes, int64_t src_num_blocks,
                    int64_t dst_num_blocks, int* error_flags,
                    pa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Host-side block manager (no GPU work; not thread-safe: one owner thread).
+ *
+ * It keeps the free block pool (a FIFO queue: freed blocks join the back,
+ * allocation takes the front), a block table per sequence, per-block
+ * reference counts for sharing, optional prefix caching and a CPU pool for
+ * swapping, and emits exactly the inputs the kernels above take: slot
+ * mappings for pa_reshape_and_cache, block tables for the attention calls,
+ * (src, dst) pairs for pa_copy_blocks and pa_swap_blocks.  Method: "vLLM:
+ * Anatomy and Mechanisms of High-Throughput LLM Inference", sections
+ * "Block-Level Management", "Memory Sharing via Copy-on-Write (CoW)",
+ * "Preemption and Recovery", "Prefix Caching"; "Inside vLLM: Anatomy of a
+ * High-Throughput LLM Inference System", KV-cache manager (free_block_queue,
+ * allocate_slots); "vLLM Internals", "The Block Manager".
+ * ---------------------------------------------------------------------- */
+typedef struct pa_block_manager pa_block_manager;
+
+/* Chained hash of one block for prefix caching: FNV-1a over the block's
+ * token ids started from the parent block's hash (pa_prefix_hash_seed() for
+ * the first block) and mixed with it again. */
+uint64_t pa_prefix_block_hash(uint64_t parent_hash, const int32_t* token_ids,
+                              int num_tokens);
+uint64_t pa_prefix_hash_seed(void);
+
+/* A manager over num_blocks GPU blocks and num_cpu_blocks CPU blocks of
+ * block_size tokens.  NULL on bad arguments or allocation failure.  With
+ * enable_prefix_caching, every full block of a sequence whose token ids are
+ * known is registered under its chained hash; a freed registered block stays
+ * reusable until the allocator hands it out again (oldest first). */
+pa_block_manager* pa_bm_create(int num_blocks, int num_cpu_blocks,
+                               int block_size, int enable_prefix_caching);
+void pa_bm_destroy(pa_block_manager* m);
+int pa_bm_num_free_blocks(const pa_block_manager* m);
+int pa_bm_num_free_cpu_blocks(const pa_block_manager* m);
+
+/* New sequence holding the prompt token_ids[0..num_tokens).  With prefix
+ * caching, leading full blocks whose chained hash and token ids match a
+ * registered block are shared instead of allocated; *num_cached_tokens (if
+ * non-NULL) gets their token count c.  slot_mapping (nullable, host,
+ * num_tokens - c entries) receives the slots of tokens c..num_tokens-1, the
+ * ones whose K/V the caller must write.  Returns the sequence id (>= 0),
+ * PA_ERR_NO_BLOCKS (nothing changed) or PA_ERR_INVALID_ARG. */
+int pa_bm_add_sequence(pa_block_manager* m, const int32_t* token_ids,
+                       int num_tokens, int64_t* slot_mapping,
+                       int* num_cached_tokens);
+
+/* New sequence sharing every block of `parent` (reference counts + 1):
+ * parallel sampling / beam branches.  Returns its id or a negative status. */
+int pa_bm_fork(pa_block_manager* m, int parent);
+
+/* Reserve slots for num_new_tokens tokens at the end of sequence seq_id:
+ * slot_mapping (host, num_new_tokens entries) gets their slots.  Blocks are
+ * allocated on demand; if the sequence's partial last block is shared, it is
+ * first replaced by a fresh copy and the pair (old, new) is written to
+ * cow_pairs (host int64 [cow_capacity][2]) for pa_copy_blocks, with the count
+ * in *num_cow.  token_ids (nullable) feed prefix caching; once a call passes
+ * NULL, the sequence's later blocks are not registered.  Returns PA_OK,
+ * PA_ERR_NO_BLOCKS (nothing changed) or PA_ERR_INVALID_ARG. */
+int pa_bm_append_slots(pa_block_manager* m, int seq_id, int num_new_tokens,
+                       const int32_t* token_ids, int64_t* slot_mapping,
+                       int64_t* cow_pairs, int cow_capacity, int* num_cow);
+
+/* Finish a sequence: its blocks' reference counts drop, unshared blocks go
+ * back to the free pool.  Returns PA_OK or PA_ERR_INVALID_ARG. */
+int pa_bm_free_sequence(pa_block_manager* m, int seq_id);
+
+/* Tokens held by the sequence, or a negative status. */
+int pa_bm_seq_len(const pa_block_manager* m, int seq_id);
+
+/* Copy the sequence's block table (physical ids, logical order) into out
+ * (nullable, capacity entries).  Returns the number of blocks. */
+int pa_bm_block_table(const pa_block_manager* m, int seq_id, int32_t* out,
+                      int capacity);
+
+/* Reference count of a GPU block (0 = free). */
+int pa_bm_block_refcount(const pa_block_manager* m, int block);
+
+/* Preemption by swapping: move every block of an unshared sequence to the CPU
+ * pool (pa_bm_swap_out) or back to fresh GPU blocks (pa_bm_swap_in).  pairs
+ * (host int64 [capacity][2]) receives the (src, dst) pairs for
+ * pa_swap_blocks.  Returns the pair count or a negative status
+ * (PA_ERR_INVALID_ARG if a block is shared or the sequence is already there). */
+int pa_bm_swap_out(pa_block_manager* m, int seq_id, int64_t* pairs,
+                   int capacity);
+int pa_bm_swap_in(pa_block_manager* m, int seq_id, int64_t* pairs,
+                  int capacity);
 
 /* Capacity, in bytes, of the workspace built into the library for
  * pa_decode_attention_static_ws (32 MiB per GPU that uses the library). */

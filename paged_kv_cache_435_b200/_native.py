@@ -20,6 +20,7 @@ PA_ERR_INVALID_ARG = -1
 PA_ERR_UNSUPPORTED = -2
 PA_ERR_WORKSPACE = -3
 PA_ERR_CUDA = -4
+PA_ERR_NO_BLOCKS = -5
 
 PA_DEVERR_BLOCK_ID = 0x1
 PA_DEVERR_CONTEXT_LEN = 0x2
