@@ -3,6 +3,8 @@
 // launch; a failed check enqueues nothing.
 #include <atomic>
 #include <cmath>
+#include <cstdlib>
+#include <cstring>
 #include <cstddef>
 #include <cstdint>
 
@@ -286,8 +288,19 @@ int pa_multi_query_attention(float* out, const void* q, const void* k_cache,
     p.num_blocks = num_blocks;
     p.group = G;
     p.scale_log2 = pa::mq_log2e_scale(scale);
-    cudaError_t e = pa::launch_paged_multi_query(
-        p, head_size, block_size, reinterpret_cast<cudaStream_t>(stream));
+    // Kernel choice: the tcgen05 kernel for 128-row tiles (prefill chunks),
+    // the mma.sync kernel for few rows per sequence (speculative verify).
+    // PA_MULTI_QUERY_KERNEL=mma|tc overrides the choice (tests, benchmarks).
+    bool use_tc = pa::multi_query_tc_eligible(head_size, max_query_len, G);
+    if (const char* force = std::getenv("PA_MULTI_QUERY_KERNEL")) {
+        if (std::strcmp(force, "mma") == 0) use_tc = false;
+        if (std::strcmp(force, "tc") == 0 && head_size == 128) use_tc = true;
+    }
+    cudaError_t e = use_tc
+        ? pa::launch_paged_multi_query_tc(p, block_size,
+                                          reinterpret_cast<cudaStream_t>(stream))
+        : pa::launch_paged_multi_query(p, head_size, block_size,
+                                       reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

@@ -34,4 +34,10 @@ int multi_query_row_tiles(int max_query_len, int group);
 cudaError_t launch_paged_multi_query(const MultiQueryParams& p, int head_size,
                                      int block_size, cudaStream_t stream);
 
+// tcgen05 kernel for 128-row tiles (pa_multi_query_tc.cu): head_size 128 and
+// at least 128 (query token, head) rows per sequence.
+bool multi_query_tc_eligible(int head_size, int max_query_len, int group);
+cudaError_t launch_paged_multi_query_tc(const MultiQueryParams& p,
+                                        int block_size, cudaStream_t stream);
+
 }  // namespace pa
