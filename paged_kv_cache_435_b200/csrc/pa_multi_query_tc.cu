@@ -465,10 +465,13 @@ paged_multi_query_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
             tmem_ld32(tmem + lane_off + st * kTok, sraw[0]);
             tmem_ld32(tmem + lane_off + st * kTok + 32, sraw[1]);
             tmem_wait_ld();
+            // Raw logits; the scale (log2 domain) folds into one FFMA per
+            // exponent below, and the row max is taken on raw values
+            // (scale > 0 preserves order).
             float sv[64];
             const int ctok = c * kTok;
 #pragma unroll
-            for (int i = 0; i < 64; ++i) sv[i] = __uint_as_float(sraw[i >> 5][i & 31]) * sl2;
+            for (int i = 0; i < 64; ++i) sv[i] = __uint_as_float(sraw[i >> 5][i & 31]);
             if (ctok + kTok - 1 > min_lim) {
 #pragma unroll
                 for (int i = 0; i < 64; ++i)
@@ -479,8 +482,8 @@ paged_multi_query_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
             for (int i = 0; i < 8; ++i) mx8[i] = sv[i];
 #pragma unroll
             for (int i = 8; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
-            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            const float mx = sl2 * fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             if (c == 0) {
                 m_ref = mx;
             } else if (__any_sync(0xffffffffu, mx > m_ref + kRescaleThreshold)) {
@@ -508,21 +511,22 @@ paged_multi_query_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                 }
                 tmem_wait_st();
             }
-            // p and its bf16 split (truncation: hi keeps 8 significant bits,
-            // the residual another 8, so P carries ~16 bits into PV).
+            // p = 2^(scale*s - m) (masked logits give 2^-inf = 0) and its bf16
+            // split by truncation: the high half keeps 8 significant bits, the
+            // residual another 8, so P carries ~16 bits into PV.
             uint32_t hi[32], lo[32];
             float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            const float neg_m = -m_ref;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float a = sv[2 * i] == -INFINITY ? 0.f : exp2f(sv[2 * i] - m_ref);
-                const float b = sv[2 * i + 1] == -INFINITY ? 0.f : exp2f(sv[2 * i + 1] - m_ref);
+                const float a = exp2f(fmaf(sv[2 * i], sl2, neg_m));
+                const float b = exp2f(fmaf(sv[2 * i + 1], sl2, neg_m));
                 ps8[i & 7] += a + b;
-                const uint32_t ah = __float_as_uint(a) & 0xFFFF0000u;
-                const uint32_t bh = __float_as_uint(b) & 0xFFFF0000u;
-                const uint32_t al = __float_as_uint(a - __uint_as_float(ah));
-                const uint32_t bl = __float_as_uint(b - __uint_as_float(bh));
-                hi[i] = (ah >> 16) | bh;
-                lo[i] = (al >> 16) | (bl & 0xFFFF0000u);
+                const uint32_t ab = __float_as_uint(a), bb = __float_as_uint(b);
+                const float al = a - __uint_as_float(ab & 0xFFFF0000u);
+                const float bl = b - __uint_as_float(bb & 0xFFFF0000u);
+                hi[i] = __byte_perm(ab, bb, 0x7632);
+                lo[i] = __byte_perm(__float_as_uint(al), __float_as_uint(bl), 0x7632);
             }
             l_sum += ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) +
                      ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
