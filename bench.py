@@ -232,7 +232,7 @@ def max_over_ranks(dist, x: float, device) -> float:
 class Step:
     """Device buffers and the library calls of one decode step."""
 
-    def __init__(self, case, partition_size: int):
+    def __init__(self, case, partition_size: int, shared_prefix: bool = False):
         import paged_kv_cache_435_b200 as pa
         self.pa = pa
         self.case = case
@@ -245,9 +245,12 @@ class Step:
         self.partition = pa.pa_decode_partition_size(
             B, Hq, w.num_kv_heads, D, w.block_size, self.maxlen, partition_size)
         self.partition_arg = partition_size
-        nbytes = pa.pa_decode_workspace_size(B, Hq, w.num_kv_heads, D,
-                                             w.block_size, self.maxlen,
-                                             partition_size)
+        # Groups of sequences sharing prompt blocks: the shared-prefix call.
+        self.shared_prefix = shared_prefix and case.group_start is not None
+        size_fn = (pa.pa_shared_prefix_workspace_size if self.shared_prefix
+                   else pa.pa_decode_workspace_size)
+        nbytes = size_fn(B, Hq, w.num_kv_heads, D, w.block_size, self.maxlen,
+                         partition_size)
         self.ws = (torch.empty(nbytes, dtype=torch.uint8, device=case.q.device)
                    if nbytes else None)
         self.flags = torch.zeros(1, dtype=torch.int32, device=case.q.device)
@@ -269,6 +272,13 @@ class Step:
                 c.context_lens, c.query_start_loc, self.maxlen,
                 int(c.query_lens_np.max()), c.scale, error_flags=self.flags)
             return
+        if self.shared_prefix:
+            self.pa.pa_decode_attention_shared_prefix(
+                self.out, c.q, c.k_cache, c.v_cache, c.block_tables,
+                c.context_lens, c.group_start, c.prefix_lens, self.maxlen,
+                c.max_group_size, c.scale, self.ws,
+                partition_size=self.partition_arg, error_flags=self.flags)
+            return
         self.pa.pa_decode_attention(
             self.out, c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens,
             self.maxlen, c.scale, partition_size=self.partition_arg,
@@ -288,7 +298,7 @@ def run_gpu(args):
     case = inputs.make_case(args.workload, device=dev, num_seqs=args.seqs)
     w = case.workload
     part = args.partition if args.partition is not None else w.partition_size
-    step = Step(case, part)
+    step = Step(case, part, shared_prefix=not args.plain_decode)
     stream = torch.cuda.current_stream(dev)
 
     # in-run copy bandwidth (read + write bytes of a 1 GiB device copy)
@@ -358,7 +368,8 @@ def run_gpu(args):
                                if peak_kind == "measured" else "fallback 6.65 TB/s",
                 "unit": "GB/s", "frac": round(achieved / peak, 4)}
     kernel_name = ("paged_multi_query_kernel" if case.query_start_loc is not None
-                   else "paged_decode_kernel" +
+                   else ("paged_multi_row_kernel (group pass) + " if step.shared_prefix
+                         else "") + "paged_decode_kernel" +
                    (" + reduce" if step.partition < case.max_context_len else ""))
 
     result = None
@@ -392,6 +403,7 @@ def run_gpu(args):
                 "step": ("copy_blocks + " if case.copy_pairs.shape[0] else "") +
                         "reshape_and_cache + " +
                         ("paged_multi_query_attention" if case.query_start_loc is not None
+                         else "paged_decode_attention_shared_prefix" if step.shared_prefix
                          else "paged_decode_attention"),
                 "query_tokens_per_seq": (1 if case.query_lens_np is None
                                          else w.query_len),
@@ -437,7 +449,8 @@ def run_e2e(case, step, args, dist, dev):
     c = case
     names = ["q", "new_key", "new_value", "slot_mapping", "block_tables",
              "context_lens"] + (["copy_pairs"] if c.copy_pairs.shape[0] else []) \
-        + (["query_start_loc"] if c.query_start_loc is not None else [])
+        + (["query_start_loc"] if c.query_start_loc is not None else []) \
+        + (["group_start", "prefix_lens"] if step.shared_prefix else [])
     host_in = {n: getattr(c, n).cpu().pin_memory() for n in names}
     dev_in = [{n: torch.empty_like(getattr(c, n)) for n in names} for _ in range(2)]
     outs = [torch.empty_like(step.out) for _ in range(2)]
@@ -477,6 +490,13 @@ def run_e2e(case, step, args, dist, dev):
                 outs[b], d["q"], c.k_cache, c.v_cache, d["block_tables"],
                 d["context_lens"], d["query_start_loc"], step.maxlen,
                 int(c.query_lens_np.max()), c.scale, error_flags=step.flags,
+                stream=comp)
+        elif step.shared_prefix:
+            pa.pa_decode_attention_shared_prefix(
+                outs[b], d["q"], c.k_cache, c.v_cache, d["block_tables"],
+                d["context_lens"], d["group_start"], d["prefix_lens"],
+                step.maxlen, c.max_group_size, c.scale, step.ws,
+                partition_size=step.partition_arg, error_flags=step.flags,
                 stream=comp)
         else:
             pa.pa_decode_attention(outs[b], d["q"], c.k_cache, c.v_cache,
@@ -690,6 +710,9 @@ def main():
                     help="keep only the first N sequences of the workload")
     ap.add_argument("--swap", action="store_true",
                     help="measure swap_blocks bandwidth instead (own JSON line)")
+    ap.add_argument("--plain-decode", action="store_true",
+                    help="attend workloads with shared-prefix groups with the "
+                         "plain decode call (no group pass)")
     ap.add_argument("--kernel-only", action="store_true",
                     help="time the device step only: no e2e leg, no in-run "
                          "copy peak, no CPU baseline (profiling runs)")

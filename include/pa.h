@@ -85,6 +85,7 @@ typedef enum {
 #define PA_DEVERR_TIMEOUT 0x10    /* an async-copy wait exceeded its time limit */
 #define PA_DEVERR_INTERNAL 0x20   /* shared memory not 1024-byte aligned (no work done) */
 #define PA_DEVERR_QUERY_LEN 0x40  /* query count < 0, > context length or > max_query_len */
+#define PA_DEVERR_PREFIX 0x80     /* a shared-prefix group description is invalid */
 
 /* Human-readable name of a pa_status value (static string, never NULL). */
 const char* pa_status_string(int status);
@@ -217,6 +218,59 @@ int pa_multi_query_attention(float* out, const void* q, const void* k_cache,
                              int head_size, int block_size, int num_blocks,
                              float scale, int* error_flags,
                              pa_stream_t stream);
+
+/*
+ * pa_decode_attention_shared_prefix - decode attention for batches whose
+ * sequences share prompt blocks, as parallel samples of one prompt or beams
+ * with a common history do ("vLLM: Anatomy and Mechanisms of High-Throughput
+ * LLM Inference", "Memory Sharing via Copy-on-Write (CoW)": the outputs of
+ * one prompt share the prompt's KV blocks).  The result is that of
+ * pa_decode_attention on the same arguments; the pages share the memory, and
+ * this call also shares the reading of it.
+ *
+ * Group i is the sequences group_start[i] .. group_start[i+1]-1.  Their
+ * block tables agree on the first prefix_lens[i] / block_size entries (the
+ * shared blocks); the library reads those entries from the group's first
+ * sequence only.  For each sequence s of a group with context length L, the
+ * first min(prefix_lens[i], L) tokens are attended in a group pass that
+ * streams every shared block once for all of the group's query rows (the
+ * tcgen05 tensor cores, up to 32 rows per kv head and pass); the remaining
+ * tokens of s are attended per sequence by the decode kernel, which merges
+ * the two partial softmax results exactly:
+ *     out = (l1 2^(m1-M) o1 + l2 2^(m2-M) o2) / (l1 2^(m1-M) + l2 2^(m2-M)).
+ * Sequences outside every group, and groups whose description is invalid
+ * (reported with PA_DEVERR_PREFIX), are attended as by pa_decode_attention.
+ *
+ *   group_start     int32 [num_groups + 1], device, non-decreasing, in
+ *                   [0, num_seqs]; groups need not cover every sequence.
+ *   prefix_lens     int32 [num_groups], device: shared tokens of each group,
+ *                   a non-negative multiple of block_size (0 = no sharing).
+ *   num_groups      >= 0 (0 is exactly pa_decode_attention).
+ *   max_group_size  host-known upper bound of the group sizes (>= 1 when
+ *                   num_groups > 0); a larger group is reported and runs
+ *                   without the group pass.
+ *   workspace       device buffer of at least
+ *                   pa_shared_prefix_workspace_size(...) bytes, 256-byte
+ *                   aligned; scratch, needs no initialisation.
+ *   other arguments as for pa_decode_attention.
+ * Supports head_size 128, block_size in {16, 32}, num_heads / num_kv_heads
+ * in 1..8 (head_size 64 returns PA_ERR_UNSUPPORTED).  Returns PA_OK or a
+ * negative pa_status; run-to-run results are bitwise deterministic.
+ */
+size_t pa_shared_prefix_workspace_size(int num_seqs, int num_heads,
+                                       int num_kv_heads, int head_size,
+                                       int block_size, int max_context_len,
+                                       int partition_size);
+
+int pa_decode_attention_shared_prefix(
+    float* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, int max_blocks_per_seq,
+    const int32_t* context_lens, int max_context_len,
+    const int32_t* group_start, const int32_t* prefix_lens, int num_groups,
+    int max_group_size, int num_seqs, int num_heads, int num_kv_heads,
+    int head_size, int block_size, int num_blocks, float scale,
+    int partition_size, void* workspace, size_t workspace_bytes,
+    int* error_flags, pa_stream_t stream);
 
 /*
  * pa_swap_blocks - move whole KV blocks between pools in different memories:

@@ -29,6 +29,7 @@ PA_DEVERR_COPY_PAIR = 0x8
 PA_DEVERR_TIMEOUT = 0x10
 PA_DEVERR_INTERNAL = 0x20
 PA_DEVERR_QUERY_LEN = 0x40
+PA_DEVERR_PREFIX = 0x80
 
 _lock = threading.Lock()
 _lib = None
@@ -78,6 +79,12 @@ def raw():
             p, p, p, p, p, i32, p, i32, p, i32, i32, i32, i32, i32, i32, i32,
             f32, p, p]
         lib.pa_multi_query_attention.restype = i32
+        lib.pa_shared_prefix_workspace_size.argtypes = [i32] * 7
+        lib.pa_shared_prefix_workspace_size.restype = sz
+        lib.pa_decode_attention_shared_prefix.argtypes = [
+            p, p, p, p, p, i32, p, i32, p, p, i32, i32, i32, i32, i32, i32,
+            i32, i32, f32, i32, p, sz, p, p]
+        lib.pa_decode_attention_shared_prefix.restype = i32
         lib.pa_swap_blocks.argtypes = [p, p, i32, p, i32, i64, i64, i64, p, p]
         lib.pa_swap_blocks.restype = i32
         lib.pa_copy_blocks.argtypes = [p, p, i32, p, i32, i32, i32, i32, i32,
@@ -235,6 +242,58 @@ def pa_multi_query_attention(out, q, k_cache, v_cache, block_tables,
         _ptr(query_start_loc), int(max_query_len), B, Hq, Hkv, D, bs, NB,
         float(scale), _ptr(error_flags), _stream(stream))
     return _check(rc, "pa_multi_query_attention")
+
+
+def pa_shared_prefix_workspace_size(num_seqs, num_heads, num_kv_heads,
+                                    head_size, block_size, max_context_len,
+                                    partition_size=0) -> int:
+    return int(raw().pa_shared_prefix_workspace_size(
+        num_seqs, num_heads, num_kv_heads, head_size, block_size,
+        max_context_len, partition_size))
+
+
+def pa_decode_attention_shared_prefix(out, q, k_cache, v_cache, block_tables,
+                                      context_lens, group_start, prefix_lens,
+                                      max_context_len: int,
+                                      max_group_size: int, scale: float,
+                                      workspace, partition_size: int = 0,
+                                      error_flags=None, stream=None) -> int:
+    """pa_decode_attention for batches whose sequences share prompt blocks:
+    sequences group_start[i] .. group_start[i+1]-1 (int32 [G+1]) share their
+    first prefix_lens[i] tokens (int32 [G]); workspace of at least
+    pa_shared_prefix_workspace_size(...) bytes."""
+    import torch
+    bf = torch.bfloat16
+    _cuda(out, "out", torch.float32, 3); _cuda(q, "q", bf, 3)
+    _cuda(k_cache, "k_cache", bf, 4); _cuda(v_cache, "v_cache", bf, 4)
+    _cuda(block_tables, "block_tables", torch.int32, 2)
+    _cuda(context_lens, "context_lens", torch.int32, 1)
+    _cuda(group_start, "group_start", torch.int32, 1)
+    _cuda(prefix_lens, "prefix_lens", torch.int32, 1)
+    _cuda(workspace, "workspace")
+    for name, t in (("out", out), ("q", q), ("k_cache", k_cache),
+                    ("v_cache", v_cache), ("block_tables", block_tables),
+                    ("context_lens", context_lens),
+                    ("group_start", group_start), ("prefix_lens", prefix_lens)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    B, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_cache.shape
+    G = prefix_lens.shape[0]
+    if out.shape != q.shape or D2 != D or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch between q, out and the pools")
+    if block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise ValueError("block_tables / context_lens must have B rows")
+    if group_start.shape[0] != G + 1:
+        raise ValueError("group_start must have one more entry than prefix_lens")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = raw().pa_decode_attention_shared_prefix(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), int(max_context_len),
+        _ptr(group_start), _ptr(prefix_lens), G, int(max_group_size), B, Hq,
+        Hkv, D, bs, NB, float(scale), int(partition_size), _ptr(workspace),
+        ws_bytes, _ptr(error_flags), _stream(stream))
+    return _check(rc, "pa_decode_attention_shared_prefix")
 
 
 def pa_swap_blocks(src_caches: Sequence, dst_caches: Sequence, block_mapping,

@@ -13,6 +13,7 @@
 #include "pa_common.cuh"
 #include "pa_decode.cuh"
 #include "pa_multi_query.cuh"
+#include "pa_multi_row.cuh"
 #include "pa_swap.cuh"
 
 namespace pa {
@@ -79,6 +80,25 @@ size_t workspace_bytes_for(int num_seqs, int num_heads, int head_size,
     bytes = (bytes + 255) & ~(size_t)255;
     bytes += ((rows * 4 + 255) & ~(size_t)255) * 2;  // tmp_m, tmp_l
     return bytes;
+}
+
+// Shared-prefix call: the decode split's scratch, then the group pass's
+// partial results (O/l, max, sum per row).
+struct PrefixLayout {
+    size_t split_bytes, o_off, m_off, l_off, total;
+};
+
+PrefixLayout prefix_layout(int num_seqs, int num_heads, int head_size,
+                           int max_partitions) {
+    PrefixLayout L;
+    const size_t rows = (size_t)num_seqs * num_heads;
+    L.split_bytes = (workspace_bytes_for(num_seqs, num_heads, head_size,
+                                         max_partitions) + 255) & ~(size_t)255;
+    L.o_off = L.split_bytes;
+    L.m_off = L.o_off + ((rows * head_size * 4 + 255) & ~(size_t)255);
+    L.l_off = L.m_off + ((rows * 4 + 255) & ~(size_t)255);
+    L.total = L.l_off + ((rows * 4 + 255) & ~(size_t)255);
+    return L;
 }
 
 }  // namespace
@@ -229,6 +249,7 @@ int pa_decode_attention(float* out, const void* q, const void* k_cache,
     p.partition_size = part;
     p.max_partitions = np;
     p.scale_log2 = pa::log2e_scale(scale);
+    p.block_size = block_size;
     cudaError_t e = pa::launch_paged_decode(
         p, head_size, block_size, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
@@ -291,16 +312,178 @@ int pa_multi_query_attention(float* out, const void* q, const void* k_cache,
     // Kernel choice: the tcgen05 kernel for 128-row tiles (prefill chunks),
     // the mma.sync kernel for few rows per sequence (speculative verify).
     // PA_MULTI_QUERY_KERNEL=mma|tc overrides the choice (tests, benchmarks).
-    bool use_tc = pa::multi_query_tc_eligible(head_size, max_query_len, G);
+    enum { kMma, kTc, kRows } kind = kMma;
+    if (pa::multi_query_tc_eligible(head_size, max_query_len, G)) kind = kTc;
     if (const char* force = std::getenv("PA_MULTI_QUERY_KERNEL")) {
-        if (std::strcmp(force, "mma") == 0) use_tc = false;
-        if (std::strcmp(force, "tc") == 0 && head_size == 128) use_tc = true;
+        if (std::strcmp(force, "mma") == 0) kind = kMma;
+        if (std::strcmp(force, "tc") == 0 && head_size == 128) kind = kTc;
+        if (std::strcmp(force, "rows") == 0 && head_size == 128) kind = kRows;
     }
-    cudaError_t e = use_tc
-        ? pa::launch_paged_multi_query_tc(p, block_size,
-                                          reinterpret_cast<cudaStream_t>(stream))
-        : pa::launch_paged_multi_query(p, head_size, block_size,
-                                       reinterpret_cast<cudaStream_t>(stream));
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (kind == kRows) {
+        pa::MultiRowParams r{};
+        r.out = out;
+        r.q = p.q;
+        r.k_cache = p.k_cache;
+        r.v_cache = p.v_cache;
+        r.block_tables = block_tables;
+        r.context_lens = context_lens;
+        r.query_start_loc = query_start_loc;
+        r.error_flags = error_flags;
+        r.shared_prefix_mode = 0;
+        r.num_seqs = num_seqs;
+        r.max_blocks_per_seq = max_blocks_per_seq;
+        r.max_context_len = max_context_len;
+        r.max_query_len = max_query_len;
+        r.num_heads = num_heads;
+        r.num_kv_heads = num_kv_heads;
+        r.num_blocks = num_blocks;
+        r.block_size = block_size;
+        r.group = G;
+        r.tiles = (int)(((long long)max_query_len * G + pa::kMultiRowTile - 1) /
+                        pa::kMultiRowTile);
+        r.num_units = num_seqs;
+        r.scale_log2 = p.scale_log2;
+        if ((long long)r.num_units * r.tiles * num_kv_heads > 0x7fffffffLL)
+            return PA_ERR_UNSUPPORTED;
+        e = pa::launch_paged_multi_row(r, st);
+    } else if (kind == kTc) {
+        e = pa::launch_paged_multi_query_tc(p, block_size, st);
+    } else {
+        e = pa::launch_paged_multi_query(p, head_size, block_size, st);
+    }
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+size_t pa_shared_prefix_workspace_size(int num_seqs, int num_heads,
+                                       int num_kv_heads, int head_size,
+                                       int block_size, int max_context_len,
+                                       int partition_size) {
+    const int part = pa_decode_partition_size(num_seqs, num_heads, num_kv_heads,
+                                              head_size, block_size,
+                                              max_context_len, partition_size);
+    if (part <= 0 || num_heads <= 0 || head_size <= 0) return 0;
+    return pa::prefix_layout(num_seqs, num_heads, head_size,
+                             pa::num_partitions(max_context_len, part)).total;
+}
+
+int pa_decode_attention_shared_prefix(
+    float* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, int max_blocks_per_seq,
+    const int32_t* context_lens, int max_context_len,
+    const int32_t* group_start, const int32_t* prefix_lens, int num_groups,
+    int max_group_size, int num_seqs, int num_heads, int num_kv_heads,
+    int head_size, int block_size, int num_blocks, float scale,
+    int partition_size, void* workspace, size_t workspace_bytes,
+    int* error_flags, pa_stream_t stream) {
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 ||
+        head_size <= 0 || block_size <= 0 || num_blocks <= 0 ||
+        max_blocks_per_seq <= 0 || max_context_len < 0 || partition_size < 0 ||
+        num_groups < 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    if ((long long)max_context_len > (long long)max_blocks_per_seq * block_size)
+        return PA_ERR_INVALID_ARG;
+    if (partition_size > 0 && partition_size % block_size != 0)
+        return PA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+    if (num_groups > 0 && (max_group_size < 1 || !group_start || !prefix_lens ||
+                           (reinterpret_cast<uintptr_t>(group_start) & 3u) ||
+                           (reinterpret_cast<uintptr_t>(prefix_lens) & 3u)))
+        return PA_ERR_INVALID_ARG;
+    if (head_size != 128 ||
+        !pa::decode_shape_supported(num_heads, num_kv_heads, head_size, block_size))
+        return PA_ERR_UNSUPPORTED;
+    if ((long long)num_blocks * block_size > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PA_OK;
+    if (num_seqs > pa::kMaxGridYZ) return PA_ERR_UNSUPPORTED;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+        return PA_ERR_INVALID_ARG;
+    if (!pa::aligned16(out) || !pa::aligned16(q) || !pa::aligned16(k_cache) ||
+        !pa::aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+        (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+        return PA_ERR_INVALID_ARG;
+
+    const int part = pa::plan_partition(num_seqs, num_kv_heads, block_size,
+                                        max_context_len, partition_size);
+    const int np = pa::num_partitions(max_context_len, part);
+    if (np > pa::kMaxGridYZ) return PA_ERR_INVALID_ARG;
+    const pa::PrefixLayout lay = pa::prefix_layout(num_seqs, num_heads, head_size, np);
+    if (!workspace || workspace_bytes < lay.total) return PA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PA_ERR_INVALID_ARG;
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    const int G = num_heads / num_kv_heads;
+    // A group cannot hold more than num_seqs sequences: the bound changes
+    // no group's validity and keeps the grid small.
+    const int mgs = max_group_size < num_seqs ? max_group_size : num_seqs;
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    pa::CascadeGroups groups{group_start, prefix_lens, num_groups, mgs};
+    if (num_groups > 0) {
+        const int per_tile = pa::kMultiRowTile / G;
+        pa::MultiRowParams r{};
+        r.out = reinterpret_cast<float*>(ws + lay.o_off);
+        r.out_m = reinterpret_cast<float*>(ws + lay.m_off);
+        r.out_l = reinterpret_cast<float*>(ws + lay.l_off);
+        r.q = static_cast<const uint16_t*>(q);
+        r.k_cache = static_cast<const uint16_t*>(k_cache);
+        r.v_cache = static_cast<const uint16_t*>(v_cache);
+        r.block_tables = block_tables;
+        r.context_lens = context_lens;
+        r.groups = groups;
+        r.error_flags = error_flags;
+        r.shared_prefix_mode = 1;
+        r.num_seqs = num_seqs;
+        r.max_blocks_per_seq = max_blocks_per_seq;
+        r.max_context_len = max_context_len;
+        r.num_heads = num_heads;
+        r.num_kv_heads = num_kv_heads;
+        r.num_blocks = num_blocks;
+        r.block_size = block_size;
+        r.group = G;
+        r.tiles = (mgs + per_tile - 1) / per_tile;
+        r.num_units = num_groups;
+        r.scale_log2 = pa::log2e_scale(scale);
+        if ((long long)num_groups * r.tiles * num_kv_heads > 0x7fffffffLL)
+            return PA_ERR_UNSUPPORTED;
+        if (pa::launch_paged_multi_row(r, st) != cudaSuccess) return PA_ERR_CUDA;
+    }
+
+    pa::DecodeParams p{};
+    p.out = out;
+    p.q = static_cast<const uint16_t*>(q);
+    p.k_cache = static_cast<const uint16_t*>(k_cache);
+    p.v_cache = static_cast<const uint16_t*>(v_cache);
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    if (np > 1) {
+        const size_t rows = (size_t)num_seqs * num_heads * np;
+        const size_t o_bytes = (rows * head_size * 4 + 255) & ~(size_t)255;
+        const size_t s_bytes = (rows * 4 + 255) & ~(size_t)255;
+        p.tmp_o = reinterpret_cast<float*>(ws);
+        p.tmp_m = reinterpret_cast<float*>(ws + o_bytes);
+        p.tmp_l = reinterpret_cast<float*>(ws + o_bytes + s_bytes);
+    }
+    p.error_flags = error_flags;
+    p.num_seqs = num_seqs;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.max_context_len = max_context_len;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.num_blocks = num_blocks;
+    p.group = G;
+    p.partition_size = part;
+    p.max_partitions = np;
+    p.scale_log2 = pa::log2e_scale(scale);
+    p.block_size = block_size;
+    p.cascade = num_groups > 0 ? 1 : 0;
+    p.groups = groups;
+    p.pref_o = reinterpret_cast<const float*>(ws + lay.o_off);
+    p.pref_m = reinterpret_cast<const float*>(ws + lay.m_off);
+    p.pref_l = reinterpret_cast<const float*>(ws + lay.l_off);
+    cudaError_t e = pa::launch_paged_decode(p, head_size, block_size, st);
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

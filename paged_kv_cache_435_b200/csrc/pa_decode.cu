@@ -84,6 +84,7 @@ struct Item {
     int tok0;    // first token of the partition
     int tok1;    // one past its last token
     int nparts;  // partitions of this sequence
+    int sh;      // tokens before tok0 left to the shared-prefix group pass
 };
 
 __device__ __forceinline__ int clamped_len(const DecodeParams& p, int s) {
@@ -99,8 +100,15 @@ __device__ __forceinline__ int parts_of(int L, int P) {
     return L <= 0 ? 1 : (L + P - 1) / P;  // an empty context still owns one item
 }
 
+// First token of sequence s this kernel attends (0 unless a shared-prefix
+// group pass covers the tokens before it).
+template <bool kCascade, int BS>
+__device__ __forceinline__ int first_token(const DecodeParams& p, int s, int L) {
+    return kCascade ? cascade_shared_len(p.groups, s, L, p.num_seqs, BS) : 0;
+}
+
 // Item k of this CTA (k = 0, 1, ...).
-template <bool kPersist>
+template <bool kPersist, bool kCascade, int BS>
 __device__ __forceinline__ Item get_item(const DecodeParams& p,
                                          const int* prefix, int k) {
     Item it;
@@ -122,13 +130,15 @@ __device__ __forceinline__ Item get_item(const DecodeParams& p,
         part = blockIdx.y;
     }
     const int L = clamped_len(p, s);
-    const int np = parts_of(L, p.partition_size);
+    const int sh = first_token<kCascade, BS>(p, s, L);
+    const int np = parts_of(L - sh, p.partition_size);
     if (part >= np) return it;
     it.s = s;
     it.part = part;
     it.L = L;
     it.nparts = np;
-    it.tok0 = part * p.partition_size;
+    it.sh = sh;
+    it.tok0 = sh + part * p.partition_size;
     it.tok1 = min(L, it.tok0 + p.partition_size);
     return it;
 }
@@ -158,7 +168,7 @@ __device__ __forceinline__ void named_bar_arrive(int id) {
     asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(kThreads) : "memory");
 }
 
-template <int D, int BS, bool kPersist>
+template <int D, int BS, bool kPersist, bool kCascade>
 __global__ void __launch_bounds__(kThreads, kTargetCtasPerSM)
 paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
@@ -196,7 +206,11 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         if (threadIdx.x == 0) prefix[0] = 0;
         for (int base = 0; base < p.num_seqs; base += kThreads) {
             const int s = base + threadIdx.x;
-            int v = s < p.num_seqs ? parts_of(clamped_len(p, s), p.partition_size) : 0;
+            int v = 0;
+            if (s < p.num_seqs) {
+                const int L = clamped_len(p, s);
+                v = parts_of(L - first_token<kCascade, BS>(p, s, L), p.partition_size);
+            }
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int t = __shfl_up_sync(0xffffffffu, v, o);
@@ -240,7 +254,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
     // Lane l finds the (ids_base + l)-th chunk of the stream and its slot.
     auto refill = [&]() {
         int k = prod_k, i = prod_i, n = lane;
-        Item it = get_item<kPersist>(p, prefix, k);
+        Item it = get_item<kPersist, kCascade, BS>(p, prefix, k);
         for (;;) {
             if (it.s < 0) break;
             const int rem = warp_chunks(it, warp) - i;
@@ -248,7 +262,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
             n -= rem > 0 ? rem : 0;
             ++k;
             i = 0;
-            it = get_item<kPersist>(p, prefix, k);
+            it = get_item<kPersist, kCascade, BS>(p, prefix, k);
         }
         int slot = -1;
         if (it.s >= 0) {
@@ -315,7 +329,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
             dst[ks][1] = live ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8 + qc) : 0u;
         }
     };
-    Item next_it = get_item<kPersist>(p, prefix, 0);
+    Item next_it = get_item<kPersist, kCascade, BS>(p, prefix, 0);
     uint32_t qnext[D / 16][2];
     load_q(next_it, qnext);
     for (;; ++k) {
@@ -328,7 +342,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
             qa[ks][0] = qnext[ks][0];
             qa[ks][1] = qnext[ks][1];
         }
-        next_it = get_item<kPersist>(p, prefix, k + 1);
+        next_it = get_item<kPersist, kCascade, BS>(p, prefix, k + 1);
         load_q(next_it, qnext);
 
         float o[D / 8][4];
@@ -482,6 +496,18 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                 const int64_t row = (int64_t)it.s * Hq + h;
                 const int64_t idx = row * p.max_partitions + it.part;
                 float* dst = direct ? p.out + row * D : p.tmp_o + idx * D;
+                // Shared-prefix call, unsplit sequence: fold in the group
+                // pass's partial (its O/l, max and sum) here.
+                float wa = 1.f, wb = 0.f;
+                const float* po = nullptr;
+                if (kCascade && direct && it.sh > 0) {
+                    const float mp = p.pref_m[row], lp = p.pref_l[row];
+                    const float Mt = fmaxf(M, mp);
+                    wa = M == -INFINITY ? 0.f : exp2f(M - Mt);
+                    wb = lp * exp2f(mp - Mt);
+                    den = den * wa + wb;
+                    po = p.pref_o + row * D;
+                }
 #pragma unroll
                 for (int j = 0; j < D / 8; ++j) {
                     float v[2];
@@ -491,6 +517,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
 #pragma unroll
                         for (int w = 1; w < kWarps; ++w)
                             acc += sc[w] * red_o[((w - 1) * kMaxGroup + qr) * C::kRedStride + 8 * j + qc + e];
+                        if (kCascade && po != nullptr) acc = acc * wa + wb * po[8 * j + qc + e];
                         v[e] = it.L > 0 ? acc / den : 0.f;
                     }
                     *reinterpret_cast<float2*>(dst + 8 * j + qc) = make_float2(v[0], v[1]);
@@ -532,9 +559,11 @@ paged_decode_reduce_kernel(const DecodeParams p) {
     pdl_wait();  // the partials come from the grid launched just before
     int L = p.context_lens[s];
     L = L < 0 ? 0 : (L > p.max_context_len ? p.max_context_len : L);
-    const int np = (L + p.partition_size - 1) / p.partition_size;
+    const int sh = p.cascade ? cascade_shared_len(p.groups, s, L, p.num_seqs, p.block_size) : 0;
+    const int np = (L - sh + p.partition_size - 1) / p.partition_size;
     if (np <= 1) return;  // written directly by the partition kernel
     const int64_t base = ((int64_t)s * p.num_heads + h) * p.max_partitions;
+    const int64_t row = (int64_t)s * p.num_heads + h;
 
     __shared__ float warp_max[kReduceWarps];
     __shared__ float part_acc[kReduceWarps][D];
@@ -550,6 +579,7 @@ paged_decode_reduce_kernel(const DecodeParams p) {
     M = warp_max[0];
 #pragma unroll
     for (int w = 1; w < kReduceWarps; ++w) M = fmaxf(M, warp_max[w]);
+    if (sh > 0) M = fmaxf(M, p.pref_m[row]);  // the group pass's partial joins
 
     float acc[V];
 #pragma unroll
@@ -585,6 +615,13 @@ paged_decode_reduce_kernel(const DecodeParams p) {
 #pragma unroll
             for (int v = 0; v < V; ++v) acc[v] += wts[u] * vals[u][v];
         }
+    }
+    if (sh > 0 && warp == 0) {
+        const float wp = p.pref_l[row] * exp2f(p.pref_m[row] - M);
+        den += wp;
+        const float* po = p.pref_o + row * D + lane * V;
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[v] += wp * po[v];
     }
 #pragma unroll
     for (int v = 0; v < V; ++v) part_acc[warp][lane * V + v] = acc[v];
@@ -671,36 +708,45 @@ cudaError_t set_smem(Kernel kernel, int bytes, int* flags) {
     return cudaSuccess;
 }
 
-template <int D, int BS>
-cudaError_t launch_typed(const DecodeParams& p, cudaStream_t stream) {
+template <int D, int BS, bool kCascade>
+cudaError_t launch_partition_kernel(const DecodeParams& p, const CUtensorMap& tmk,
+                                    const CUtensorMap& tmv, cudaStream_t stream) {
     using C = Cfg<D>;
     static int grid_ready[64] = {0};
     static int persist_ready[64] = {0};
-    CUtensorMap tmk, tmv;
-    if (!encode_pool_map(&tmk, p.k_cache, p.num_blocks, BS, p.num_kv_heads, D) ||
-        !encode_pool_map(&tmv, p.v_cache, p.num_blocks, BS, p.num_kv_heads, D))
-        return cudaErrorInvalidValue;
     const bool persist = p.max_partitions > 1 && p.num_seqs <= kMaxPersistSeqs;
     cudaError_t e;
     if (persist) {
-        e = set_smem(paged_decode_kernel<D, BS, true>, C::kSmemPersist, persist_ready);
+        e = set_smem(paged_decode_kernel<D, BS, true, kCascade>, C::kSmemPersist,
+                     persist_ready);
         if (e != cudaSuccess) return e;
         long long per_head = (kTargetCtasPerSM * kNumSMs + p.num_kv_heads - 1) / p.num_kv_heads;
         const long long items = (long long)p.num_seqs * p.max_partitions;
         if (per_head > items) per_head = items;
         if (per_head < 1) per_head = 1;
         dim3 grid((unsigned)p.num_kv_heads, (unsigned)per_head, 1);
-        e = launch_pdl(paged_decode_kernel<D, BS, true>, grid, dim3(kThreads),
+        e = launch_pdl(paged_decode_kernel<D, BS, true, kCascade>, grid, dim3(kThreads),
                        C::kSmemPersist, stream, tmk, tmv, p);
     } else {
-        e = set_smem(paged_decode_kernel<D, BS, false>, C::kSmemGrid, grid_ready);
+        e = set_smem(paged_decode_kernel<D, BS, false, kCascade>, C::kSmemGrid, grid_ready);
         if (e != cudaSuccess) return e;
         dim3 grid((unsigned)p.num_kv_heads, (unsigned)p.max_partitions,
                   (unsigned)p.num_seqs);
-        e = launch_pdl(paged_decode_kernel<D, BS, false>, grid, dim3(kThreads),
+        e = launch_pdl(paged_decode_kernel<D, BS, false, kCascade>, grid, dim3(kThreads),
                        C::kSmemGrid, stream, tmk, tmv, p);
     }
     count_launch();
+    return e;
+}
+
+template <int D, int BS>
+cudaError_t launch_typed(const DecodeParams& p, cudaStream_t stream) {
+    CUtensorMap tmk, tmv;
+    if (!encode_pool_map(&tmk, p.k_cache, p.num_blocks, BS, p.num_kv_heads, D) ||
+        !encode_pool_map(&tmv, p.v_cache, p.num_blocks, BS, p.num_kv_heads, D))
+        return cudaErrorInvalidValue;
+    cudaError_t e = p.cascade ? launch_partition_kernel<D, BS, true>(p, tmk, tmv, stream)
+                              : launch_partition_kernel<D, BS, false>(p, tmk, tmv, stream);
     if (e != cudaSuccess) return e;
     if (p.max_partitions > 1) {
         dim3 rgrid((unsigned)p.num_heads, (unsigned)p.num_seqs);

@@ -4,6 +4,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "pa_cascade.cuh"
+
 namespace pa {
 
 struct DecodeParams {
@@ -27,6 +29,15 @@ struct DecodeParams {
     int partition_size;          // tokens, multiple of block_size
     int max_partitions;          // ceil(max_context_len / partition_size)
     float scale_log2;            // scale * log2(e)
+    int block_size;
+    // Shared-prefix call: each sequence starts at its shared length (the
+    // group pass covered the tokens before it) and its result is merged
+    // with the group pass's partial (pref_o = O/l, pref_m, pref_l per row).
+    int cascade;
+    CascadeGroups groups;
+    const float* pref_o;         // fp32 [B][Hq][D]
+    const float* pref_m;         // fp32 [B][Hq] (log2 domain)
+    const float* pref_l;         // fp32 [B][Hq]
 };
 
 // scale * log2(e): logits are kept in the log2 domain (exp2f).

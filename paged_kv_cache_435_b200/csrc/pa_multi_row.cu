@@ -1,0 +1,919 @@
+// Paged attention for up to 32 query rows per kv head on the tcgen05 tensor
+// cores, with the operands swapped so that the tokens fill the MMA's M.
+//
+// Two callers share it:
+//  * speculative verification (pa_multi_query_attention): the k proposed
+//    tokens of a sequence times the G query heads of a kv head are the rows,
+//    causal within the chunk ("vLLM: Anatomy and Mechanisms of
+//    High-Throughput LLM Inference", "Speculative Decoding");
+//  * the group pass of pa_decode_attention_shared_prefix: the samples of one
+//    prompt times the G heads are the rows, over the prompt blocks they share
+//    ("Memory Sharing via Copy-on-Write (CoW)"), written as partial softmax
+//    results for the decode kernel to merge.
+// With 32 rows over a stream of KV the work is 32 flop per KV byte, far below
+// the tensor roofline: the goal is to read every block once at HBM speed with
+// the math hidden behind it.  A 128-row M tile would waste 3/4 of the tensor
+// core on such a stream, so the products are transposed:
+//     S^T (128 tokens x 32 rows)  = K (128 x 128 d) . Q^T (128 d x 32 rows)
+//     O^T (128 d x 64)           += V^T (128 d x 128 tokens) . [P_hi^T | P_lo^T]
+// with M = 128 in both.  K comes from its TMA tile as a K-major A operand, V
+// as an MN-major A operand (the same tile, read transposed by the
+// descriptor).  Q^T is a K-major B operand; P's bf16 high part and its bf16
+// residual sit side by side as one MN-major B operand of N = 64 (one
+// 128-byte row per token, written by that token's thread), so V is read
+// once per chunk and O_hi, O_lo accumulate in adjacent TMEM columns, summed
+// at the end.  Accumulators live in tensor memory: S^T double-buffered (2 x 32
+// columns), O^T double-buffered across items (2 x 64 columns).
+//
+// CTA: 7 warps, one CTA per SM, persistent over items (row tile, kv head):
+//   warps 0-3  softmax: thread i owns token i of the chunk (TMEM lane i) and
+//              all 32 rows; P = 2^(s - m) as bf16 high part + bf16 residual
+//              (~16 bits into the PV product), one 128-byte row of P^T;
+//   warp 4     K producer, warp 5 V producer: 16-token TMA tensor tiles
+//              (128-byte swizzle) of each 128-token chunk into 2- and 3-stage
+//              rings (V waits for the softmax, so it runs deeper);
+//   warp 6     TMEM allocation and the MMA issue (one thread).
+// Online softmax with a lazy reference: every chunk, one barrier-reduction
+// over the 4 warps (bar.red.popc) asks whether any row's logit exceeds its
+// reference max by more than 2^8; only then is the exact per-row chunk max
+// formed (warp transpose-reduction + shared memory), O^T rescaled in TMEM and
+// the reference moved.  Sums are kept per thread and reduced at item end.
+// The producers and the MMA warp run ahead across item boundaries; the
+// epilogue of an item runs one chunk into the next item.  Every wait is
+// bounded; the softmax warps decide aborts together at their per-chunk
+// barrier, and TMEM is released on every exit path.
+#include <cuda.h>
+
+#include <cfloat>
+#include <cstdint>
+#include <mutex>
+
+#include "pa_cascade.cuh"
+#include "pa_common.cuh"
+#include "pa_multi_row.cuh"
+
+namespace pa {
+namespace {
+
+constexpr int kTok = 128;                 // tokens per chunk (M of both products)
+constexpr int kN = kMultiRowTile;         // rows (N of both products)
+constexpr int kD = 128;
+constexpr int kKStages = 2;
+constexpr int kVStages = 3;
+constexpr int kThreads = 224;
+constexpr int kHalf = kTok * 128;         // 16 KB: 128 tokens x 64 d (one swizzle column)
+constexpr int kStageBytes = 2 * kHalf;    // 32 KB: one chunk of K or V
+constexpr int kQHalf = kN * 128;          // 4 KB: 32 rows x 64 d
+constexpr int kQBytes = 2 * kQHalf;
+constexpr int kPBytes = kTok * 128;       // 16 KB: P^T of a chunk, 128 B per token
+constexpr int kKOff = 0;
+constexpr int kVOff = kKOff + kKStages * kStageBytes;
+constexpr int kQOff = kVOff + kVStages * kStageBytes;  // 2 item buffers
+constexpr int kPOff = kQOff + 2 * kQBytes;             // 2 chunk buffers x (hi | lo)
+constexpr int kMiscOff = kPOff + 2 * kPBytes;
+constexpr int kCmaxOff = kMiscOff;                     // float [32][4]
+constexpr int kRedLOff = kCmaxOff + 512;               // float [3][32][4]
+constexpr int kItemMOff = kRedLOff + 3 * 512;          // float [3][32]
+constexpr int kRowLimOff = kItemMOff + 3 * 128;        // int [3][32]
+constexpr int kRowOutOff = kRowLimOff + 3 * 128;       // int64 [3][32]
+constexpr int kBarOff = kRowOutOff + 3 * 256;
+// barriers: k_full[KS] k_empty[KS] v_full[VS] v_empty[VS] s_full[2] p_full[2]
+//           pv_done[2] o_full[2] o_empty[2] q_ready[2] drain
+constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 11;
+constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16;
+constexpr uint32_t kTmemCols = 256;       // S0 | S1 | O0 (hi, lo) | O1 (hi, lo)
+constexpr uint32_t kTmemO = 64;           // first O column
+constexpr float kRescaleThreshold = 8.f;  // log2 units
+constexpr float kNoMax = -FLT_MAX;        // reference of a row with no token yet
+constexpr int kNumSMs = 148;
+
+static_assert(kStageBytes % 1024 == 0 && kQBytes % 1024 == 0 && kPBytes % 1024 == 0,
+              "swizzled tiles need 1024-byte alignment");
+static_assert(kRowOutOff % 8 == 0 && kBarOff % 8 == 0, "8-byte alignment");
+static_assert(kSmemBytes <= 232448, "shared memory");
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity) {
+    return mbar_wait_bounded(bar, parity);
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// Instruction descriptor, kind::f16: fp32 D, bf16 A and B; A / B MN-major
+// when the flag is set (K-major otherwise).
+__host__ __device__ constexpr uint32_t instr_desc(int M, int N, bool a_mn, bool b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
+           ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate),
+        "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+        ::"r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+          "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+          "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+          "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]),
+          "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]),
+          "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]),
+          "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+          "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]),
+          "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+          "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* map, int c1,
+                                         int c2, uint64_t* bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::"
+        "complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(c1), "r"(c2),
+        "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_plain(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Barrier of the four softmax warps only.
+__device__ __forceinline__ void softmax_sync() {
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// Barrier of the softmax warps that returns how many threads passed `pred`.
+__device__ __forceinline__ int softmax_sync_count(bool pred) {
+    int n;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.popc.u32 %0, 1, 128, p;\n\t}"
+        : "=r"(n)
+        : "r"(pred ? 1u : 0u)
+        : "memory");
+    return n;
+}
+
+__device__ __forceinline__ void set_abort(int* flag, int* error_flags) {
+    if (atomicExch(flag, 1) == 0) report(error_flags, PA_DEVERR_TIMEOUT);
+}
+__device__ __forceinline__ bool aborted(int* flag) {
+    return *reinterpret_cast<volatile int*>(flag) != 0;
+}
+
+// Lane r ends with the reduction over the warp of row r of v (v is consumed).
+template <bool kMax>
+__device__ __forceinline__ float transpose_reduce(float (&v)[32], int lane) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < o; ++i) {
+            const float send = upper ? v[i] : v[i + o];
+            const float keep = upper ? v[i + o] : v[i];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, o);
+            v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+        }
+    }
+    return v[0];
+}
+
+__device__ __forceinline__ int clamp_len(const MultiRowParams& p, int s, bool report_errors) {
+    int L = p.context_lens[s];
+    if (L < 0 || L > p.max_context_len) {
+        if (report_errors) report(p.error_flags, PA_DEVERR_CONTEXT_LEN);
+        L = L < 0 ? 0 : p.max_context_len;
+    }
+    return L;
+}
+
+// Query count of sequence s in multi-query mode, clamped to [0, min(L, max_query_len)].
+__device__ __forceinline__ int clamp_queries(const MultiRowParams& p, int s, int L,
+                                             bool report_errors) {
+    int k = p.query_start_loc[s + 1] - p.query_start_loc[s];
+    if (k < 0 || k > L || k > p.max_query_len) {
+        if (report_errors) report(p.error_flags, PA_DEVERR_QUERY_LEN);
+        k = k < 0 ? 0 : min(k, min(L, p.max_query_len));
+    }
+    return k;
+}
+
+// Work item idx = (unit * tiles + tile) * Hkv + kv head.
+struct RowItem {
+    int unit;       // sequence or group; -1: nothing to do
+    int tile;
+    int g;
+    int table_seq;  // sequence whose block table is read
+    int range_end;  // tokens [0, range_end) are streamed
+    int nch;        // 128-token chunks
+};
+
+__device__ RowItem row_item(const MultiRowParams& p, int idx, bool report_errors) {
+    RowItem it;
+    it.unit = -1;
+    const int g = idx % p.num_kv_heads;
+    const int rest = idx / p.num_kv_heads;
+    const int tile = rest % p.tiles;
+    const int unit = rest / p.tiles;
+    const int G = p.group;
+    int range_end = 0, table_seq = 0;
+    if (!p.shared_prefix_mode) {
+        const int s = unit;
+        const int L = clamp_len(p, s, report_errors);
+        const int k = clamp_queries(p, s, L, report_errors && tile == 0 && g == 0);
+        const int r0 = tile * kN;
+        const int rows = min(kN, k * G - r0);
+        if (rows <= 0) return it;
+        range_end = L - k + (r0 + rows - 1) / G + 1;
+        table_seq = s;
+    } else {
+        const int P = cascade_group_prefix(p.groups, unit, p.num_seqs, p.block_size,
+                                           p.error_flags, report_errors);
+        if (P == 0) return it;
+        const int a = p.groups.group_start[unit];
+        const int b = p.groups.group_start[unit + 1];
+        const int mpt = kN / G;
+        const int m0 = a + tile * mpt;
+        const int m1 = min(b, m0 + mpt);
+        for (int s = m0; s < m1; ++s)
+            range_end = max(range_end, min(P, clamp_len(p, s, report_errors)));
+        table_seq = a;
+    }
+    if (range_end <= 0) return it;
+    it.unit = unit;
+    it.tile = tile;
+    it.g = g;
+    it.table_seq = table_seq;
+    it.range_end = range_end;
+    it.nch = (range_end + kTok - 1) / kTok;
+    return it;
+}
+
+// Row r of a live item: last visible token (lim) and the q / out row index
+// (-1 for a row that does not exist).
+__device__ void row_of(const MultiRowParams& p, const RowItem& it, int r, int& lim,
+                       long long& row) {
+    lim = -1;
+    row = -1;
+    const int G = p.group;
+    const int Hq = p.num_heads;
+    if (!p.shared_prefix_mode) {
+        const int s = it.unit;
+        const int L = clamp_len(p, s, false);
+        const int k = clamp_queries(p, s, L, false);
+        const int R = it.tile * kN + r;
+        if (R >= k * G) return;
+        const int j = R / G;
+        lim = L - k + j;
+        row = (long long)(p.query_start_loc[s] + j) * Hq + it.g * G + R % G;
+    } else {
+        const int mpt = kN / G;
+        const int m = r / G;
+        if (m >= mpt) return;
+        const int s = p.groups.group_start[it.unit] + it.tile * mpt + m;
+        if (s >= p.groups.group_start[it.unit + 1]) return;
+        const int P = cascade_group_prefix(p.groups, it.unit, p.num_seqs, p.block_size,
+                                           nullptr, false);
+        lim = min(P, clamp_len(p, s, false)) - 1;
+        row = (long long)s * Hq + it.g * G + r % G;
+    }
+}
+
+template <int BS>
+__global__ void __launch_bounds__(kThreads, 1)
+paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v,
+                       const MultiRowParams p, int num_items) {
+    extern __shared__ __align__(1024) unsigned char smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
+    uint64_t* k_full = bars;
+    uint64_t* k_empty = k_full + kKStages;
+    uint64_t* v_full = k_empty + kKStages;
+    uint64_t* v_empty = v_full + kVStages;
+    uint64_t* s_full = v_empty + kVStages;
+    uint64_t* p_full = s_full + 2;
+    uint64_t* pv_done = p_full + 2;
+    uint64_t* o_full = pv_done + 2;
+    uint64_t* o_empty = o_full + 2;
+    uint64_t* q_ready = o_empty + 2;
+    uint64_t* drain = q_ready + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
+    int* abort_flag = reinterpret_cast<int*>(smem + kBarOff + kNumBars * 8 + 4);
+    float* cmax = reinterpret_cast<float*>(smem + kCmaxOff);
+    float* red_l = reinterpret_cast<float*>(smem + kRedLOff);
+    float* item_m = reinterpret_cast<float*>(smem + kItemMOff);
+    int* row_lim = reinterpret_cast<int*>(smem + kRowLimOff);
+    long long* row_out = reinterpret_cast<long long*>(smem + kRowOutOff);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (smem_u32(smem) & 1023u) {
+        if (threadIdx.x == 0) report(p.error_flags, PA_DEVERR_INTERNAL);
+        return;
+    }
+    pdl_wait();
+    pdl_launch_dependents();
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kKStages; ++i) {
+            mbar_init(&k_full[i], 1);
+            mbar_init(&k_empty[i], 1);
+        }
+        for (int i = 0; i < kVStages; ++i) {
+            mbar_init(&v_full[i], 1);
+            mbar_init(&v_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&p_full[i], 128);
+            mbar_init(&pv_done[i], 1);
+            mbar_init(&o_full[i], 1);
+            mbar_init(&o_empty[i], 128);
+            mbar_init(&q_ready[i], 128);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
+    if (warp == 6) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint64_t pol = l2_policy_evict_first();
+
+    if (warp == 4 || warp == 5) {
+        // ------------------------------------------------ K / V producers
+        const bool is_v = warp == 5;
+        const int S = is_v ? kVStages : kKStages;
+        uint64_t* full = is_v ? v_full : k_full;
+        uint64_t* empty = is_v ? v_empty : k_empty;
+        const CUtensorMap* map = is_v ? &tm_v : &tm_k;
+        const uint32_t ring = smem_u32(smem + (is_v ? kVOff : kKOff));
+        int n = 0;  // chunks issued by this stream
+        bool ok = true;
+        for (int idx = blockIdx.x; idx < num_items && ok; idx += gridDim.x) {
+            const RowItem it = row_item(p, idx, false);
+            if (it.unit < 0) continue;
+            const int32_t* bt = p.block_tables + (int64_t)it.table_seq * p.max_blocks_per_seq;
+            int win = -1;  // lane l: slot of 16-token piece l of chunks c..c+3
+            for (int c = 0; c < it.nch; ++c) {
+                if ((c & 3) == 0) {
+                    const int t0 = (c * 8 + lane) * 16;
+                    int v = -1;
+                    if (t0 < it.range_end) {
+                        int id = bt[t0 / BS];
+                        if (id < 0 || id >= p.num_blocks) {
+                            report(p.error_flags, PA_DEVERR_BLOCK_ID);
+                            id = 0;
+                        }
+                        v = id * BS + t0 % BS;
+                    }
+                    win = v;
+                }
+                const int stage = n % S;
+                if (n >= S) {
+                    bool okw = true;
+                    if (lane == 0) okw = wait_bar(&empty[stage], ((n / S) - 1) & 1);
+                    if (__shfl_sync(0xffffffffu, okw ? 1 : 0, 0) == 0) {
+                        if (lane == 0) set_abort(abort_flag, p.error_flags);
+                        ok = false;
+                        break;
+                    }
+                }
+                if (aborted(abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const int sl = __shfl_sync(0xffffffffu, win, (c & 3) * 8 + (lane & 7));
+                const bool mine = lane < 8 && sl >= 0;
+                const uint32_t pieces = __popc(__ballot_sync(0xffffffffu, mine));
+                if (lane == 0) mbar_arrive_expect_tx(&full[stage], pieces * 2 * 2048);
+                __syncwarp();
+                if (mine) {
+                    const uint32_t dst = ring + stage * kStageBytes + lane * 2048;
+                    tma_load(dst, map, it.g * 2, sl, &full[stage], pol);
+                    tma_load(dst + kHalf, map, it.g * 2 + 1, sl, &full[stage], pol);
+                }
+                __syncwarp();
+                ++n;
+            }
+        }
+        // Copies still in flight land before the CTA may exit.
+        if (lane == 0)
+            for (int m = (n > S ? n - S : 0); m < n; ++m)
+                (void)wait_bar(&full[m % S], (m / S) & 1);
+    } else if (warp == 6) {
+        // -------------------------------------------------------- MMA issuer
+        constexpr uint32_t idesc_s = instr_desc(kTok, kN, false, false);
+        constexpr uint32_t idesc_pv = instr_desc(kD, 2 * kN, true, true);
+        struct Pending {
+            int n, valid, item;
+            bool first, last;
+        };
+        Pending pend = {0, 0, 0, false, false};
+        bool have_pend = false;
+        bool ok = true;
+
+        auto issue_pv = [&](const Pending& pd) -> bool {
+            const int vs = pd.n % kVStages;
+            bool good = __all_sync(0xffffffffu, wait_bar(&v_full[vs], (pd.n / kVStages) & 1));
+            if (good && lane == 0) good = wait_bar(&p_full[pd.n & 1], (pd.n >> 1) & 1);
+            if (good && lane == 0 && pd.first && pd.item >= 2)
+                good = wait_bar(&o_empty[pd.item & 1], ((pd.item - 2) >> 1) & 1);
+            good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+            if (!good) {
+                if (lane == 0) set_abort(abort_flag, p.error_flags);
+                return false;
+            }
+            if (pd.valid < kTok) {
+                // Token rows past the range hold stale or unwritten data; P
+                // is 0 there, but 0 x NaN is NaN.
+                unsigned char* vt = smem + kVOff + vs * kStageBytes;
+                const int rows = kTok - pd.valid;
+                for (int e = lane; e < rows * 16; e += 32) {
+                    const int r = pd.valid + (e >> 4);
+                    const int h = (e >> 3) & 1;
+                    *reinterpret_cast<uint4*>(vt + h * kHalf + r * 128 + (e & 7) * 16) =
+                        make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t v_base = smem_u32(smem + kVOff + vs * kStageBytes);
+                const uint32_t p_base = smem_u32(smem + kPOff + (pd.n & 1) * kPBytes);
+                const uint32_t d_tmem = tmem + kTmemO + (pd.item & 1) * 2 * kN;
+#pragma unroll
+                for (int kt = 0; kt < kTok / 16; ++kt) {
+                    // V^T: MN-major, M = d in two 64-wide swizzle columns
+                    // 16 KB apart (LBO), 8-token groups 1 KB apart (SBO).
+                    // [P_hi^T | P_lo^T]: MN-major, N = 64 = one swizzle column.
+                    const uint64_t ad = smem_desc(v_base + kt * 2048, kHalf, 1024);
+                    const uint64_t bd = smem_desc(p_base + kt * 2048, kPBytes, 1024);
+                    mma_ss(d_tmem, ad, bd, idesc_pv, (pd.first && kt == 0) ? 0u : 1u);
+                }
+                mma_commit(&v_empty[vs]);
+                mma_commit(&pv_done[pd.n & 1]);
+                if (pd.last) mma_commit(&o_full[pd.item & 1]);
+            }
+            __syncwarp();
+            return true;
+        };
+
+        int n = 0, item = 0;
+        for (int idx = blockIdx.x; idx < num_items && ok; idx += gridDim.x) {
+            const RowItem it = row_item(p, idx, false);
+            if (it.unit < 0) continue;
+            const uint32_t q_base = smem_u32(smem + kQOff + (item & 1) * kQBytes);
+            for (int c = 0; c < it.nch; ++c, ++n) {
+                bool good = true;
+                if (lane == 0) {
+                    if (c == 0) good = wait_bar(&q_ready[item & 1], (item >> 1) & 1);
+                    if (good) good = wait_bar(&k_full[n % kKStages], (n / kKStages) & 1);
+                }
+                good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+                if (!good || aborted(abort_flag)) {
+                    if (lane == 0) set_abort(abort_flag, p.error_flags);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t k_base = smem_u32(smem + kKOff + (n % kKStages) * kStageBytes);
+#pragma unroll
+                    for (int ks = 0; ks < kD / 16; ++ks) {
+                        const uint32_t off = (ks & 3) * 32;  // 16-wide d slice in the atom
+                        const uint64_t ad = smem_desc(k_base + (ks >> 2) * kHalf + off, 16, 1024);
+                        const uint64_t bd = smem_desc(q_base + (ks >> 2) * kQHalf + off, 16, 1024);
+                        mma_ss(tmem + (n & 1) * 32, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&s_full[n & 1]);
+                    mma_commit(&k_empty[n % kKStages]);
+                }
+                __syncwarp();
+                if (have_pend && !issue_pv(pend)) {
+                    ok = false;
+                    break;
+                }
+                pend.n = n;
+                pend.valid = min(kTok, it.range_end - c * kTok);
+                pend.item = item;
+                pend.first = c == 0;
+                pend.last = c == it.nch - 1;
+                have_pend = true;
+            }
+            ++item;
+        }
+        if (ok && have_pend) (void)issue_pv(pend);
+        if (lane == 0) {
+            mma_commit(drain);               // everything issued so far
+            (void)wait_bar(drain, 0);        // drained before TMEM goes away
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ softmax, epilogue
+        const int tid = threadIdx.x;             // 0..127: token of the chunk / d
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const float sl2 = p.scale_log2;
+
+        // Item setup: Q^T rows into Q buffer item%2 (K-major, 128-byte
+        // swizzle), row limits and output rows into slot item%3.
+        auto setup = [&](int idx, int item) {
+            const RowItem it = row_item(p, idx, false);
+            const int r = tid >> 2;
+            int lim;
+            long long row;
+            row_of(p, it, r, lim, row);
+            if ((tid & 3) == 0) {
+                row_lim[(item % 3) * 32 + r] = lim;
+                row_out[(item % 3) * 32 + r] = row;
+            }
+            const uint4* src = reinterpret_cast<const uint4*>(p.q + (row < 0 ? 0 : row) * kD);
+            unsigned char* qb = smem + kQOff + (item & 1) * kQBytes;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int c16 = (tid & 3) * 4 + u;
+                const uint4 v = row >= 0 ? src[c16] : make_uint4(0, 0, 0, 0);
+                const int h = c16 >> 3, cc = c16 & 7;
+                *reinterpret_cast<uint4*>(qb + h * kQHalf + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
+            }
+            fence_proxy_async_smem();
+            mbar_arrive_plain(&q_ready[item & 1]);
+        };
+
+        // Live items of this CTA in order.  Every item of the CTA is scanned
+        // exactly once here, so this is where bad inputs are reported.
+        auto next_live = [&](int from) -> int {
+            for (int idx = from; idx < num_items; idx += gridDim.x)
+                if (row_item(p, idx, tid == 0).unit >= 0) return idx;
+            return -1;
+        };
+
+        bool fail = false;  // a bounded wait of this thread gave up
+        bool stop = false;  // all four warps agreed to stop
+        int cur = next_live(blockIdx.x);
+        int nxt = cur >= 0 ? next_live(cur + gridDim.x) : -1;
+        if (cur >= 0) setup(cur, 0);
+        if (nxt >= 0) setup(nxt, 1);
+
+        // Epilogue of item i: O^T (thread = d) / l into the output rows.
+        auto epilogue = [&](int i) {
+            const int slot = i % 3;
+            const int ob = i & 1;
+            bool okw = __all_sync(0xffffffffu, wait_bar(&o_full[ob], (i >> 1) & 1));
+            if (!okw) {
+                fail = true;
+                return;
+            }
+            tc_fence_after();
+            uint32_t o[32], olo[32];
+            tmem_ld32(tmem + kTmemO + ob * 2 * kN + lane_off, o);
+            tmem_ld32(tmem + kTmemO + ob * 2 * kN + kN + lane_off, olo);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive_plain(&o_empty[ob]);
+#pragma unroll
+            for (int r = 0; r < 32; ++r) {
+                const long long row = row_out[slot * 32 + r];
+                if (row < 0) continue;
+                const float4 l4 = *reinterpret_cast<const float4*>(red_l + slot * 128 + r * 4);
+                const float l = (l4.x + l4.y) + (l4.z + l4.w);
+                const float acc = __uint_as_float(o[r]) + __uint_as_float(olo[r]);
+                p.out[row * kD + tid] = l > 0.f ? acc / l : 0.f;
+                if (p.shared_prefix_mode && tid == r) {
+                    p.out_m[row] = item_m[slot * 32 + r];
+                    p.out_l[row] = l;
+                }
+            }
+        };
+
+        float m_ref[32], l_part[32];
+#pragma unroll
+        for (int r = 0; r < 32; ++r) {
+            m_ref[r] = kNoMax;
+            l_part[r] = 0.f;
+        }
+        int n = 0, item = 0;
+        bool pending_epi = false;
+        // This token's 128-byte row of [P_hi^T | P_lo^T] (MN-major, 128-byte
+        // swizzle: 16-byte chunk j of row t sits at chunk j ^ (t % 8)).
+        const uint32_t p_row = (uint32_t)tid * 128;
+        const uint32_t p_sw = (uint32_t)(tid & 7);
+
+        while (cur >= 0 && !stop) {
+            // This item's row data (written one item earlier) is visible, and
+            // every warp is done with the slot the next setup overwrites.
+            softmax_sync();
+            const RowItem it = row_item(p, cur, false);
+            const int slot = item % 3;
+            int min_lim = 0x7fffffff;
+#pragma unroll
+            for (int r = 0; r < 32; ++r)
+                if (row_out[slot * 32 + r] >= 0) min_lim = min(min_lim, row_lim[slot * 32 + r]);
+            const int ob = item & 1;
+
+            for (int c = 0; c < it.nch; ++c, ++n) {
+                const int sb = n & 1;
+                bool ok = !fail && __all_sync(0xffffffffu, wait_bar(&s_full[sb], (n >> 1) & 1));
+                float x[32];
+                if (ok) {
+                    tc_fence_after();
+                    uint32_t raw[32];
+                    tmem_ld32(tmem + sb * 32 + lane_off, raw);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int r = 0; r < 32; ++r) x[r] = __uint_as_float(raw[r]) * sl2;
+                    const int tok = c * kTok + tid;
+                    if (c * kTok + kTok - 1 > min_lim) {
+#pragma unroll
+                        for (int r = 0; r < 32; ++r)
+                            if (tok > row_lim[slot * 32 + r]) x[r] = -INFINITY;
+                    }
+                } else {
+#pragma unroll
+                    for (int r = 0; r < 32; ++r) x[r] = -INFINITY;
+                }
+                bool grow = false;
+#pragma unroll
+                for (int r = 0; r < 32; ++r) grow = grow || x[r] > m_ref[r] + kRescaleThreshold;
+                if (lane == 0 && aborted(abort_flag)) ok = false;
+                ok = __all_sync(0xffffffffu, ok);
+                bool slow = softmax_sync_count(grow || !ok) != 0;
+                if (slow && softmax_sync_count(!ok) != 0) {
+                    if (tid == 0) set_abort(abort_flag, p.error_flags);
+                    stop = true;
+                    break;
+                }
+                if (slow) {
+                    // Exact chunk max per row, then move the references.
+                    float v[32];
+#pragma unroll
+                    for (int r = 0; r < 32; ++r) v[r] = x[r];
+                    cmax[lane * 4 + warp] = transpose_reduce<true>(v, lane);
+                    softmax_sync();
+                    float alpha[32];
+                    bool resc = false;
+#pragma unroll
+                    for (int r = 0; r < 32; ++r) {
+                        const float4 c4 = *reinterpret_cast<const float4*>(cmax + r * 4);
+                        const float cm = fmaxf(fmaxf(c4.x, c4.y), fmaxf(c4.z, c4.w));
+                        const float mn = fmaxf(m_ref[r], cm);
+                        alpha[r] = exp2f(m_ref[r] - mn);
+                        resc = resc || mn != m_ref[r];
+                        m_ref[r] = mn;
+                        l_part[r] *= alpha[r];
+                    }
+                    if (resc && c > 0) {
+                        // O^T must be stable: the previous PV has to be done.
+                        const bool okw = __all_sync(
+                            0xffffffffu, wait_bar(&pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1));
+                        if (okw) {
+                            tc_fence_after();
+#pragma unroll
+                            for (int part = 0; part < 2; ++part) {
+                                const uint32_t ta = tmem + kTmemO + ob * 2 * kN + part * kN + lane_off;
+                                uint32_t o[32];
+                                tmem_ld32(ta, o);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int r = 0; r < 32; ++r)
+                                    o[r] = __float_as_uint(__uint_as_float(o[r]) * alpha[r]);
+                                tmem_st32(ta, o);
+                            }
+                            tmem_wait_st();
+                        } else {
+                            fail = true;
+                        }
+                    }
+                }
+                // P buffer sb is free once PV(n-2) is done.
+                if (n >= 2 && !__all_sync(0xffffffffu,
+                                          wait_bar(&pv_done[sb], ((n - 2) >> 1) & 1)))
+                    fail = true;
+                // P = 2^(x - m) split by truncation: the high half keeps 8
+                // significant bits, the residual's high half another 8.
+                uint32_t hi[16], lo[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float a = exp2f(x[2 * i] - m_ref[2 * i]);
+                    const float b = exp2f(x[2 * i + 1] - m_ref[2 * i + 1]);
+                    l_part[2 * i] += a;
+                    l_part[2 * i + 1] += b;
+                    const uint32_t ab = __float_as_uint(a), bb = __float_as_uint(b);
+                    const float al = a - __uint_as_float(ab & 0xFFFF0000u);
+                    const float bl = b - __uint_as_float(bb & 0xFFFF0000u);
+                    hi[i] = __byte_perm(ab, bb, 0x7632);
+                    lo[i] = __byte_perm(__float_as_uint(al), __float_as_uint(bl), 0x7632);
+                }
+                unsigned char* prow = smem + kPOff + sb * kPBytes + p_row;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint32_t* src = j < 4 ? &hi[4 * j] : &lo[4 * (j - 4)];
+                    *reinterpret_cast<uint4*>(prow + ((j ^ p_sw) << 4)) =
+                        make_uint4(src[0], src[1], src[2], src[3]);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive_plain(&p_full[sb]);
+
+                if (c == 0) {
+                    if (pending_epi) epilogue(item - 1);
+                    pending_epi = false;
+                    if (item >= 1 && nxt >= 0) setup(nxt, item + 1);
+                }
+            }
+            if (stop) break;
+            // Item end: per-row sums over the 128 tokens' threads, the reference.
+            {
+                float v[32];
+#pragma unroll
+                for (int r = 0; r < 32; ++r) v[r] = l_part[r];
+                red_l[slot * 128 + lane * 4 + warp] = transpose_reduce<false>(v, lane);
+                float mine = 0.f;
+#pragma unroll
+                for (int r = 0; r < 32; ++r)
+                    if (r == lane) mine = m_ref[r];
+                if (warp == 0) item_m[slot * 32 + lane] = mine;
+#pragma unroll
+                for (int r = 0; r < 32; ++r) {
+                    m_ref[r] = kNoMax;
+                    l_part[r] = 0.f;
+                }
+            }
+            pending_epi = true;
+            cur = nxt;
+            nxt = cur >= 0 ? next_live(cur + gridDim.x) : -1;
+            ++item;
+        }
+        if (pending_epi && !stop) {
+            softmax_sync();  // the sums of the last item are in shared memory
+            epilogue(item - 1);
+        }
+        if (fail && tid == 0) set_abort(abort_flag, p.error_flags);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 6)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+                     ::"r"(tmem), "r"(kTmemCols)
+                     : "memory");
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
+                                   void*, const cuuint64_t*, const cuuint64_t*,
+                                   const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn mr_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr,
+                                    cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// Pool [NB*bs][Hkv][D] as {64 elements, Hkv*D/64 column tiles, NB*bs slots};
+// box = one 128-byte column tile of 16 slots.
+bool mr_encode_map(CUtensorMap* map, const void* pool, int num_blocks, int block_size,
+                   int num_kv_heads) {
+    EncodeTiledFn fn = mr_encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {64, (cuuint64_t)num_kv_heads * kD / 64,
+                                (cuuint64_t)num_blocks * block_size};
+    const cuuint64_t strides[2] = {128, (cuuint64_t)num_kv_heads * kD * 2};
+    const cuuint32_t box[3] = {64, 1, 16};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(pool), dims,
+              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+    static int sms[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return kNumSMs;
+    if (sms[dev] == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            v <= 0)
+            v = kNumSMs;
+        sms[dev] = v;
+    }
+    return sms[dev];
+}
+
+template <int BS>
+cudaError_t mr_launch_typed(const MultiRowParams& p, cudaStream_t stream) {
+    static int ready[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!__atomic_load_n(&ready[dev], __ATOMIC_ACQUIRE)) {
+        e = cudaFuncSetAttribute(paged_multi_row_kernel<BS>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess) return e;
+        __atomic_store_n(&ready[dev], 1, __ATOMIC_RELEASE);
+    }
+    CUtensorMap tmk, tmv;
+    if (!mr_encode_map(&tmk, p.k_cache, p.num_blocks, BS, p.num_kv_heads) ||
+        !mr_encode_map(&tmv, p.v_cache, p.num_blocks, BS, p.num_kv_heads))
+        return cudaErrorInvalidValue;
+    const long long items = (long long)p.num_units * p.tiles * p.num_kv_heads;
+    if (items <= 0) return cudaSuccess;
+    if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const int grid = (int)(items < num_sms() ? items : num_sms());
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, paged_multi_row_kernel<BS>, tmk, tmv, p, (int)items);
+    count_launch();
+    return e;
+}
+
+}  // namespace
+
+cudaError_t launch_paged_multi_row(const MultiRowParams& p, cudaStream_t stream) {
+    if (p.block_size == 16) return mr_launch_typed<16>(p, stream);
+    if (p.block_size == 32) return mr_launch_typed<32>(p, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace pa

@@ -1,0 +1,50 @@
+// Internal interface of the tcgen05 kernel for up to 32 query rows per kv
+// head (pa_multi_row.cu): speculative verification in the multi-query call
+// and the group pass of the shared-prefix call.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "pa_cascade.cuh"
+
+namespace pa {
+
+struct MultiRowParams {
+    // Multi-query mode: out fp32 [T][Hq][D], normalised.  Shared-prefix mode:
+    // out fp32 [B][Hq][D] holds each row's partial O / l over its shared
+    // tokens, out_m / out_l fp32 [B][Hq] the matching running max (log2
+    // domain, scaled) and sum.
+    float* out;
+    float* out_m;
+    float* out_l;
+    const uint16_t* q;               // bf16 [T or B][Hq][D]
+    const uint16_t* k_cache;         // bf16 [NB][bs][Hkv][D]
+    const uint16_t* v_cache;
+    const int32_t* block_tables;     // int32 [B][max_blocks_per_seq]
+    const int32_t* context_lens;     // int32 [B]
+    const int32_t* query_start_loc;  // int32 [B+1] (multi-query mode)
+    CascadeGroups groups;            // shared-prefix mode
+    int* error_flags;                // nullable
+    int shared_prefix_mode;
+    int num_seqs;
+    int max_blocks_per_seq;
+    int max_context_len;
+    int max_query_len;
+    int num_heads;
+    int num_kv_heads;
+    int num_blocks;
+    int block_size;
+    int group;                       // num_heads / num_kv_heads
+    int tiles;                       // 32-row tiles per sequence or group
+    int num_units;                   // sequences or groups
+    float scale_log2;                // scale * log2(e)
+};
+
+// Rows handled per tile.
+constexpr int kMultiRowTile = 32;
+
+// head_size 128 only; block_size 16 or 32.
+cudaError_t launch_paged_multi_row(const MultiRowParams& p, cudaStream_t stream);
+
+}  // namespace pa

@@ -129,6 +129,11 @@ class DecodeCase:
     # queries; q / new_key / new_value / slot_mapping then have sum(k_s) rows
     query_start_loc: Optional[torch.Tensor] = None   # int32 [B+1]
     query_lens_np: Optional[np.ndarray] = None        # int64 [B]
+    # shared-prefix cases: sequences group_start[i] .. group_start[i+1]-1
+    # share their first prefix_lens[i] tokens (whole blocks)
+    group_start: Optional[torch.Tensor] = None        # int32 [G+1]
+    prefix_lens: Optional[torch.Tensor] = None        # int32 [G]
+    max_group_size: int = 0
 
     @property
     def scale(self) -> float:
@@ -238,9 +243,16 @@ def build_shared_prefix_case(w: Workload, device="cpu",
             tables[s, pblk:pblk + n] = perm[cursor:cursor + n]
             cursor += n
     unique = P * (pblk - 1) * bs + B * bs + int(tails.sum())
-    return _finish(w, lens, tables, NB, pairs, device,
+    case = _finish(w, lens, tables, NB, pairs, device,
                    2000 + w.wid if seed is None else seed + 1, pool_device,
                    unique_tokens=unique)
+    # The samples of a prompt share its blocks up to the copied last one.
+    dev = torch.device(device)
+    gs = (np.arange(P + 1) * S).astype(np.int32)
+    pl = np.full(P, (pblk - 1) * bs, dtype=np.int32)
+    return dataclasses.replace(case, group_start=torch.from_numpy(gs).to(dev),
+                               prefix_lens=torch.from_numpy(pl).to(dev),
+                               max_group_size=S)
 
 
 def _finish(w: Workload, lens, tables, NB, pairs, device, vseed, pool_device,
@@ -350,3 +362,54 @@ def multi_query_case(num_seqs: int, num_heads: int, num_kv_heads: int,
         base, q=q.to(dev), new_key=nk.to(dev), new_value=nv.to(dev),
         slot_mapping=torch.from_numpy(slots).to(dev),
         query_start_loc=torch.from_numpy(qsl).to(dev), query_lens_np=qlens)
+
+
+def grouped_case(num_heads: int, num_kv_heads: int, head_size: int,
+                 block_size: int, lens, group_start, prefix_lens, seed: int,
+                 device="cpu", max_group_size: Optional[int] = None) -> DecodeCase:
+    """Sequences whose block tables share leading blocks.  Sequence s of
+    group i (group_start[i] <= s < group_start[i+1]) maps its first
+    min(L_s, P_i) tokens (P_i = prefix_lens[i], whole blocks) to the group's
+    blocks and the rest to private blocks; sequences outside every group
+    have private blocks only.  Block ids are a seeded permutation of the
+    pool.  No step writes: only the attention inputs are meaningful."""
+    lens = np.asarray(lens, dtype=np.int64)
+    gs = np.asarray(group_start, dtype=np.int32)
+    pl = np.asarray(prefix_lens, dtype=np.int32)
+    B, bs = len(lens), block_size
+    rng = np.random.default_rng(seed)
+    shared_of = np.zeros(B, dtype=np.int64)   # tokens mapped to group blocks
+    owner = np.full(B, -1)
+    for i in range(len(pl)):
+        for s in range(int(gs[i]), int(gs[i + 1])):
+            owner[s] = i
+            shared_of[s] = min(int(lens[s]), int(pl[i]))
+    group_blocks = [int(pl[i]) // bs for i in range(len(pl))]
+    private = [int(blocks_for(np.array([lens[s] - shared_of[s]]), bs)[0])
+               for s in range(B)]
+    need = sum(group_blocks) + sum(private)
+    NB = max(1, math.ceil(need * (1 + POOL_SLACK)) + 1)
+    perm = rng.permutation(NB).astype(np.int32)
+    cursor = 0
+    gblk = []
+    for n in group_blocks:
+        gblk.append(perm[cursor:cursor + n])
+        cursor += n
+    MB = max(1, int(max(blocks_for(lens, bs).max(initial=0), 1)))
+    tables = np.full((B, MB), -1, dtype=np.int32)
+    for s in range(B):
+        nsh = int(blocks_for(np.array([shared_of[s]]), bs)[0])
+        if owner[s] >= 0 and nsh:
+            tables[s, :nsh] = gblk[owner[s]][:nsh]
+        n = private[s]
+        tables[s, nsh:nsh + n] = perm[cursor:cursor + n]
+        cursor += n
+    w = Workload(f"grouped{seed}", 0, B, num_heads, num_kv_heads, head_size,
+                 block_size, "fixed")
+    case = _finish(w, lens, tables, NB, np.zeros((0, 2), dtype=np.int64),
+                   device, seed + 1, None, unique_tokens=0)
+    dev = torch.device(device)
+    mgs = int(np.max(np.diff(gs), initial=1)) if max_group_size is None else max_group_size
+    return dataclasses.replace(case, group_start=torch.from_numpy(gs).to(dev),
+                               prefix_lens=torch.from_numpy(pl).to(dev),
+                               max_group_size=max(1, mgs))

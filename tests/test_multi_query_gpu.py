@@ -119,3 +119,33 @@ def test_query_count_above_context_sets_flag():
                                 error_flags=flags)
     torch.cuda.synchronize()
     assert int(flags.item()) & pa.PA_DEVERR_QUERY_LEN
+
+
+ROWS_SHAPES = [
+    (64, 8, 128, 16, [300, 1000, 17, 4096], [4, 4, 4, 4]),      # spec verify
+    (32, 8, 128, 32, [700, 64, 129], [5, 3, 8]),
+    (16, 16, 128, 16, [257, 40, 90], [2, 1, 7]),                # MHA
+    (4, 4, 128, 16, [1, 2, 3], [1, 2, 3]),
+    (32, 2, 128, 16, [2048, 300], [200, 64]),                   # G=16, 100 tiles
+    (24, 8, 128, 16, [129, 128, 127, 1000], [11, 1, 16, 3]),    # G=3, ragged tiles
+]
+
+
+@pytest.mark.parametrize("Hq,Hkv,D,bs,lens,qlens", ROWS_SHAPES)
+def test_multi_row_kernel_shapes(monkeypatch, Hq, Hkv, D, bs, lens, qlens):
+    """The tcgen05 kernel for <= 32 rows per tile (tokens as the MMA's M),
+    forced for every shape: 32-row tiles of (query token, head) rows."""
+    monkeypatch.setenv("PA_MULTI_QUERY_KERNEL", "rows")
+    case = inputs.multi_query_case(len(lens), Hq, Hkv, D, bs, lens, qlens,
+                                   seed=sum(lens) + Hq + 1, device="cuda")
+    check(case)
+
+
+def test_multi_row_kernel_spec_verify_batch256(monkeypatch):
+    monkeypatch.setenv("PA_MULTI_QUERY_KERNEL", "rows")
+    test_speculative_verify_batch256_sampled()
+
+
+def test_multi_row_kernel_determinism(monkeypatch):
+    monkeypatch.setenv("PA_MULTI_QUERY_KERNEL", "rows")
+    test_run_to_run_determinism()

@@ -1,0 +1,144 @@
+"""pa_decode_attention_shared_prefix on the GPU through the C ABI against the
+fp64 oracle.  The oracle knows nothing of groups: it attends every sequence
+over its whole block table, so these tests check that the group pass (shared
+blocks read once for all members' rows, tcgen05) plus the per-sequence pass
+and their merge reproduce plain paged attention ("Memory Sharing via
+Copy-on-Write (CoW)": parallel samples share the prompt's blocks).
+Tolerance as for decode: max-abs <= 4e-3 and relative L2 <= 1e-3."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_435_b200 as pa
+from paged_kv_cache_435_b200 import inputs
+from tests.helpers import assert_attn_close, bits
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _need_gpu():
+    assert torch.cuda.is_available(), "GPU test run without a CUDA device"
+
+
+def run(case, flags=None, partition_size=0, group_start=None, prefix_lens=None,
+        max_group_size=None):
+    B, Hq, D = case.q.shape
+    Hkv, bs = case.workload.num_kv_heads, case.workload.block_size
+    gs = case.group_start if group_start is None else group_start
+    pl = case.prefix_lens if prefix_lens is None else prefix_lens
+    mgs = case.max_group_size if max_group_size is None else max_group_size
+    out = torch.full((B, Hq, D), float("nan"), dtype=torch.float32, device="cuda")
+    nbytes = pa.pa_shared_prefix_workspace_size(B, Hq, Hkv, D, bs,
+                                                case.max_context_len,
+                                                partition_size)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    pa.pa_decode_attention_shared_prefix(
+        out, case.q, case.k_cache, case.v_cache, case.block_tables,
+        case.context_lens, gs.cuda(), pl.cuda(), case.max_context_len, mgs,
+        case.scale, ws, partition_size=partition_size, error_flags=flags)
+    return out
+
+
+def reference(case):
+    return oracle.paged_decode_attention(
+        case.q.cpu(), bits(case.k_cache), bits(case.v_cache), case.tables_np,
+        case.lens_np.astype(np.int32), case.scale, case.workload.num_kv_heads)
+
+
+def check(case, expect_flags=0, **kw):
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = run(case, flags, **kw)
+    torch.cuda.synchronize()
+    assert int(flags.item()) == expect_flags
+    return assert_attn_close(out, reference(case), case.workload.name), out
+
+
+def test_parallel_sampling_workload():
+    """32 prompts x 8 samples (32q/8kv, D=128, bs=16): the copy-on-write step
+    and the new token's write run first; groups share 63 of the 64 prompt
+    blocks (the 64th is each sample's private copy)."""
+    case = inputs.make_case("shared_prefix_cow", device="cuda")
+    ek, ev = bits(case.k_cache), bits(case.v_cache)
+    pa.pa_copy_blocks([case.k_cache], [case.v_cache], case.copy_pairs)
+    pa.pa_reshape_and_cache(case.new_key, case.new_value, case.k_cache,
+                            case.v_cache, case.slot_mapping)
+    oracle.copy_blocks([ek], [ev], case.copy_pairs.cpu().numpy())
+    oracle.reshape_and_cache(case.new_key.cpu(), case.new_value.cpu(), ek, ev,
+                             case.slot_mapping.cpu().numpy())
+    (_, _), out = check(case)
+    # The plain decode call on the same inputs agrees within rounding.
+    B, Hq, D = case.q.shape
+    plain = torch.empty_like(out)
+    pa.pa_decode_attention(plain, case.q, case.k_cache, case.v_cache,
+                           case.block_tables, case.context_lens,
+                           case.max_context_len, case.scale)
+    torch.cuda.synchronize()
+    assert (plain - out).abs().max().item() <= 2e-5
+
+
+@pytest.mark.parametrize("Hq,Hkv,bs", [(32, 8, 16), (64, 8, 16), (8, 8, 32),
+                                       (24, 8, 16), (64, 8, 32)])
+def test_group_shapes(Hq, Hkv, bs):
+    """G = 4, 8, 1, 3 and both block sizes.  Groups of 8, 5, 1 and 12 members
+    (G=8 x 12 members = 3 row tiles), a member shorter than its prefix, two
+    whose context ends exactly at the prefix, a group with prefix 0 in the
+    middle of the batch and sequences after the last group."""
+    P0, P1, P2, P3 = 20 * bs, 6 * bs, 3 * bs, 40 * bs
+    lens = ([P0 + t for t in (1, 17, 200, 0, 33, 5, 64, 129)] +   # [0, 8)
+            [P1 + 3, P1 - bs - 3, P1 + 90, P1, P1 + 1] +            # [8, 13)
+            [555] +                                                 # [13, 14), P=0
+            [P2 + 7] +                                              # [14, 15)
+            [P3 + 11 * t for t in range(12)] +                      # [15, 27)
+            [42, 1])                                                # no group
+    gs = [0, 8, 13, 14, 15, 27]
+    pl = [P0, P1, 0, P2, P3]
+    case = inputs.grouped_case(Hq, Hkv, 128, bs, lens, gs, pl, seed=Hq + bs,
+                               device="cuda")
+    check(case)
+
+
+def test_split_suffix_and_determinism():
+    """Long private tails with 64-token partitions: the split merge kernel
+    folds in the group pass's partial; repeated calls are bitwise equal."""
+    bs = 16
+    lens = [512 + 700, 512 + 1, 512 + 333, 300, 512 + 64]
+    case = inputs.grouped_case(32, 8, 128, bs, lens, [0, 3], [512], seed=77,
+                               device="cuda")
+    (_, _), a = check(case, partition_size=64)
+    b = run(case, partition_size=64)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_invalid_groups_are_flagged_and_still_exact():
+    """A prefix that is not a multiple of the block size, a group larger than
+    max_group_size and an inverted group all fall back to the per-sequence
+    pass (PA_DEVERR_PREFIX) with exact results."""
+    bs = 16
+    lens = [200, 210, 220, 230, 240, 250, 260, 270]
+    case = inputs.grouped_case(32, 8, 128, bs, lens, [0, 2, 5, 8], [64, 64, 48],
+                               seed=3, device="cuda")
+    check(case, expect_flags=pa.PA_DEVERR_PREFIX,
+          prefix_lens=torch.tensor([64, 72, 48], dtype=torch.int32))
+    check(case, expect_flags=pa.PA_DEVERR_PREFIX, max_group_size=2)
+    check(case, expect_flags=pa.PA_DEVERR_PREFIX,
+          group_start=torch.tensor([0, 2, 1, 8], dtype=torch.int32),
+          prefix_lens=torch.tensor([64, 0, 0], dtype=torch.int32))
+
+
+def test_no_groups_is_plain_decode():
+    case = inputs.custom_case(6, 32, 8, 128, 16, [1, 16, 17, 100, 1000, 3000],
+                              seed=11, device="cuda")
+    out = torch.empty(case.q.shape, dtype=torch.float32, device="cuda")
+    B, Hq, D = case.q.shape
+    ws = torch.empty(pa.pa_shared_prefix_workspace_size(
+        B, Hq, 8, D, 16, case.max_context_len), dtype=torch.uint8, device="cuda")
+    empty = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.pa_decode_attention_shared_prefix(
+        out, case.q, case.k_cache, case.v_cache, case.block_tables,
+        case.context_lens, empty, empty[:0], case.max_context_len, 1,
+        case.scale, ws)
+    torch.cuda.synchronize()
+    assert_attn_close(out, reference(case), "no groups")
