@@ -25,14 +25,18 @@
 // at the end.  Accumulators live in tensor memory: S^T double-buffered (2 x 32
 // columns), O^T double-buffered across items (2 x 64 columns).
 //
-// CTA: 7 warps, one CTA per SM, persistent over items (row tile, kv head):
+// CTA: 8 warps, one CTA per SM, persistent over items (row tile, kv head):
 //   warps 0-3  softmax: thread i owns token i of the chunk (TMEM lane i) and
 //              all 32 rows; P = 2^(s - m) as bf16 high part + bf16 residual
 //              (~16 bits into the PV product), one 128-byte row of P^T;
 //   warp 4     K producer, warp 5 V producer: 16-token TMA tensor tiles
 //              (128-byte swizzle) of each 128-token chunk into 2- and 3-stage
 //              rings (V waits for the softmax, so it runs deeper);
-//   warp 6     TMEM allocation and the MMA issue (one thread).
+//   warp 6     TMEM allocation and the MMA issue (one thread);
+//   warp 7     scheduler: works out the CTA's next items (token range, block
+//              table row, each row's limit and output row) into a 4-slot
+//              shared-memory ring and copies their Q rows (cp.async), so no
+//              other warp waits on a global load at an item boundary.
 // Online softmax with a lazy reference: every chunk, one barrier-reduction
 // over the 4 warps (bar.red.popc) asks whether any row's logit exceeds its
 // reference max by more than 2^8; only then is the exact per-row chunk max
@@ -60,7 +64,8 @@ constexpr int kN = kMultiRowTile;         // rows (N of both products)
 constexpr int kD = 128;
 constexpr int kKStages = 2;
 constexpr int kVStages = 3;
-constexpr int kThreads = 224;
+constexpr int kThreads = 256;
+constexpr int kSlots = 4;                 // items published ahead by the scheduler
 constexpr int kHalf = kTok * 128;         // 16 KB: 128 tokens x 64 d (one swizzle column)
 constexpr int kStageBytes = 2 * kHalf;    // 32 KB: one chunk of K or V
 constexpr int kQHalf = kN * 128;          // 4 KB: 32 rows x 64 d
@@ -72,14 +77,27 @@ constexpr int kQOff = kVOff + kVStages * kStageBytes;  // 2 item buffers
 constexpr int kPOff = kQOff + 2 * kQBytes;             // 2 chunk buffers x (hi | lo)
 constexpr int kMiscOff = kPOff + 2 * kPBytes;
 constexpr int kCmaxOff = kMiscOff;                     // float [32][4]
-constexpr int kRedLOff = kCmaxOff + 512;               // float [3][32][4]
-constexpr int kItemMOff = kRedLOff + 3 * 512;          // float [3][32]
-constexpr int kRowLimOff = kItemMOff + 3 * 128;        // int [3][32]
-constexpr int kRowOutOff = kRowLimOff + 3 * 128;       // int64 [3][32]
-constexpr int kBarOff = kRowOutOff + 3 * 256;
+
+// One published item: what every role needs, and the per-row results the
+// epilogue writes out.
+struct ItemSlot {
+    int table_seq, g, range_end, nch;   // nch < 0: no further items
+    int min_lim, pad[3];                // smallest limit over existing rows
+    int lim[32];                        // last visible token of each row
+    long long row[32];                  // q / out row of each row (-1: none)
+    float red_l[32][4];                 // per-warp partial row sums
+    float m[32];                        // reference max of each row
+    float l[32];                        // row sums
+    float inv_l[32];                    // 1 / row sum (0 for an empty row)
+};
+static_assert(sizeof(ItemSlot) == 1312, "slot layout");
+
+constexpr int kSlotOff = kCmaxOff + 512;
+constexpr int kBarOff = kSlotOff + kSlots * (int)sizeof(ItemSlot);
 // barriers: k_full[KS] k_empty[KS] v_full[VS] v_empty[VS] s_full[2] p_full[2]
-//           pv_done[2] o_full[2] o_empty[2] q_ready[2] drain
-constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 11;
+//           pv_done[2] o_full[2] o_empty[2] q_empty[2] item_ready[4]
+//           slot_free[4] drain
+constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 13 + 2 * kSlots;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16;
 constexpr uint32_t kTmemCols = 256;       // S0 | S1 | O0 (hi, lo) | O1 (hi, lo)
 constexpr uint32_t kTmemO = 64;           // first O column
@@ -89,7 +107,7 @@ constexpr int kNumSMs = 148;
 
 static_assert(kStageBytes % 1024 == 0 && kQBytes % 1024 == 0 && kPBytes % 1024 == 0,
               "swizzled tiles need 1024-byte alignment");
-static_assert(kRowOutOff % 8 == 0 && kBarOff % 8 == 0, "8-byte alignment");
+static_assert(kSlotOff % 16 == 0 && kBarOff % 8 == 0, "alignment");
 static_assert(kSmemBytes <= 232448, "shared memory");
 
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity) {
@@ -181,6 +199,16 @@ __device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* map, i
         "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(c1), "r"(c2),
         "r"(smem_u32(bar)), "l"(policy)
         : "memory");
+}
+
+// 16-byte global -> shared copy; bytes past src_bytes (0 or 16) are zero.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_plain(uint64_t* bar) {
@@ -347,15 +375,14 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
     uint64_t* pv_done = p_full + 2;
     uint64_t* o_full = pv_done + 2;
     uint64_t* o_empty = o_full + 2;
-    uint64_t* q_ready = o_empty + 2;
-    uint64_t* drain = q_ready + 2;
+    uint64_t* q_empty = o_empty + 2;
+    uint64_t* item_ready = q_empty + 2;
+    uint64_t* slot_free = item_ready + kSlots;
+    uint64_t* drain = slot_free + kSlots;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
     int* abort_flag = reinterpret_cast<int*>(smem + kBarOff + kNumBars * 8 + 4);
     float* cmax = reinterpret_cast<float*>(smem + kCmaxOff);
-    float* red_l = reinterpret_cast<float*>(smem + kRedLOff);
-    float* item_m = reinterpret_cast<float*>(smem + kItemMOff);
-    int* row_lim = reinterpret_cast<int*>(smem + kRowLimOff);
-    long long* row_out = reinterpret_cast<long long*>(smem + kRowOutOff);
+    ItemSlot* slots = reinterpret_cast<ItemSlot*>(smem + kSlotOff);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -382,12 +409,21 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             mbar_init(&pv_done[i], 1);
             mbar_init(&o_full[i], 1);
             mbar_init(&o_empty[i], 128);
-            mbar_init(&q_ready[i], 128);
+            mbar_init(&q_empty[i], 1);
+        }
+        for (int i = 0; i < kSlots; ++i) {
+            mbar_init(&item_ready[i], 32);
+            mbar_init(&slot_free[i], 128);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
         mbar_init_fence();
     }
+    // V stages start zeroed: the token rows a tail chunk does not load must be
+    // finite (P is 0 there, but 0 x NaN is NaN).
+    for (int i = threadIdx.x; i < kVStages * kStageBytes / 16; i += kThreads)
+        reinterpret_cast<uint4*>(smem + kVOff)[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
     if (warp == 6) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols)
@@ -400,7 +436,66 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
     const uint32_t tmem = *tmem_slot;
     const uint64_t pol = l2_policy_evict_first();
 
-    if (warp == 4 || warp == 5) {
+    if (warp == 7) {
+        // -------------------------------------------------------- scheduler
+        int live = 0;
+        for (int idx = blockIdx.x;; idx += gridDim.x) {
+            const bool end = idx >= num_items;
+            RowItem it;
+            it.unit = -1;
+            if (!end) {
+                it = row_item(p, idx, lane == 0);
+                if (it.unit < 0) continue;
+            }
+            const int s = live % kSlots;
+            bool good = true;
+            // The slot's previous item has been written out.
+            if (lane == 0 && live >= kSlots)
+                good = wait_bar(&slot_free[s], ((live / kSlots) - 1) & 1);
+            // The Q buffer's previous item (live - 2) has had all its S products.
+            if (good && lane == 0 && !end && live >= 2)
+                good = wait_bar(&q_empty[live & 1], ((live - 2) >> 1) & 1);
+            if (__shfl_sync(0xffffffffu, good ? 1 : 0, 0) == 0) {
+                if (lane == 0) set_abort(abort_flag, p.error_flags);
+                break;
+            }
+            ItemSlot& S = slots[s];
+            if (end) {
+                if (lane == 0) S.nch = -1;
+                mbar_arrive_plain(&item_ready[s]);
+                break;
+            }
+            int lim;
+            long long row;
+            row_of(p, it, lane, lim, row);
+            S.lim[lane] = lim;
+            S.row[lane] = row;
+            int ml = row >= 0 ? lim : 0x7fffffff;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) ml = min(ml, __shfl_xor_sync(0xffffffffu, ml, o));
+            if (lane == 0) {
+                S.table_seq = it.table_seq;
+                S.g = it.g;
+                S.range_end = it.range_end;
+                S.nch = it.nch;
+                S.min_lim = ml;
+            }
+            // Q^T row `lane` (K-major, 128-byte swizzle; zeros for a missing row).
+            const uint32_t qb = smem_u32(smem + kQOff + (live & 1) * kQBytes);
+            const unsigned char* src =
+                reinterpret_cast<const unsigned char*>(p.q + (row < 0 ? 0 : row) * kD);
+            const int nbytes = row < 0 ? 0 : 16;
+#pragma unroll
+            for (int c16 = 0; c16 < 16; ++c16)
+                cp_async_16(qb + (c16 >> 3) * kQHalf + lane * 128 +
+                                (((c16 & 7) ^ (lane & 7)) << 4),
+                            src + c16 * 16, nbytes);
+            cp_async_wait_all();
+            fence_proxy_async_smem();
+            mbar_arrive_plain(&item_ready[s]);
+            ++live;
+        }
+    } else if (warp == 4 || warp == 5) {
         // ------------------------------------------------ K / V producers
         const bool is_v = warp == 5;
         const int S = is_v ? kVStages : kKStages;
@@ -410,16 +505,23 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
         const uint32_t ring = smem_u32(smem + (is_v ? kVOff : kKOff));
         int n = 0;  // chunks issued by this stream
         bool ok = true;
-        for (int idx = blockIdx.x; idx < num_items && ok; idx += gridDim.x) {
-            const RowItem it = row_item(p, idx, false);
-            if (it.unit < 0) continue;
-            const int32_t* bt = p.block_tables + (int64_t)it.table_seq * p.max_blocks_per_seq;
+        for (int item = 0; ok; ++item) {
+            const int sl = item % kSlots;
+            if (!__all_sync(0xffffffffu, wait_bar(&item_ready[sl], (item / kSlots) & 1))) {
+                if (lane == 0) set_abort(abort_flag, p.error_flags);
+                break;
+            }
+            const int nch = slots[sl].nch;
+            if (nch < 0) break;
+            const int g = slots[sl].g;
+            const int range_end = slots[sl].range_end;
+            const int32_t* bt = p.block_tables + (int64_t)slots[sl].table_seq * p.max_blocks_per_seq;
             int win = -1;  // lane l: slot of 16-token piece l of chunks c..c+3
-            for (int c = 0; c < it.nch; ++c) {
+            for (int c = 0; c < nch; ++c) {
                 if ((c & 3) == 0) {
                     const int t0 = (c * 8 + lane) * 16;
                     int v = -1;
-                    if (t0 < it.range_end) {
+                    if (t0 < range_end) {
                         int id = bt[t0 / BS];
                         if (id < 0 || id >= p.num_blocks) {
                             report(p.error_flags, PA_DEVERR_BLOCK_ID);
@@ -443,15 +545,15 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                     ok = false;
                     break;
                 }
-                const int sl = __shfl_sync(0xffffffffu, win, (c & 3) * 8 + (lane & 7));
-                const bool mine = lane < 8 && sl >= 0;
+                const int sl16 = __shfl_sync(0xffffffffu, win, (c & 3) * 8 + (lane & 7));
+                const bool mine = lane < 8 && sl16 >= 0;
                 const uint32_t pieces = __popc(__ballot_sync(0xffffffffu, mine));
                 if (lane == 0) mbar_arrive_expect_tx(&full[stage], pieces * 2 * 2048);
                 __syncwarp();
                 if (mine) {
                     const uint32_t dst = ring + stage * kStageBytes + lane * 2048;
-                    tma_load(dst, map, it.g * 2, sl, &full[stage], pol);
-                    tma_load(dst + kHalf, map, it.g * 2 + 1, sl, &full[stage], pol);
+                    tma_load(dst, map, g * 2, sl16, &full[stage], pol);
+                    tma_load(dst + kHalf, map, g * 2 + 1, sl16, &full[stage], pol);
                 }
                 __syncwarp();
                 ++n;
@@ -484,11 +586,11 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 if (lane == 0) set_abort(abort_flag, p.error_flags);
                 return false;
             }
-            if (pd.valid < kTok) {
-                // Token rows past the range hold stale or unwritten data; P
-                // is 0 there, but 0 x NaN is NaN.
+            if (pd.valid % 16 != 0) {
+                // The last loaded 16-token piece ends past the range: its
+                // extra token rows hold whatever the block holds.
                 unsigned char* vt = smem + kVOff + vs * kStageBytes;
-                const int rows = kTok - pd.valid;
+                const int rows = 16 - pd.valid % 16;
                 for (int e = lane; e < rows * 16; e += 32) {
                     const int r = pd.valid + (e >> 4);
                     const int h = (e >> 3) & 1;
@@ -520,17 +622,22 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             return true;
         };
 
-        int n = 0, item = 0;
-        for (int idx = blockIdx.x; idx < num_items && ok; idx += gridDim.x) {
-            const RowItem it = row_item(p, idx, false);
-            if (it.unit < 0) continue;
+        int n = 0;
+        for (int item = 0; ok; ++item) {
+            const int sl = item % kSlots;
+            // Also covers the item's Q rows, copied before publication.
+            if (!__all_sync(0xffffffffu, wait_bar(&item_ready[sl], (item / kSlots) & 1))) {
+                if (lane == 0) set_abort(abort_flag, p.error_flags);
+                ok = false;
+                break;
+            }
+            const int nch = slots[sl].nch;
+            if (nch < 0) break;
+            const int range_end = slots[sl].range_end;
             const uint32_t q_base = smem_u32(smem + kQOff + (item & 1) * kQBytes);
-            for (int c = 0; c < it.nch; ++c, ++n) {
+            for (int c = 0; c < nch; ++c, ++n) {
                 bool good = true;
-                if (lane == 0) {
-                    if (c == 0) good = wait_bar(&q_ready[item & 1], (item >> 1) & 1);
-                    if (good) good = wait_bar(&k_full[n % kKStages], (n / kKStages) & 1);
-                }
+                if (lane == 0) good = wait_bar(&k_full[n % kKStages], (n / kKStages) & 1);
                 good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
                 if (!good || aborted(abort_flag)) {
                     if (lane == 0) set_abort(abort_flag, p.error_flags);
@@ -549,6 +656,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                     }
                     mma_commit(&s_full[n & 1]);
                     mma_commit(&k_empty[n % kKStages]);
+                    if (c == nch - 1) mma_commit(&q_empty[item & 1]);
                 }
                 __syncwarp();
                 if (have_pend && !issue_pv(pend)) {
@@ -556,13 +664,12 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                     break;
                 }
                 pend.n = n;
-                pend.valid = min(kTok, it.range_end - c * kTok);
+                pend.valid = min(kTok, range_end - c * kTok);
                 pend.item = item;
                 pend.first = c == 0;
-                pend.last = c == it.nch - 1;
+                pend.last = c == nch - 1;
                 have_pend = true;
             }
-            ++item;
         }
         if (ok && have_pend) (void)issue_pv(pend);
         if (lane == 0) {
@@ -575,52 +682,24 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
         const int tid = threadIdx.x;             // 0..127: token of the chunk / d
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         const float sl2 = p.scale_log2;
-
-        // Item setup: Q^T rows into Q buffer item%2 (K-major, 128-byte
-        // swizzle), row limits and output rows into slot item%3.
-        auto setup = [&](int idx, int item) {
-            const RowItem it = row_item(p, idx, false);
-            const int r = tid >> 2;
-            int lim;
-            long long row;
-            row_of(p, it, r, lim, row);
-            if ((tid & 3) == 0) {
-                row_lim[(item % 3) * 32 + r] = lim;
-                row_out[(item % 3) * 32 + r] = row;
-            }
-            const uint4* src = reinterpret_cast<const uint4*>(p.q + (row < 0 ? 0 : row) * kD);
-            unsigned char* qb = smem + kQOff + (item & 1) * kQBytes;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int c16 = (tid & 3) * 4 + u;
-                const uint4 v = row >= 0 ? src[c16] : make_uint4(0, 0, 0, 0);
-                const int h = c16 >> 3, cc = c16 & 7;
-                *reinterpret_cast<uint4*>(qb + h * kQHalf + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
-            }
-            fence_proxy_async_smem();
-            mbar_arrive_plain(&q_ready[item & 1]);
-        };
-
-        // Live items of this CTA in order.  Every item of the CTA is scanned
-        // exactly once here, so this is where bad inputs are reported.
-        auto next_live = [&](int from) -> int {
-            for (int idx = from; idx < num_items; idx += gridDim.x)
-                if (row_item(p, idx, tid == 0).unit >= 0) return idx;
-            return -1;
-        };
-
         bool fail = false;  // a bounded wait of this thread gave up
         bool stop = false;  // all four warps agreed to stop
-        int cur = next_live(blockIdx.x);
-        int nxt = cur >= 0 ? next_live(cur + gridDim.x) : -1;
-        if (cur >= 0) setup(cur, 0);
-        if (nxt >= 0) setup(nxt, 1);
 
-        // Epilogue of item i: O^T (thread = d) / l into the output rows.
-        auto epilogue = [&](int i) {
-            const int slot = i % 3;
+        // Row sums of the item in slot sl from the four warps' partials.
+        auto finish_sums = [&](int sl) {
+            if (warp == 0) {
+                ItemSlot& S = slots[sl];
+                const float4 v = *reinterpret_cast<const float4*>(S.red_l[lane]);
+                const float l = (v.x + v.y) + (v.z + v.w);
+                S.l[lane] = l;
+                S.inv_l[lane] = l > 0.f ? 1.f / l : 0.f;
+            }
+        };
+        // Epilogue of item i (slot sl): O^T (thread = d) / l into the output rows.
+        auto epilogue = [&](int i, int sl) {
+            const ItemSlot& S = slots[sl];
             const int ob = i & 1;
-            bool okw = __all_sync(0xffffffffu, wait_bar(&o_full[ob], (i >> 1) & 1));
+            const bool okw = __all_sync(0xffffffffu, wait_bar(&o_full[ob], (i >> 1) & 1));
             if (!okw) {
                 fail = true;
                 return;
@@ -634,17 +713,19 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             mbar_arrive_plain(&o_empty[ob]);
 #pragma unroll
             for (int r = 0; r < 32; ++r) {
-                const long long row = row_out[slot * 32 + r];
+                const long long row = S.row[r];
                 if (row < 0) continue;
-                const float4 l4 = *reinterpret_cast<const float4*>(red_l + slot * 128 + r * 4);
-                const float l = (l4.x + l4.y) + (l4.z + l4.w);
-                const float acc = __uint_as_float(o[r]) + __uint_as_float(olo[r]);
-                p.out[row * kD + tid] = l > 0.f ? acc / l : 0.f;
-                if (p.shared_prefix_mode && tid == r) {
-                    p.out_m[row] = item_m[slot * 32 + r];
-                    p.out_l[row] = l;
+                p.out[row * kD + tid] =
+                    (__uint_as_float(o[r]) + __uint_as_float(olo[r])) * S.inv_l[r];
+            }
+            if (p.shared_prefix_mode && tid < 32) {
+                const long long row = S.row[tid];
+                if (row >= 0) {
+                    p.out_m[row] = S.m[tid];
+                    p.out_l[row] = S.l[tid];
                 }
             }
+            mbar_arrive_plain(&slot_free[sl]);
         };
 
         float m_ref[32], l_part[32];
@@ -654,25 +735,31 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             l_part[r] = 0.f;
         }
         int n = 0, item = 0;
-        bool pending_epi = false;
+        int prev = -1;  // slot of the item whose epilogue is pending
         // This token's 128-byte row of [P_hi^T | P_lo^T] (MN-major, 128-byte
         // swizzle: 16-byte chunk j of row t sits at chunk j ^ (t % 8)).
         const uint32_t p_row = (uint32_t)tid * 128;
         const uint32_t p_sw = (uint32_t)(tid & 7);
 
-        while (cur >= 0 && !stop) {
-            // This item's row data (written one item earlier) is visible, and
-            // every warp is done with the slot the next setup overwrites.
-            softmax_sync();
-            const RowItem it = row_item(p, cur, false);
-            const int slot = item % 3;
-            int min_lim = 0x7fffffff;
-#pragma unroll
-            for (int r = 0; r < 32; ++r)
-                if (row_out[slot * 32 + r] >= 0) min_lim = min(min_lim, row_lim[slot * 32 + r]);
+        for (;; ++item) {
+            const int sl = item % kSlots;
+            const bool okw = wait_bar(&item_ready[sl], (item / kSlots) & 1);
+            // One barrier per item: the four warps agree on stopping, and the
+            // previous item's partial sums are visible.
+            const bool bad = !okw || fail || (tid == 0 && aborted(abort_flag));
+            if (softmax_sync_count(bad) != 0) {
+                if (tid == 0) set_abort(abort_flag, p.error_flags);
+                stop = true;
+                break;
+            }
+            ItemSlot& S = slots[sl];
+            const int nch = S.nch;
+            if (nch < 0) break;
+            if (prev >= 0) finish_sums(prev);
+            const int min_lim = S.min_lim;
             const int ob = item & 1;
 
-            for (int c = 0; c < it.nch; ++c, ++n) {
+            for (int c = 0; c < nch; ++c, ++n) {
                 const int sb = n & 1;
                 bool ok = !fail && __all_sync(0xffffffffu, wait_bar(&s_full[sb], (n >> 1) & 1));
                 float x[32];
@@ -687,7 +774,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                     if (c * kTok + kTok - 1 > min_lim) {
 #pragma unroll
                         for (int r = 0; r < 32; ++r)
-                            if (tok > row_lim[slot * 32 + r]) x[r] = -INFINITY;
+                            if (tok > S.lim[r]) x[r] = -INFINITY;
                     }
                 } else {
 #pragma unroll
@@ -698,7 +785,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 for (int r = 0; r < 32; ++r) grow = grow || x[r] > m_ref[r] + kRescaleThreshold;
                 if (lane == 0 && aborted(abort_flag)) ok = false;
                 ok = __all_sync(0xffffffffu, ok);
-                bool slow = softmax_sync_count(grow || !ok) != 0;
+                const bool slow = softmax_sync_count(grow || !ok) != 0;
                 if (slow && softmax_sync_count(!ok) != 0) {
                     if (tid == 0) set_abort(abort_flag, p.error_flags);
                     stop = true;
@@ -725,9 +812,9 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                     }
                     if (resc && c > 0) {
                         // O^T must be stable: the previous PV has to be done.
-                        const bool okw = __all_sync(
+                        const bool okp = __all_sync(
                             0xffffffffu, wait_bar(&pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1));
-                        if (okw) {
+                        if (okp) {
                             tc_fence_after();
 #pragma unroll
                             for (int part = 0; part < 2; ++part) {
@@ -776,38 +863,36 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 tc_fence_before();
                 mbar_arrive_plain(&p_full[sb]);
 
-                if (c == 0) {
-                    if (pending_epi) epilogue(item - 1);
-                    pending_epi = false;
-                    if (item >= 1 && nxt >= 0) setup(nxt, item + 1);
+                if (c == 0 && prev >= 0) {
+                    epilogue(item - 1, prev);
+                    prev = -1;
                 }
             }
             if (stop) break;
-            // Item end: per-row sums over the 128 tokens' threads, the reference.
+            // Item end: per-row partial sums of this warp's 32 tokens, the reference.
             {
                 float v[32];
 #pragma unroll
                 for (int r = 0; r < 32; ++r) v[r] = l_part[r];
-                red_l[slot * 128 + lane * 4 + warp] = transpose_reduce<false>(v, lane);
+                S.red_l[lane][warp] = transpose_reduce<false>(v, lane);
                 float mine = 0.f;
 #pragma unroll
                 for (int r = 0; r < 32; ++r)
                     if (r == lane) mine = m_ref[r];
-                if (warp == 0) item_m[slot * 32 + lane] = mine;
+                if (warp == 0) S.m[lane] = mine;
 #pragma unroll
                 for (int r = 0; r < 32; ++r) {
                     m_ref[r] = kNoMax;
                     l_part[r] = 0.f;
                 }
             }
-            pending_epi = true;
-            cur = nxt;
-            nxt = cur >= 0 ? next_live(cur + gridDim.x) : -1;
-            ++item;
+            prev = sl;
         }
-        if (pending_epi && !stop) {
-            softmax_sync();  // the sums of the last item are in shared memory
-            epilogue(item - 1);
+        if (prev >= 0 && !stop) {
+            softmax_sync();  // the last item's partial sums
+            finish_sums(prev);
+            softmax_sync();
+            epilogue(item - 1, prev);
         }
         if (fail && tid == 0) set_abort(abort_flag, p.error_flags);
     }
