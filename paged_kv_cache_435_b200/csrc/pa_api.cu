@@ -83,9 +83,9 @@ size_t workspace_bytes_for(int num_seqs, int num_heads, int head_size,
 }
 
 // Shared-prefix call: the decode split's scratch, then the group pass's
-// partial results (O/l, max, sum per row).
+// partial results (O/l, max, sum per row) and each sequence's shared length.
 struct PrefixLayout {
-    size_t split_bytes, o_off, m_off, l_off, total;
+    size_t split_bytes, o_off, m_off, l_off, sh_off, total;
 };
 
 PrefixLayout prefix_layout(int num_seqs, int num_heads, int head_size,
@@ -97,7 +97,8 @@ PrefixLayout prefix_layout(int num_seqs, int num_heads, int head_size,
     L.o_off = L.split_bytes;
     L.m_off = L.o_off + ((rows * head_size * 4 + 255) & ~(size_t)255);
     L.l_off = L.m_off + ((rows * 4 + 255) & ~(size_t)255);
-    L.total = L.l_off + ((rows * 4 + 255) & ~(size_t)255);
+    L.sh_off = L.l_off + ((rows * 4 + 255) & ~(size_t)255);
+    L.total = L.sh_off + (((size_t)num_seqs * 4 + 255) & ~(size_t)255);
     return L;
 }
 
@@ -433,6 +434,7 @@ int pa_decode_attention_shared_prefix(
         r.block_tables = block_tables;
         r.context_lens = context_lens;
         r.groups = groups;
+        r.seq_shared = reinterpret_cast<int32_t*>(ws + lay.sh_off);
         r.error_flags = error_flags;
         r.shared_prefix_mode = 1;
         r.num_seqs = num_seqs;
@@ -479,10 +481,10 @@ int pa_decode_attention_shared_prefix(
     p.scale_log2 = pa::log2e_scale(scale);
     p.block_size = block_size;
     p.cascade = num_groups > 0 ? 1 : 0;
-    p.groups = groups;
     p.pref_o = reinterpret_cast<const float*>(ws + lay.o_off);
     p.pref_m = reinterpret_cast<const float*>(ws + lay.m_off);
     p.pref_l = reinterpret_cast<const float*>(ws + lay.l_off);
+    p.seq_shared = reinterpret_cast<const int32_t*>(ws + lay.sh_off);
     cudaError_t e = pa::launch_paged_decode(p, head_size, block_size, st);
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

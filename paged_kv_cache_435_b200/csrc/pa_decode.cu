@@ -101,21 +101,23 @@ __device__ __forceinline__ int parts_of(int L, int P) {
 }
 
 // First token of sequence s this kernel attends (0 unless a shared-prefix
-// group pass covers the tokens before it).
+// group pass covered the tokens before it; that pass wrote the length).
 template <bool kCascade, int BS>
 __device__ __forceinline__ int first_token(const DecodeParams& p, int s, int L) {
-    return kCascade ? cascade_shared_len(p.groups, s, L, p.num_seqs, BS) : 0;
+    return kCascade ? min(p.seq_shared[s], L) : 0;
 }
 
-// Item k of this CTA (k = 0, 1, ...).
-template <bool kPersist, bool kCascade, int BS>
+// Item k (k = 0, 1, ...) of this CTA, or of this warp when warps take
+// items of their own (kWarp: short items, no merge across warps).
+template <bool kPersist, bool kCascade, bool kWarp, int BS>
 __device__ __forceinline__ Item get_item(const DecodeParams& p,
-                                         const int* prefix, int k) {
+                                         const int* prefix, int k, int warp) {
     Item it;
     it.s = -1;
     int s, part;
     if (kPersist) {
-        const int j = blockIdx.y + k * gridDim.y;
+        const int j = kWarp ? (int)(blockIdx.y * kWarps + warp) + k * (int)(gridDim.y * kWarps)
+                            : (int)blockIdx.y + k * (int)gridDim.y;
         if (j >= prefix[p.num_seqs]) return it;
         int lo = 0, hi = p.num_seqs - 1;  // largest s with prefix[s] <= j
         while (lo < hi) {
@@ -143,11 +145,20 @@ __device__ __forceinline__ Item get_item(const DecodeParams& p,
     return it;
 }
 
-// Chunks of `it` that warp w owns.
+// Chunks of `it` that warp w owns: w, w+4, ... of the item, or all of them
+// when the warp owns the item.
+template <bool kWarp>
 __device__ __forceinline__ int warp_chunks(const Item& it, int warp) {
     if (it.s < 0) return 0;
     const int n = (it.tok1 - it.tok0 + kChunk - 1) / kChunk;
+    if (kWarp) return n;
     return n > warp ? (n - warp + kWarps - 1) / kWarps : 0;
+}
+
+// Chunk index within the item of the warp's i-th chunk.
+template <bool kWarp>
+__device__ __forceinline__ int chunk_of(int warp, int i) {
+    return kWarp ? i : warp + kWarps * i;
 }
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map,
@@ -168,7 +179,7 @@ __device__ __forceinline__ void named_bar_arrive(int id) {
     asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(kThreads) : "memory");
 }
 
-template <int D, int BS, bool kPersist, bool kCascade>
+template <int D, int BS, bool kPersist, bool kCascade, bool kWarp>
 __global__ void __launch_bounds__(kThreads, kTargetCtasPerSM)
 paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
@@ -254,20 +265,20 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
     // Lane l finds the (ids_base + l)-th chunk of the stream and its slot.
     auto refill = [&]() {
         int k = prod_k, i = prod_i, n = lane;
-        Item it = get_item<kPersist, kCascade, BS>(p, prefix, k);
+        Item it = get_item<kPersist, kCascade, kWarp, BS>(p, prefix, k, warp);
         for (;;) {
             if (it.s < 0) break;
-            const int rem = warp_chunks(it, warp) - i;
+            const int rem = warp_chunks<kWarp>(it, warp) - i;
             if (rem > n) break;
             n -= rem > 0 ? rem : 0;
             ++k;
             i = 0;
-            it = get_item<kPersist, kCascade, BS>(p, prefix, k);
+            it = get_item<kPersist, kCascade, kWarp, BS>(p, prefix, k, warp);
         }
         int slot = -1;
         if (it.s >= 0) {
             i += n;
-            const int ctok = it.tok0 + (warp + kWarps * i) * kChunk;
+            const int ctok = it.tok0 + chunk_of<kWarp>(warp, i) * kChunk;
             int id = tables[(int64_t)it.s * p.max_blocks_per_seq + ctok / BS];
             if (id < 0 || id >= p.num_blocks) {
                 report(p.error_flags, PA_DEVERR_BLOCK_ID);
@@ -329,20 +340,20 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
             dst[ks][1] = live ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8 + qc) : 0u;
         }
     };
-    Item next_it = get_item<kPersist, kCascade, BS>(p, prefix, 0);
+    Item next_it = get_item<kPersist, kCascade, kWarp, BS>(p, prefix, 0, warp);
     uint32_t qnext[D / 16][2];
     load_q(next_it, qnext);
     for (;; ++k) {
         const Item it = next_it;
         if (it.s < 0) break;
-        const int my_n = warp_chunks(it, warp);
+        const int my_n = warp_chunks<kWarp>(it, warp);
         uint32_t qa[D / 16][2];
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
             qa[ks][0] = qnext[ks][0];
             qa[ks][1] = qnext[ks][1];
         }
-        next_it = get_item<kPersist, kCascade, BS>(p, prefix, k + 1);
+        next_it = get_item<kPersist, kCascade, kWarp, BS>(p, prefix, k + 1, warp);
         load_q(next_it, qnext);
 
         float o[D / 8][4];
@@ -365,7 +376,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
             ++cons_count;
             if (aborted) continue;
 
-            const int ctok = it.tok0 + (warp + kWarps * i) * kChunk;
+            const int ctok = it.tok0 + chunk_of<kWarp>(warp, i) * kChunk;
             const int valid = min(kChunk, it.tok1 - ctok);
             const uint32_t kaddr = smem_u32(my_ring + stage * C::kStageBytes);
             const uint32_t vaddr = kaddr + C::kKVBytes;
@@ -465,7 +476,42 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         // ---------------- item end: merge the four warps ----------------
         l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
         l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
-        if (warp != 0) {
+        if (kWarp) {
+            // The warp holds the whole item: row qr is o[.][0..1] (P_hi V)
+            // plus o[.][2..3] (P_lo V), with max m_run and sum l_run.
+            if (qr < G) {
+                const int h = g * G + qr;
+                const bool direct = it.nparts == 1;
+                const int64_t row = (int64_t)it.s * Hq + h;
+                const int64_t idx = row * p.max_partitions + it.part;
+                float* dst = direct ? p.out + row * D : p.tmp_o + idx * D;
+                float den = l_run, wa = 1.f, wb = 0.f;
+                const float* po = nullptr;
+                if (kCascade && direct && it.sh > 0) {
+                    const float mp = p.pref_m[row], lp = p.pref_l[row];
+                    const float Mt = fmaxf(m_run, mp);
+                    wa = m_run == -INFINITY ? 0.f : exp2f(m_run - Mt);
+                    wb = lp * exp2f(mp - Mt);
+                    den = den * wa + wb;
+                    po = p.pref_o + row * D;
+                }
+#pragma unroll
+                for (int j = 0; j < D / 8; ++j) {
+                    float v[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        float acc = o[j][e] + o[j][e + 2];
+                        if (kCascade && po != nullptr) acc = acc * wa + wb * po[8 * j + qc + e];
+                        v[e] = it.L > 0 ? acc / den : 0.f;
+                    }
+                    *reinterpret_cast<float2*>(dst + 8 * j + qc) = make_float2(v[0], v[1]);
+                }
+                if (!direct && (lane & 3) == 0) {
+                    p.tmp_m[idx] = m_run;
+                    p.tmp_l[idx] = den;
+                }
+            }
+        } else if (warp != 0) {
             if (k > 0) named_bar_sync(2);  // warp 0 has read the previous item
             float* dst = red_o + ((warp - 1) * kMaxGroup + qr) * C::kRedStride + qc;
 #pragma unroll
@@ -531,7 +577,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         }
     }
     // Consume warp 0's last "merged" arrival so no barrier is left pending.
-    if (warp != 0 && k > 0) named_bar_sync(2);
+    if (!kWarp && warp != 0 && k > 0) named_bar_sync(2);
 
     if (aborted) {
         // Drain copies still in flight on this warp's ring (bounded) before
@@ -559,7 +605,7 @@ paged_decode_reduce_kernel(const DecodeParams p) {
     pdl_wait();  // the partials come from the grid launched just before
     int L = p.context_lens[s];
     L = L < 0 ? 0 : (L > p.max_context_len ? p.max_context_len : L);
-    const int sh = p.cascade ? cascade_shared_len(p.groups, s, L, p.num_seqs, p.block_size) : 0;
+    const int sh = p.cascade ? min(p.seq_shared[s], L) : 0;
     const int np = (L - sh + p.partition_size - 1) / p.partition_size;
     if (np <= 1) return;  // written directly by the partition kernel
     const int64_t base = ((int64_t)s * p.num_heads + h) * p.max_partitions;
@@ -714,25 +760,32 @@ cudaError_t launch_partition_kernel(const DecodeParams& p, const CUtensorMap& tm
     using C = Cfg<D>;
     static int grid_ready[64] = {0};
     static int persist_ready[64] = {0};
-    const bool persist = p.max_partitions > 1 && p.num_seqs <= kMaxPersistSeqs;
+    // Persistent CTAs when sequences are split; for the short private tails
+    // of a shared-prefix call, persistent warps that each own whole items
+    // (the copies of the next item stay in flight across item boundaries
+    // and no warp waits for another's merge).
+    const bool persist = (p.max_partitions > 1 || kCascade) && p.num_seqs <= kMaxPersistSeqs;
     cudaError_t e;
     if (persist) {
-        e = set_smem(paged_decode_kernel<D, BS, true, kCascade>, C::kSmemPersist,
+        constexpr bool kWarp = kCascade;
+        e = set_smem(paged_decode_kernel<D, BS, true, kCascade, kWarp>, C::kSmemPersist,
                      persist_ready);
         if (e != cudaSuccess) return e;
         long long per_head = (kTargetCtasPerSM * kNumSMs + p.num_kv_heads - 1) / p.num_kv_heads;
         const long long items = (long long)p.num_seqs * p.max_partitions;
-        if (per_head > items) per_head = items;
+        const long long streams = kWarp ? (items + kWarps - 1) / kWarps : items;
+        if (per_head > streams) per_head = streams;
         if (per_head < 1) per_head = 1;
         dim3 grid((unsigned)p.num_kv_heads, (unsigned)per_head, 1);
-        e = launch_pdl(paged_decode_kernel<D, BS, true, kCascade>, grid, dim3(kThreads),
+        e = launch_pdl(paged_decode_kernel<D, BS, true, kCascade, kWarp>, grid, dim3(kThreads),
                        C::kSmemPersist, stream, tmk, tmv, p);
     } else {
-        e = set_smem(paged_decode_kernel<D, BS, false, kCascade>, C::kSmemGrid, grid_ready);
+        e = set_smem(paged_decode_kernel<D, BS, false, kCascade, false>, C::kSmemGrid,
+                     grid_ready);
         if (e != cudaSuccess) return e;
         dim3 grid((unsigned)p.num_kv_heads, (unsigned)p.max_partitions,
                   (unsigned)p.num_seqs);
-        e = launch_pdl(paged_decode_kernel<D, BS, false, kCascade>, grid, dim3(kThreads),
+        e = launch_pdl(paged_decode_kernel<D, BS, false, kCascade, false>, grid, dim3(kThreads),
                        C::kSmemGrid, stream, tmk, tmv, p);
     }
     count_launch();

@@ -4,8 +4,6 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
-#include "pa_cascade.cuh"
-
 namespace pa {
 
 struct DecodeParams {
@@ -34,10 +32,10 @@ struct DecodeParams {
     // group pass covered the tokens before it) and its result is merged
     // with the group pass's partial (pref_o = O/l, pref_m, pref_l per row).
     int cascade;
-    CascadeGroups groups;
     const float* pref_o;         // fp32 [B][Hq][D]
     const float* pref_m;         // fp32 [B][Hq] (log2 domain)
     const float* pref_l;         // fp32 [B][Hq]
+    const int32_t* seq_shared;   // int32 [B]: tokens the group pass covered
 };
 
 // scale * log2(e): logits are kept in the log2 domain (exp2f).

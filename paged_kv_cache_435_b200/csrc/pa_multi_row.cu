@@ -438,6 +438,13 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
 
     if (warp == 7) {
         // -------------------------------------------------------- scheduler
+        if (p.shared_prefix_mode) {
+            // Each sequence's shared length, for the per-sequence pass: the
+            // CTAs split the batch.
+            for (int s = blockIdx.x * 32 + lane; s < p.num_seqs; s += gridDim.x * 32)
+                p.seq_shared[s] = cascade_shared_len(p.groups, s, clamp_len(p, s, false),
+                                                     p.num_seqs, p.block_size);
+        }
         int live = 0;
         for (int idx = blockIdx.x;; idx += gridDim.x) {
             const bool end = idx >= num_items;

@@ -25,6 +25,8 @@ struct MultiRowParams {
     const int32_t* context_lens;     // int32 [B]
     const int32_t* query_start_loc;  // int32 [B+1] (multi-query mode)
     CascadeGroups groups;            // shared-prefix mode
+    int32_t* seq_shared;             // shared-prefix mode: int32 [B], each
+                                     // sequence's shared length (written)
     int* error_flags;                // nullable
     int shared_prefix_mode;
     int num_seqs;
