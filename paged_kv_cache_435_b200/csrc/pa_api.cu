@@ -310,11 +310,14 @@ int pa_multi_query_attention(float* out, const void* q, const void* k_cache,
     p.num_blocks = num_blocks;
     p.group = G;
     p.scale_log2 = pa::mq_log2e_scale(scale);
-    // Kernel choice: the tcgen05 kernel for 128-row tiles (prefill chunks),
-    // the mma.sync kernel for few rows per sequence (speculative verify).
-    // PA_MULTI_QUERY_KERNEL=mma|tc overrides the choice (tests, benchmarks).
+    // Kernel choice (head_size 128): the 128-row tcgen05 kernel for prefill
+    // chunks (>= 128 rows per sequence), the 32-row tcgen05 kernel (tokens as
+    // the MMA's M) below that; head_size 64 runs on the mma.sync kernel.
+    // PA_MULTI_QUERY_KERNEL=mma|tc|rows overrides the choice (tests,
+    // benchmarks).
     enum { kMma, kTc, kRows } kind = kMma;
     if (pa::multi_query_tc_eligible(head_size, max_query_len, G)) kind = kTc;
+    else if (head_size == 128) kind = kRows;
     if (const char* force = std::getenv("PA_MULTI_QUERY_KERNEL")) {
         if (std::strcmp(force, "mma") == 0) kind = kMma;
         if (std::strcmp(force, "tc") == 0 && head_size == 128) kind = kTc;

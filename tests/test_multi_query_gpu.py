@@ -149,3 +149,13 @@ def test_multi_row_kernel_spec_verify_batch256(monkeypatch):
 def test_multi_row_kernel_determinism(monkeypatch):
     monkeypatch.setenv("PA_MULTI_QUERY_KERNEL", "rows")
     test_run_to_run_determinism()
+
+
+@pytest.mark.parametrize("Hq,Hkv,D,bs,lens,qlens", ROWS_SHAPES[:3])
+def test_mma_kernel_head128_shapes(monkeypatch, Hq, Hkv, D, bs, lens, qlens):
+    """The mma.sync kernel, forced at head_size 128 (the default there is the
+    tcgen05 kernel), stays exact."""
+    monkeypatch.setenv("PA_MULTI_QUERY_KERNEL", "mma")
+    case = inputs.multi_query_case(len(lens), Hq, Hkv, D, bs, lens, qlens,
+                                   seed=sum(lens) + Hq + 2, device="cuda")
+    check(case)
