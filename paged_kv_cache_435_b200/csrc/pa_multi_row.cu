@@ -32,11 +32,19 @@
 //   warp 4     K producer, warp 5 V producer: 16-token TMA tensor tiles
 //              (128-byte swizzle) of each 128-token chunk into 2- and 3-stage
 //              rings (V waits for the softmax, so it runs deeper);
-//   warp 6     TMEM allocation and the MMA issue (one thread);
-//   warp 7     scheduler: works out the CTA's next items (token range, block
-//              table row, each row's limit and output row) into a 4-slot
-//              shared-memory ring and copies their Q rows (cp.async), so no
-//              other warp waits on a global load at an item boundary.
+//   warp 6     TMEM allocation and the MMA issue (one thread), S two chunks
+//              ahead of PV: S(n) needs only that the softmax has loaded
+//              S(n-2) out of its TMEM buffer, PV(n-2) that it wrote P(n-2);
+//   warp 7     scheduler: deals the items to the CTAs by work (a CTA serves
+//              one kv head; among the CTAs of a head, each takes the items
+//              whose cumulative weight starts in its share, computed
+//              identically everywhere; the heads move through the batch in
+//              step, so the head slices of a block are read together), works
+//              out its next
+//              items (token range, block-table row, each row's limit and
+//              output row) into a 4-slot shared-memory ring and copies their
+//              Q rows (cp.async), so no other warp waits on a global load at
+//              an item boundary.
 // Online softmax with a lazy reference: every chunk, one barrier-reduction
 // over the 4 warps (bar.red.popc) asks whether any row's logit exceeds its
 // reference max by more than 2^8; only then is the exact per-row chunk max
@@ -94,10 +102,10 @@ static_assert(sizeof(ItemSlot) == 1312, "slot layout");
 
 constexpr int kSlotOff = kCmaxOff + 512;
 constexpr int kBarOff = kSlotOff + kSlots * (int)sizeof(ItemSlot);
-// barriers: k_full[KS] k_empty[KS] v_full[VS] v_empty[VS] s_full[2] p_full[2]
-//           pv_done[2] o_full[2] o_empty[2] q_empty[2] item_ready[4]
+// barriers: k_full[KS] k_empty[KS] v_full[VS] v_empty[VS] s_full[2] s_free[2]
+//           p_full[2] pv_done[2] o_full[2] o_empty[2] q_empty[2] item_ready[4]
 //           slot_free[4] drain
-constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 13 + 2 * kSlots;
+constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 15 + 2 * kSlots;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16;
 constexpr uint32_t kTmemCols = 256;       // S0 | S1 | O0 (hi, lo) | O1 (hi, lo)
 constexpr uint32_t kTmemO = 64;           // first O column
@@ -329,6 +337,27 @@ __device__ RowItem row_item(const MultiRowParams& p, int idx, bool report_errors
     return it;
 }
 
+// Work of unit u (sequence or group) for the item deal: its live row tiles
+// and the weight of each of its items (128-token chunks, plus one for the
+// per-item overhead).  Invalid groups have no tiles.
+__device__ void unit_work(const MultiRowParams& p, int u, bool report_errors, int& tiles,
+                          int& w) {
+    if (!p.shared_prefix_mode) {
+        const int L = clamp_len(p, u, report_errors);
+        const int k = clamp_queries(p, u, L, report_errors);
+        tiles = (k * p.group + kN - 1) / kN;
+        w = (L + kTok - 1) / kTok + 1;
+    } else {
+        const int P = cascade_group_prefix(p.groups, u, p.num_seqs, p.block_size,
+                                           p.error_flags, report_errors);
+        const int members = p.groups.group_start[u + 1] - p.groups.group_start[u];
+        const int mpt = kN / p.group;
+        tiles = P > 0 ? (members + mpt - 1) / mpt : 0;
+        w = (P + kTok - 1) / kTok + 1;
+    }
+    tiles = min(tiles, p.tiles);
+}
+
 // Row r of a live item: last visible token (lim) and the q / out row index
 // (-1 for a row that does not exist).
 __device__ void row_of(const MultiRowParams& p, const RowItem& it, int r, int& lim,
@@ -363,7 +392,7 @@ template <int BS>
 __global__ void __launch_bounds__(kThreads, 1)
 paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v,
-                       const MultiRowParams p, int num_items) {
+                       const MultiRowParams p) {
     extern __shared__ __align__(1024) unsigned char smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
     uint64_t* k_full = bars;
@@ -371,7 +400,8 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
     uint64_t* v_full = k_empty + kKStages;
     uint64_t* v_empty = v_full + kVStages;
     uint64_t* s_full = v_empty + kVStages;
-    uint64_t* p_full = s_full + 2;
+    uint64_t* s_free = s_full + 2;
+    uint64_t* p_full = s_free + 2;
     uint64_t* pv_done = p_full + 2;
     uint64_t* o_full = pv_done + 2;
     uint64_t* o_empty = o_full + 2;
@@ -405,6 +435,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
+            mbar_init(&s_free[i], 128);
             mbar_init(&p_full[i], 128);
             mbar_init(&pv_done[i], 1);
             mbar_init(&o_full[i], 1);
@@ -446,13 +477,14 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                      p.num_seqs, p.block_size);
         }
         int live = 0;
-        for (int idx = blockIdx.x;; idx += gridDim.x) {
-            const bool end = idx >= num_items;
+        // Publish item idx (idx < 0: the end marker); false on abort.
+        auto publish = [&](int idx) -> bool {
+            const bool end = idx < 0;
             RowItem it;
             it.unit = -1;
             if (!end) {
-                it = row_item(p, idx, lane == 0);
-                if (it.unit < 0) continue;
+                it = row_item(p, idx, false);
+                if (it.unit < 0) return true;
             }
             const int s = live % kSlots;
             bool good = true;
@@ -464,13 +496,13 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 good = wait_bar(&q_empty[live & 1], ((live - 2) >> 1) & 1);
             if (__shfl_sync(0xffffffffu, good ? 1 : 0, 0) == 0) {
                 if (lane == 0) set_abort(abort_flag, p.error_flags);
-                break;
+                return false;
             }
             ItemSlot& S = slots[s];
             if (end) {
                 if (lane == 0) S.nch = -1;
                 mbar_arrive_plain(&item_ready[s]);
-                break;
+                return true;
             }
             int lim;
             long long row;
@@ -501,7 +533,62 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             fence_proxy_async_smem();
             mbar_arrive_plain(&item_ready[s]);
             ++live;
+            return true;
+        };
+
+        // Deal by work.  CTA b serves kv head g = b % Hkv as the j-th of the
+        // head's per_head CTAs.  The head's items are ordered (unit, tile);
+        // tile t of unit u starts at position start(u) + t * w(u) of the
+        // head's total T and belongs to the CTA whose share
+        // [T*j/per_head, T*(j+1)/per_head) holds that start, so every item
+        // has exactly one CTA.
+        const int Hkv = p.num_kv_heads;
+        const int g = blockIdx.x % Hkv;
+        const int j = blockIdx.x / Hkv;
+        const int per_head = gridDim.x / Hkv;
+        long long T = 0;
+        for (int base = 0; base < p.num_units; base += 32) {
+            const int u = base + lane;
+            int tl = 0, w = 0;
+            if (u < p.num_units) unit_work(p, u, blockIdx.x == 0, tl, w);
+            long long W = (long long)tl * w;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
+            T += W;
         }
+        const long long lo = T * j / per_head;
+        const long long hi = T * (j + 1) / per_head;
+        bool stopped = false;
+        long long pos = 0;  // start of the current batch of units
+        for (int base = 0; base < p.num_units && pos < hi && !stopped; base += 32) {
+            const int u = base + lane;
+            int tl = 0, w = 0;
+            if (u < p.num_units) unit_work(p, u, false, tl, w);
+            const long long W = (long long)tl * w;
+            long long incl = W;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const long long t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            const long long total = __shfl_sync(0xffffffffu, incl, 31);
+            if (pos + total > lo) {
+                for (int i = 0; i < 32 && base + i < p.num_units && !stopped; ++i) {
+                    const long long us = pos + __shfl_sync(0xffffffffu, incl - W, i);
+                    const int ti = __shfl_sync(0xffffffffu, tl, i);
+                    const int wi = __shfl_sync(0xffffffffu, w, i);
+                    if (us >= hi) break;
+                    if (us + (long long)ti * wi <= lo) continue;
+                    for (int t = 0; t < ti && !stopped; ++t) {
+                        const long long q = us + (long long)t * wi;
+                        if (q < lo || q >= hi) continue;
+                        if (!publish(((base + i) * p.tiles + t) * Hkv + g)) stopped = true;
+                    }
+                }
+            }
+            pos += total;
+        }
+        if (!stopped) (void)publish(-1);
     } else if (warp == 4 || warp == 5) {
         // ------------------------------------------------ K / V producers
         const bool is_v = warp == 5;
@@ -578,13 +665,18 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             int n, valid, item;
             bool first, last;
         };
-        Pending pend = {0, 0, 0, false, false};
-        bool have_pend = false;
+        Pending pend0 = {0, 0, 0, false, false};  // PVs still to issue:
+        Pending pend1 = pend0;                    // pend0 is the older
+        int npend = 0;
         bool ok = true;
 
         auto issue_pv = [&](const Pending& pd) -> bool {
             const int vs = pd.n % kVStages;
-            bool good = __all_sync(0xffffffffu, wait_bar(&v_full[vs], (pd.n / kVStages) & 1));
+            const bool zero_tail = pd.valid % 16 != 0;
+            // Lanes that write into the V stage (tail rows) observe it landing.
+            bool good = true;
+            if (lane == 0 || zero_tail) good = wait_bar(&v_full[vs], (pd.n / kVStages) & 1);
+            good = __all_sync(0xffffffffu, good);
             if (good && lane == 0) good = wait_bar(&p_full[pd.n & 1], (pd.n >> 1) & 1);
             if (good && lane == 0 && pd.first && pd.item >= 2)
                 good = wait_bar(&o_empty[pd.item & 1], ((pd.item - 2) >> 1) & 1);
@@ -593,7 +685,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 if (lane == 0) set_abort(abort_flag, p.error_flags);
                 return false;
             }
-            if (pd.valid % 16 != 0) {
+            if (zero_tail) {
                 // The last loaded 16-token piece ends past the range: its
                 // extra token rows hold whatever the block holds.
                 unsigned char* vt = smem + kVOff + vs * kStageBytes;
@@ -644,7 +736,11 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             const uint32_t q_base = smem_u32(smem + kQOff + (item & 1) * kQBytes);
             for (int c = 0; c < nch; ++c, ++n) {
                 bool good = true;
-                if (lane == 0) good = wait_bar(&k_full[n % kKStages], (n / kKStages) & 1);
+                if (lane == 0) {
+                    good = wait_bar(&k_full[n % kKStages], (n / kKStages) & 1);
+                    // S buffer n%2 held S(n-2): the softmax has loaded it.
+                    if (good && n >= 2) good = wait_bar(&s_free[n & 1], ((n - 2) >> 1) & 1);
+                }
                 good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
                 if (!good || aborted(abort_flag)) {
                     if (lane == 0) set_abort(abort_flag, p.error_flags);
@@ -666,19 +762,26 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                     if (c == nch - 1) mma_commit(&q_empty[item & 1]);
                 }
                 __syncwarp();
-                if (have_pend && !issue_pv(pend)) {
-                    ok = false;
-                    break;
+                if (npend == 2) {
+                    if (!issue_pv(pend0)) {
+                        ok = false;
+                        break;
+                    }
+                    pend0 = pend1;
+                    npend = 1;
                 }
-                pend.n = n;
-                pend.valid = min(kTok, range_end - c * kTok);
-                pend.item = item;
-                pend.first = c == 0;
-                pend.last = c == nch - 1;
-                have_pend = true;
+                Pending pn;
+                pn.n = n;
+                pn.valid = min(kTok, range_end - c * kTok);
+                pn.item = item;
+                pn.first = c == 0;
+                pn.last = c == nch - 1;
+                if (npend == 0) pend0 = pn; else pend1 = pn;
+                ++npend;
             }
         }
-        if (ok && have_pend) (void)issue_pv(pend);
+        if (ok && npend >= 1) ok = issue_pv(pend0);
+        if (ok && npend == 2) ok = issue_pv(pend1);
         if (lane == 0) {
             mma_commit(drain);               // everything issued so far
             (void)wait_bar(drain, 0);        // drained before TMEM goes away
@@ -775,6 +878,8 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                     uint32_t raw[32];
                     tmem_ld32(tmem + sb * 32 + lane_off, raw);
                     tmem_wait_ld();
+                    tc_fence_before();
+                    mbar_arrive_plain(&s_free[sb]);  // S(n+2) may overwrite the buffer
 #pragma unroll
                     for (int r = 0; r < 32; ++r) x[r] = __uint_as_float(raw[r]) * sl2;
                     const int tok = c * kTok + tid;
@@ -984,9 +1089,16 @@ cudaError_t mr_launch_typed(const MultiRowParams& p, cudaStream_t stream) {
     const long long items = (long long)p.num_units * p.tiles * p.num_kv_heads;
     if (items <= 0) return cudaSuccess;
     if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
-    const int grid = (int)(items < num_sms() ? items : num_sms());
+    // One kv head per CTA, the same number of CTAs for every head (at least
+    // one per head, at most one per item).
+    long long per_head = num_sms() / p.num_kv_heads;
+    const long long head_items = (long long)p.num_units * p.tiles;
+    if (per_head > head_items) per_head = head_items;
+    if (per_head < 1) per_head = 1;
+    const long long grid = per_head * p.num_kv_heads;
+    if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid);
+    cfg.gridDim = dim3((unsigned)grid);  // gridDim.x % num_kv_heads == 0
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = stream;
@@ -995,7 +1107,7 @@ cudaError_t mr_launch_typed(const MultiRowParams& p, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, paged_multi_row_kernel<BS>, tmk, tmv, p, (int)items);
+    e = cudaLaunchKernelEx(&cfg, paged_multi_row_kernel<BS>, tmk, tmv, p);
     count_launch();
     return e;
 }
