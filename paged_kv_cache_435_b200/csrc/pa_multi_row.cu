@@ -805,7 +805,8 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 S.inv_l[lane] = l > 0.f ? 1.f / l : 0.f;
             }
         };
-        // Epilogue of item i (slot sl): O^T (thread = d) / l into the output rows.
+        // Epilogue of item i (slot sl): O^T (thread = d) / l into the output rows
+        // (one 4-byte store per row and thread; rows of one warp coalesce).
         auto epilogue = [&](int i, int sl) {
             const ItemSlot& S = slots[sl];
             const int ob = i & 1;
@@ -822,11 +823,17 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             tc_fence_before();
             mbar_arrive_plain(&o_empty[ob]);
 #pragma unroll
-            for (int r = 0; r < 32; ++r) {
-                const long long row = S.row[r];
-                if (row < 0) continue;
-                p.out[row * kD + tid] =
-                    (__uint_as_float(o[r]) + __uint_as_float(olo[r])) * S.inv_l[r];
+            for (int r = 0; r < 32; r += 4) {
+                const float4 iv = *reinterpret_cast<const float4*>(&S.inv_l[r]);
+                const longlong2 ra = *reinterpret_cast<const longlong2*>(&S.row[r]);
+                const longlong2 rb = *reinterpret_cast<const longlong2*>(&S.row[r + 2]);
+                const float inv[4] = {iv.x, iv.y, iv.z, iv.w};
+                const long long row[4] = {ra.x, ra.y, rb.x, rb.y};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (row[e] >= 0)
+                        p.out[row[e] * kD + tid] =
+                            (__uint_as_float(o[r + e]) + __uint_as_float(olo[r + e])) * inv[e];
             }
             if (p.shared_prefix_mode && tid < 32) {
                 const long long row = S.row[tid];
@@ -975,7 +982,9 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 tc_fence_before();
                 mbar_arrive_plain(&p_full[sb]);
 
-                if (c == 0 && prev >= 0) {
+                // The previous item's epilogue, one chunk into this item when
+                // there is one: its last PV is then done, not just issued.
+                if (prev >= 0 && c == min(1, nch - 1)) {
                     epilogue(item - 1, prev);
                     prev = -1;
                 }

@@ -189,3 +189,33 @@ def test_multi_query_host_validation(lib):
     assert call(a13=96) == nat.PA_ERR_UNSUPPORTED
     assert call(a8=None) == nat.PA_ERR_INVALID_ARG
     assert call(a9=0) == nat.PA_OK
+
+
+def test_shared_prefix_host_validation(lib):
+    f = lib.pa_decode_attention_shared_prefix
+    #       out   q     k     v     bt   mb cl   maxlen gs    pl   G mgs B   Hq Hkv D   bs  NB  scale part ws    wsb       err   stream
+    base = [FAKE, FAKE, FAKE, FAKE, FAKE, 8, FAKE, 100, FAKE, FAKE, 2, 4, 8, 32, 8, 128, 16, 64, 0.1, 0, FAKE, 1 << 30, None, None]
+
+    def call(**kw):
+        a = list(base)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return f(*a)
+    assert call(a10=-1) == nat.PA_ERR_INVALID_ARG          # negative group count
+    assert call(a11=0) == nat.PA_ERR_INVALID_ARG           # max_group_size 0
+    assert call(a8=None) == nat.PA_ERR_INVALID_ARG         # group_start missing
+    assert call(a9=FAKE + 2) == nat.PA_ERR_INVALID_ARG     # prefix_lens misaligned
+    assert call(a15=64) == nat.PA_ERR_UNSUPPORTED          # head size 64
+    assert call(a13=128) == nat.PA_ERR_UNSUPPORTED         # 128 q / 8 kv: group 16
+    assert call(a20=None) == nat.PA_ERR_WORKSPACE          # no workspace
+    assert call(a21=16) == nat.PA_ERR_WORKSPACE            # too small
+    assert call(a20=FAKE + 16) == nat.PA_ERR_INVALID_ARG   # workspace not 256-aligned
+    assert call(a12=0, a0=None, a1=None) == nat.PA_OK      # empty batch
+
+
+def test_shared_prefix_workspace_grows_with_rows(lib):
+    a = nat.pa_shared_prefix_workspace_size(8, 32, 8, 128, 16, 1000)
+    b = nat.pa_shared_prefix_workspace_size(16, 32, 8, 128, 16, 1000)
+    assert b > a > nat.pa_decode_workspace_size(8, 32, 8, 128, 16, 1000)
+    # the group pass's partials: O/l, max and sum per (sequence, head)
+    assert a >= 8 * 32 * (128 + 2) * 4
