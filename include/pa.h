@@ -389,6 +389,22 @@ int pa_bm_swap_out(pa_block_manager* m, int seq_id, int64_t* pairs,
 int pa_bm_swap_in(pa_block_manager* m, int seq_id, int64_t* pairs,
                   int capacity);
 
+/* Shared-prefix groups of a batch, for pa_decode_attention_shared_prefix
+ * ("Memory Sharing via Copy-on-Write (CoW)": parallel samples and beams share
+ * the prompt's blocks until they diverge).  seq_ids (host int32
+ * [num_seqs]) is the batch in launch order; runs of consecutive sequences
+ * whose block tables agree on at least min_shared_blocks (>= 1) leading
+ * blocks form a group, whose prefix is the blocks all its members share
+ * (times block_size tokens); a sequence sharing nothing is a group of one
+ * with prefix 0.  Writes group_start (host int32 [num_seqs + 1]),
+ * prefix_lens (host int32 [num_seqs]) and, if non-NULL, the largest group
+ * size; returns the group count, or PA_ERR_INVALID_ARG for an unknown or
+ * swapped-out sequence. */
+int pa_bm_shared_prefix_groups(const pa_block_manager* m, const int32_t* seq_ids,
+                               int num_seqs, int min_shared_blocks,
+                               int32_t* group_start, int32_t* prefix_lens,
+                               int* max_group_size);
+
 /* Capacity, in bytes, of the workspace built into the library for
  * pa_decode_attention_static_ws (32 MiB per GPU that uses the library). */
 #define PA_STATIC_WORKSPACE_BYTES (32u << 20)

@@ -45,6 +45,8 @@ def _lib():
         lib.pa_bm_swap_out.restype = i32
         lib.pa_bm_swap_in.argtypes = [p, i32, p, i32]
         lib.pa_bm_swap_in.restype = i32
+        lib.pa_bm_shared_prefix_groups.argtypes = [p, p, i32, i32, p, p, p]
+        lib.pa_bm_shared_prefix_groups.restype = i32
         lib._bm_declared = True
     return lib
 
@@ -147,3 +149,17 @@ class BlockManager:
         n = self._check(_lib().pa_bm_swap_in(self._m, seq_id, _ptr(pairs), cap),
                         "pa_bm_swap_in")
         return pairs[:n].copy()
+
+    def shared_prefix_groups(self, seq_ids, min_shared_blocks: int = 1):
+        """(group_start int32 [G+1], prefix_lens int32 [G], max_group_size)
+        for pa_decode_attention_shared_prefix on the batch `seq_ids` (in
+        launch order): consecutive sequences sharing at least
+        min_shared_blocks leading blocks are grouped."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int32)
+        gs = np.zeros(ids.size + 1, dtype=np.int32)
+        pl = np.zeros(max(ids.size, 1), dtype=np.int32)
+        mg = ctypes.c_int(0)
+        g = self._check(_lib().pa_bm_shared_prefix_groups(
+            self._m, _ptr(ids), ids.size, int(min_shared_blocks), _ptr(gs),
+            _ptr(pl), ctypes.byref(mg)), "pa_bm_shared_prefix_groups")
+        return gs[:g + 1].copy(), pl[:g].copy(), int(mg.value)

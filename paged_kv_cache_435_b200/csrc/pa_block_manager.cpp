@@ -20,6 +20,7 @@
 //  * Swapping: a sequence's blocks can move to a CPU pool and back, producing
 //    the (src, dst) pairs for pa_swap_blocks ("Preemption and Recovery").
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 #include <new>
 #include <unordered_map>
@@ -373,6 +374,46 @@ int pa_bm_swap_in(pa_block_manager* m, int seq_id, int64_t* pairs,
     }
     s->on_cpu = false;
     return n;
+}
+
+// Groups for pa_decode_attention_shared_prefix: runs of consecutive batch
+// sequences whose block tables agree on at least min_shared_blocks leading
+// blocks; a group's prefix is the blocks all its members share.
+int pa_bm_shared_prefix_groups(const pa_block_manager* m, const int32_t* seq_ids,
+                               int num_seqs, int min_shared_blocks,
+                               int32_t* group_start, int32_t* prefix_lens,
+                               int* max_group_size) {
+    if (!m || num_seqs < 0 || min_shared_blocks < 1) return PA_ERR_INVALID_ARG;
+    if (!group_start || (num_seqs > 0 && (!seq_ids || !prefix_lens)))
+        return PA_ERR_INVALID_ARG;
+    for (int i = 0; i < num_seqs; ++i) {
+        const int id = seq_ids[i];
+        if (id < 0 || id >= (int)m->seqs.size() || !m->seqs[id].alive ||
+            m->seqs[id].on_cpu)
+            return PA_ERR_INVALID_ARG;
+    }
+    int groups = 0, largest = 1;
+    group_start[0] = 0;
+    for (int i = 0; i < num_seqs;) {
+        const std::vector<int>& first = m->seqs[seq_ids[i]].blocks;
+        int common = (int)first.size();
+        int j = i + 1;
+        for (; j < num_seqs; ++j) {
+            const std::vector<int>& b = m->seqs[seq_ids[j]].blocks;
+            const int lim = std::min(common, (int)b.size());
+            int c = 0;
+            while (c < lim && b[c] == first[c]) ++c;
+            if (c < min_shared_blocks) break;
+            common = c;
+        }
+        // A sequence alone shares nothing: it gets the per-sequence pass only.
+        prefix_lens[groups] = j - i >= 2 ? common * m->block_size : 0;
+        group_start[++groups] = j;
+        largest = std::max(largest, j - i);
+        i = j;
+    }
+    if (max_group_size) *max_group_size = largest;
+    return groups;
 }
 
 }  // extern "C"

@@ -159,3 +159,52 @@ def test_random_operations_keep_refcounts_consistent():
             np.add.at(counts, tbl, 1)
         assert all(m.refcount(b) == counts[b] for b in range(nb))
         assert m.num_free_blocks == int((counts == 0).sum())
+
+
+def shared_blocks(m, ids):
+    """Leading blocks that every sequence of ids maps to the same block."""
+    tables = [list(m.block_table(s)) for s in ids]
+    n = 0
+    while all(len(t) > n for t in tables) and len({t[n] for t in tables}) == 1:
+        n += 1
+    return n
+
+
+def test_shared_prefix_groups_follow_forks_and_copy_on_write():
+    m = BlockManager(64, 16)
+    a, _, _ = m.add_sequence(toks(40))            # 2 full blocks + 8 tokens
+    samples = [a] + [m.fork(a) for _ in range(3)]
+    b, _, _ = m.add_sequence(toks(20, 500))       # unrelated prompt
+    c = m.fork(b)
+    lone, _, _ = m.add_sequence(toks(7, 900))
+    batch = samples + [b, c, lone]
+    gs, pl, mg = m.shared_prefix_groups(batch)
+    # the four samples share all 3 blocks (the partial one too, before CoW)
+    assert list(gs) == [0, 4, 6, 7] and list(pl) == [48, 32, 0] and mg == 4
+    for i in range(len(pl)):
+        members = batch[gs[i]:gs[i + 1]]
+        if len(members) > 1:
+            assert pl[i] == 16 * shared_blocks(m, members)
+    # every sample appends a token: copy-on-write of the partial block
+    for s in samples:
+        m.append_slots(s, 1, np.array([7], dtype=np.int32))
+    gs, pl, _ = m.shared_prefix_groups(batch)
+    assert list(gs) == [0, 4, 6, 7] and list(pl) == [32, 32, 0]
+    # interleaved order: runs only, a non-sharing neighbour ends a group
+    gs, pl, _ = m.shared_prefix_groups([samples[0], b, samples[1], c])
+    assert list(gs) == [0, 1, 2, 3, 4] and list(pl) == [0, 0, 0, 0]
+    # a stricter threshold splits groups whose common prefix is too short
+    gs, pl, _ = m.shared_prefix_groups(batch, min_shared_blocks=3)
+    assert list(gs) == [0, 1, 2, 3, 4, 5, 6, 7] and not any(pl)
+
+
+def test_shared_prefix_groups_reject_bad_sequences():
+    m = BlockManager(16, 16, num_cpu_blocks=8)
+    a, _, _ = m.add_sequence(toks(20))
+    with pytest.raises(nat.PAError):
+        m.shared_prefix_groups([a, 99])
+    m.swap_out(a)
+    with pytest.raises(nat.PAError):
+        m.shared_prefix_groups([a])
+    gs, pl, mg = m.shared_prefix_groups([])
+    assert list(gs) == [0] and len(pl) == 0 and mg == 1

@@ -142,3 +142,65 @@ def test_no_groups_is_plain_decode():
         case.scale, ws)
     torch.cuda.synchronize()
     assert_attn_close(out, reference(case), "no groups")
+
+
+def test_block_manager_groups_drive_the_shared_prefix_call():
+    """Parallel sampling end to end: the block manager forks samples from
+    three prompts, two decode steps append a token to every sample (with the
+    copy-on-write copies and new-token writes on the GPU), and the manager's
+    groups feed the shared-prefix call, checked against the fp64 oracle."""
+    from paged_kv_cache_435_b200.block_manager import BlockManager
+    NB, BS, HKV, HQ, D = 256, 16, 4, 16, 128
+    gen = torch.Generator().manual_seed(21)
+
+    def rows(n):
+        return (torch.randn(n, HKV, D, generator=gen).to(torch.bfloat16),
+                torch.randn(n, HKV, D, generator=gen).to(torch.bfloat16))
+
+    k = torch.randn(NB, BS, HKV, D, generator=gen).to(torch.bfloat16).cuda()
+    v = torch.randn(NB, BS, HKV, D, generator=gen).to(torch.bfloat16).cuda()
+    m = BlockManager(NB, BS)
+    batch = []
+    for pi, plen in enumerate([300, 130, 77]):
+        p, slots, _ = m.add_sequence(np.arange(plen, dtype=np.int32) + 1000 * pi)
+        nk, nv = rows(plen)
+        pa.pa_reshape_and_cache(nk.cuda(), nv.cuda(), k, v, torch.from_numpy(slots).cuda())
+        batch += [p] + [m.fork(p) for _ in range(pi + 2)]
+    for step in range(2):
+        slots, pairs = [], []
+        for s in batch:
+            sl, pr = m.append_slots(s, 1, np.array([7 + step], dtype=np.int32))
+            slots.append(sl)
+            pairs.append(pr)
+        pairs = np.concatenate(pairs).astype(np.int64)
+        if len(pairs):
+            pa.pa_copy_blocks([k], [v], torch.from_numpy(pairs).cuda())
+        nk, nv = rows(len(batch))
+        pa.pa_reshape_and_cache(nk.cuda(), nv.cuda(), k, v,
+                                torch.from_numpy(np.concatenate(slots)).cuda())
+    tables = [m.block_table(s) for s in batch]
+    MB = max(len(t) for t in tables)
+    bt = np.full((len(batch), MB), -1, dtype=np.int32)
+    for i, t in enumerate(tables):
+        bt[i, :len(t)] = t
+    lens = np.array([m.seq_len(s) for s in batch], dtype=np.int32)
+    gs, pl, mg = m.shared_prefix_groups(batch)
+    assert len(gs) == 4 and pl.min() > 0 and mg == 5
+
+    q = torch.randn(len(batch), HQ, D, generator=gen).to(torch.bfloat16).cuda()
+    maxlen = int(lens.max())
+    out = torch.empty(len(batch), HQ, D, dtype=torch.float32, device="cuda")
+    ws = torch.empty(pa.pa_shared_prefix_workspace_size(len(batch), HQ, HKV, D, BS, maxlen),
+                     dtype=torch.uint8, device="cuda")
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bt_d, lens_d = torch.from_numpy(bt).cuda(), torch.from_numpy(lens).cuda()
+    pa.pa_decode_attention_shared_prefix(
+        out, q, k, v, bt_d, lens_d, torch.from_numpy(gs).cuda(),
+        torch.from_numpy(pl).cuda(), maxlen, mg, 0.088, ws, error_flags=flags)
+    plain = torch.empty_like(out)
+    pa.pa_decode_attention(plain, q, k, v, bt_d, lens_d, maxlen, 0.088)
+    torch.cuda.synchronize()
+    assert int(flags.item()) == 0
+    ref = oracle.paged_decode_attention(q.cpu(), bits(k), bits(v), bt, lens, 0.088, HKV)
+    assert_attn_close(out, ref, "block-manager groups")
+    assert (plain - out).abs().max().item() <= 2e-5
