@@ -229,17 +229,18 @@ int pa_multi_query_attention(float* out, const void* q, const void* k_cache,
  * this call also shares the reading of it.
  *
  * Group i is the sequences group_start[i] .. group_start[i+1]-1.  Their
- * block tables agree on the first prefix_lens[i] / block_size entries (the
- * shared blocks); the library reads those entries from the group's first
- * sequence only.  For each sequence s of a group with context length L, the
- * first min(prefix_lens[i], L) tokens are attended in a group pass that
- * streams every shared block once for all of the group's query rows (the
- * tcgen05 tensor cores, up to 32 rows per kv head and pass); the remaining
- * tokens of s are attended per sequence by the decode kernel, which merges
- * the two partial softmax results exactly:
- *     out = (l1 2^(m1-M) o1 + l2 2^(m2-M) o2) / (l1 2^(m1-M) + l2 2^(m2-M)).
- * Sequences outside every group, and groups whose description is invalid
- * (reported with PA_DEVERR_PREFIX), are attended as by pa_decode_attention.
+ * block tables agree on the shared blocks: the first prefix_lens[i] /
+ * block_size entries, or all entries of a member whose context is shorter;
+ * the library reads them from the table of one member whose context covers
+ * them.  For each (group, kv head) a group pass on the tcgen05
+ * tensor cores (up to 32 query rows per pass) streams the shared blocks once
+ * for all members' query rows, then each member's private tail for that
+ * member's rows only: sequence s with context length L attends its first
+ * min(prefix_lens[i], L) tokens through the shared blocks and the rest
+ * through its own table, in one online softmax.  Sequences outside every
+ * group, and groups whose description is invalid (reported with
+ * PA_DEVERR_PREFIX), are attended by the decode kernel as by
+ * pa_decode_attention.
  *
  *   group_start     int32 [num_groups + 1], device, non-decreasing, in
  *                   [0, num_seqs]; groups need not cover every sequence.

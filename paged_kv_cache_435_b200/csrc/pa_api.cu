@@ -82,23 +82,18 @@ size_t workspace_bytes_for(int num_seqs, int num_heads, int head_size,
     return bytes;
 }
 
-// Shared-prefix call: the decode split's scratch, then the group pass's
-// partial results (O/l, max, sum per row) and each sequence's shared length.
+// Shared-prefix call: the decode split's scratch, then one flag per
+// sequence (the group pass answered it).
 struct PrefixLayout {
-    size_t split_bytes, o_off, m_off, l_off, sh_off, total;
+    size_t done_off, total;
 };
 
 PrefixLayout prefix_layout(int num_seqs, int num_heads, int head_size,
                            int max_partitions) {
     PrefixLayout L;
-    const size_t rows = (size_t)num_seqs * num_heads;
-    L.split_bytes = (workspace_bytes_for(num_seqs, num_heads, head_size,
-                                         max_partitions) + 255) & ~(size_t)255;
-    L.o_off = L.split_bytes;
-    L.m_off = L.o_off + ((rows * head_size * 4 + 255) & ~(size_t)255);
-    L.l_off = L.m_off + ((rows * 4 + 255) & ~(size_t)255);
-    L.sh_off = L.l_off + ((rows * 4 + 255) & ~(size_t)255);
-    L.total = L.sh_off + (((size_t)num_seqs * 4 + 255) & ~(size_t)255);
+    L.done_off = (workspace_bytes_for(num_seqs, num_heads, head_size,
+                                      max_partitions) + 255) & ~(size_t)255;
+    L.total = L.done_off + (((size_t)num_seqs * 4 + 255) & ~(size_t)255);
     return L;
 }
 
@@ -428,16 +423,14 @@ int pa_decode_attention_shared_prefix(
     if (num_groups > 0) {
         const int per_tile = pa::kMultiRowTile / G;
         pa::MultiRowParams r{};
-        r.out = reinterpret_cast<float*>(ws + lay.o_off);
-        r.out_m = reinterpret_cast<float*>(ws + lay.m_off);
-        r.out_l = reinterpret_cast<float*>(ws + lay.l_off);
+        r.out = out;
         r.q = static_cast<const uint16_t*>(q);
         r.k_cache = static_cast<const uint16_t*>(k_cache);
         r.v_cache = static_cast<const uint16_t*>(v_cache);
         r.block_tables = block_tables;
         r.context_lens = context_lens;
         r.groups = groups;
-        r.seq_shared = reinterpret_cast<int32_t*>(ws + lay.sh_off);
+        r.seq_done = reinterpret_cast<int32_t*>(ws + lay.done_off);
         r.error_flags = error_flags;
         r.shared_prefix_mode = 1;
         r.num_seqs = num_seqs;
@@ -483,11 +476,8 @@ int pa_decode_attention_shared_prefix(
     p.max_partitions = np;
     p.scale_log2 = pa::log2e_scale(scale);
     p.block_size = block_size;
-    p.cascade = num_groups > 0 ? 1 : 0;
-    p.pref_o = reinterpret_cast<const float*>(ws + lay.o_off);
-    p.pref_m = reinterpret_cast<const float*>(ws + lay.m_off);
-    p.pref_l = reinterpret_cast<const float*>(ws + lay.l_off);
-    p.seq_shared = reinterpret_cast<const int32_t*>(ws + lay.sh_off);
+    p.skip_seq = num_groups > 0 ? reinterpret_cast<const int32_t*>(ws + lay.done_off)
+                                : nullptr;
     cudaError_t e = pa::launch_paged_decode(p, head_size, block_size, st);
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

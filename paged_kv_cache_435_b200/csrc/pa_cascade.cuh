@@ -4,11 +4,10 @@
 //
 // Group i is the sequences group_start[i] .. group_start[i+1]-1, whose first
 // prefix_lens[i] tokens live in the same physical blocks.  The group pass
-// (pa_multi_row.cu) attends those tokens once for all of the group's query
-// rows; the decode kernel attends each sequence's remaining tokens and merges.
-// Both derive a sequence's shared length with the functions below from the
-// same arrays, so they agree on every input, valid or not: an invalid group
-// counts as unshared and its sequences are attended by the decode kernel alone.
+// (pa_multi_row.cu) answers every member of a valid group with a prefix; the
+// decode kernel answers the other sequences.  Both sides classify a sequence
+// with the functions below from the same arrays, so they agree on every
+// input, valid or not: an invalid group counts as ungrouped.
 #pragma once
 
 #include <cstdint>
@@ -52,15 +51,6 @@ __device__ __forceinline__ int cascade_group_of(const CascadeGroups& c, int s) {
         if (c.group_start[mid] <= s) lo = mid; else hi = mid - 1;
     }
     return s < c.group_start[lo + 1] ? lo : -1;
-}
-
-// Tokens of sequence s (context length L) that the group pass attends.
-__device__ __forceinline__ int cascade_shared_len(const CascadeGroups& c, int s, int L,
-                                                  int num_seqs, int block_size) {
-    const int i = cascade_group_of(c, s);
-    if (i < 0) return 0;
-    const int P = cascade_group_prefix(c, i, num_seqs, block_size, nullptr, false);
-    return P < L ? P : L;
 }
 
 }  // namespace pa

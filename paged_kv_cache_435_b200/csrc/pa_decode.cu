@@ -84,7 +84,6 @@ struct Item {
     int tok0;    // first token of the partition
     int tok1;    // one past its last token
     int nparts;  // partitions of this sequence
-    int sh;      // tokens before tok0 left to the shared-prefix group pass
 };
 
 __device__ __forceinline__ int clamped_len(const DecodeParams& p, int s) {
@@ -100,24 +99,21 @@ __device__ __forceinline__ int parts_of(int L, int P) {
     return L <= 0 ? 1 : (L + P - 1) / P;  // an empty context still owns one item
 }
 
-// First token of sequence s this kernel attends (0 unless a shared-prefix
-// group pass covered the tokens before it; that pass wrote the length).
-template <bool kCascade, int BS>
-__device__ __forceinline__ int first_token(const DecodeParams& p, int s, int L) {
-    return kCascade ? min(p.seq_shared[s], L) : 0;
+// Sequence s has no items here: a shared-prefix group pass answered it.
+template <bool kSkip>
+__device__ __forceinline__ bool skipped(const DecodeParams& p, int s) {
+    return kSkip && p.skip_seq[s] != 0;
 }
 
-// Item k (k = 0, 1, ...) of this CTA, or of this warp when warps take
-// items of their own (kWarp: short items, no merge across warps).
-template <bool kPersist, bool kCascade, bool kWarp, int BS>
+// Item k of this CTA (k = 0, 1, ...).
+template <bool kPersist, bool kSkip>
 __device__ __forceinline__ Item get_item(const DecodeParams& p,
-                                         const int* prefix, int k, int warp) {
+                                         const int* prefix, int k) {
     Item it;
     it.s = -1;
     int s, part;
     if (kPersist) {
-        const int j = kWarp ? (int)(blockIdx.y * kWarps + warp) + k * (int)(gridDim.y * kWarps)
-                            : (int)blockIdx.y + k * (int)gridDim.y;
+        const int j = blockIdx.y + k * gridDim.y;
         if (j >= prefix[p.num_seqs]) return it;
         int lo = 0, hi = p.num_seqs - 1;  // largest s with prefix[s] <= j
         while (lo < hi) {
@@ -131,34 +127,24 @@ __device__ __forceinline__ Item get_item(const DecodeParams& p,
         s = blockIdx.z;
         part = blockIdx.y;
     }
+    if (skipped<kSkip>(p, s)) return it;
     const int L = clamped_len(p, s);
-    const int sh = first_token<kCascade, BS>(p, s, L);
-    const int np = parts_of(L - sh, p.partition_size);
+    const int np = parts_of(L, p.partition_size);
     if (part >= np) return it;
     it.s = s;
     it.part = part;
     it.L = L;
     it.nparts = np;
-    it.sh = sh;
-    it.tok0 = sh + part * p.partition_size;
+    it.tok0 = part * p.partition_size;
     it.tok1 = min(L, it.tok0 + p.partition_size);
     return it;
 }
 
-// Chunks of `it` that warp w owns: w, w+4, ... of the item, or all of them
-// when the warp owns the item.
-template <bool kWarp>
+// Chunks of `it` that warp w owns.
 __device__ __forceinline__ int warp_chunks(const Item& it, int warp) {
     if (it.s < 0) return 0;
     const int n = (it.tok1 - it.tok0 + kChunk - 1) / kChunk;
-    if (kWarp) return n;
     return n > warp ? (n - warp + kWarps - 1) / kWarps : 0;
-}
-
-// Chunk index within the item of the warp's i-th chunk.
-template <bool kWarp>
-__device__ __forceinline__ int chunk_of(int warp, int i) {
-    return kWarp ? i : warp + kWarps * i;
 }
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map,
@@ -179,7 +165,7 @@ __device__ __forceinline__ void named_bar_arrive(int id) {
     asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(kThreads) : "memory");
 }
 
-template <int D, int BS, bool kPersist, bool kCascade, bool kWarp>
+template <int D, int BS, bool kPersist, bool kSkip>
 __global__ void __launch_bounds__(kThreads, kTargetCtasPerSM)
 paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
@@ -218,10 +204,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         for (int base = 0; base < p.num_seqs; base += kThreads) {
             const int s = base + threadIdx.x;
             int v = 0;
-            if (s < p.num_seqs) {
-                const int L = clamped_len(p, s);
-                v = parts_of(L - first_token<kCascade, BS>(p, s, L), p.partition_size);
-            }
+            if (s < p.num_seqs && !skipped<kSkip>(p, s))
+                v = parts_of(clamped_len(p, s), p.partition_size);
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int t = __shfl_up_sync(0xffffffffu, v, o);
@@ -265,20 +249,20 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
     // Lane l finds the (ids_base + l)-th chunk of the stream and its slot.
     auto refill = [&]() {
         int k = prod_k, i = prod_i, n = lane;
-        Item it = get_item<kPersist, kCascade, kWarp, BS>(p, prefix, k, warp);
+        Item it = get_item<kPersist, kSkip>(p, prefix, k);
         for (;;) {
             if (it.s < 0) break;
-            const int rem = warp_chunks<kWarp>(it, warp) - i;
+            const int rem = warp_chunks(it, warp) - i;
             if (rem > n) break;
             n -= rem > 0 ? rem : 0;
             ++k;
             i = 0;
-            it = get_item<kPersist, kCascade, kWarp, BS>(p, prefix, k, warp);
+            it = get_item<kPersist, kSkip>(p, prefix, k);
         }
         int slot = -1;
         if (it.s >= 0) {
             i += n;
-            const int ctok = it.tok0 + chunk_of<kWarp>(warp, i) * kChunk;
+            const int ctok = it.tok0 + (warp + kWarps * i) * kChunk;
             int id = tables[(int64_t)it.s * p.max_blocks_per_seq + ctok / BS];
             if (id < 0 || id >= p.num_blocks) {
                 report(p.error_flags, PA_DEVERR_BLOCK_ID);
@@ -340,20 +324,20 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
             dst[ks][1] = live ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8 + qc) : 0u;
         }
     };
-    Item next_it = get_item<kPersist, kCascade, kWarp, BS>(p, prefix, 0, warp);
+    Item next_it = get_item<kPersist, kSkip>(p, prefix, 0);
     uint32_t qnext[D / 16][2];
     load_q(next_it, qnext);
     for (;; ++k) {
         const Item it = next_it;
         if (it.s < 0) break;
-        const int my_n = warp_chunks<kWarp>(it, warp);
+        const int my_n = warp_chunks(it, warp);
         uint32_t qa[D / 16][2];
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
             qa[ks][0] = qnext[ks][0];
             qa[ks][1] = qnext[ks][1];
         }
-        next_it = get_item<kPersist, kCascade, kWarp, BS>(p, prefix, k + 1, warp);
+        next_it = get_item<kPersist, kSkip>(p, prefix, k + 1);
         load_q(next_it, qnext);
 
         float o[D / 8][4];
@@ -376,7 +360,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
             ++cons_count;
             if (aborted) continue;
 
-            const int ctok = it.tok0 + chunk_of<kWarp>(warp, i) * kChunk;
+            const int ctok = it.tok0 + (warp + kWarps * i) * kChunk;
             const int valid = min(kChunk, it.tok1 - ctok);
             const uint32_t kaddr = smem_u32(my_ring + stage * C::kStageBytes);
             const uint32_t vaddr = kaddr + C::kKVBytes;
@@ -476,42 +460,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         // ---------------- item end: merge the four warps ----------------
         l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
         l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
-        if (kWarp) {
-            // The warp holds the whole item: row qr is o[.][0..1] (P_hi V)
-            // plus o[.][2..3] (P_lo V), with max m_run and sum l_run.
-            if (qr < G) {
-                const int h = g * G + qr;
-                const bool direct = it.nparts == 1;
-                const int64_t row = (int64_t)it.s * Hq + h;
-                const int64_t idx = row * p.max_partitions + it.part;
-                float* dst = direct ? p.out + row * D : p.tmp_o + idx * D;
-                float den = l_run, wa = 1.f, wb = 0.f;
-                const float* po = nullptr;
-                if (kCascade && direct && it.sh > 0) {
-                    const float mp = p.pref_m[row], lp = p.pref_l[row];
-                    const float Mt = fmaxf(m_run, mp);
-                    wa = m_run == -INFINITY ? 0.f : exp2f(m_run - Mt);
-                    wb = lp * exp2f(mp - Mt);
-                    den = den * wa + wb;
-                    po = p.pref_o + row * D;
-                }
-#pragma unroll
-                for (int j = 0; j < D / 8; ++j) {
-                    float v[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        float acc = o[j][e] + o[j][e + 2];
-                        if (kCascade && po != nullptr) acc = acc * wa + wb * po[8 * j + qc + e];
-                        v[e] = it.L > 0 ? acc / den : 0.f;
-                    }
-                    *reinterpret_cast<float2*>(dst + 8 * j + qc) = make_float2(v[0], v[1]);
-                }
-                if (!direct && (lane & 3) == 0) {
-                    p.tmp_m[idx] = m_run;
-                    p.tmp_l[idx] = den;
-                }
-            }
-        } else if (warp != 0) {
+        if (warp != 0) {
             if (k > 0) named_bar_sync(2);  // warp 0 has read the previous item
             float* dst = red_o + ((warp - 1) * kMaxGroup + qr) * C::kRedStride + qc;
 #pragma unroll
@@ -542,18 +491,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                 const int64_t row = (int64_t)it.s * Hq + h;
                 const int64_t idx = row * p.max_partitions + it.part;
                 float* dst = direct ? p.out + row * D : p.tmp_o + idx * D;
-                // Shared-prefix call, unsplit sequence: fold in the group
-                // pass's partial (its O/l, max and sum) here.
-                float wa = 1.f, wb = 0.f;
-                const float* po = nullptr;
-                if (kCascade && direct && it.sh > 0) {
-                    const float mp = p.pref_m[row], lp = p.pref_l[row];
-                    const float Mt = fmaxf(M, mp);
-                    wa = M == -INFINITY ? 0.f : exp2f(M - Mt);
-                    wb = lp * exp2f(mp - Mt);
-                    den = den * wa + wb;
-                    po = p.pref_o + row * D;
-                }
 #pragma unroll
                 for (int j = 0; j < D / 8; ++j) {
                     float v[2];
@@ -563,7 +500,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
 #pragma unroll
                         for (int w = 1; w < kWarps; ++w)
                             acc += sc[w] * red_o[((w - 1) * kMaxGroup + qr) * C::kRedStride + 8 * j + qc + e];
-                        if (kCascade && po != nullptr) acc = acc * wa + wb * po[8 * j + qc + e];
                         v[e] = it.L > 0 ? acc / den : 0.f;
                     }
                     *reinterpret_cast<float2*>(dst + 8 * j + qc) = make_float2(v[0], v[1]);
@@ -577,7 +513,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         }
     }
     // Consume warp 0's last "merged" arrival so no barrier is left pending.
-    if (!kWarp && warp != 0 && k > 0) named_bar_sync(2);
+    if (warp != 0 && k > 0) named_bar_sync(2);
 
     if (aborted) {
         // Drain copies still in flight on this warp's ring (bounded) before
@@ -605,11 +541,10 @@ paged_decode_reduce_kernel(const DecodeParams p) {
     pdl_wait();  // the partials come from the grid launched just before
     int L = p.context_lens[s];
     L = L < 0 ? 0 : (L > p.max_context_len ? p.max_context_len : L);
-    const int sh = p.cascade ? min(p.seq_shared[s], L) : 0;
-    const int np = (L - sh + p.partition_size - 1) / p.partition_size;
+    if (p.skip_seq != nullptr && p.skip_seq[s] != 0) return;  // answered elsewhere
+    const int np = (L + p.partition_size - 1) / p.partition_size;
     if (np <= 1) return;  // written directly by the partition kernel
     const int64_t base = ((int64_t)s * p.num_heads + h) * p.max_partitions;
-    const int64_t row = (int64_t)s * p.num_heads + h;
 
     __shared__ float warp_max[kReduceWarps];
     __shared__ float part_acc[kReduceWarps][D];
@@ -625,7 +560,6 @@ paged_decode_reduce_kernel(const DecodeParams p) {
     M = warp_max[0];
 #pragma unroll
     for (int w = 1; w < kReduceWarps; ++w) M = fmaxf(M, warp_max[w]);
-    if (sh > 0) M = fmaxf(M, p.pref_m[row]);  // the group pass's partial joins
 
     float acc[V];
 #pragma unroll
@@ -661,13 +595,6 @@ paged_decode_reduce_kernel(const DecodeParams p) {
 #pragma unroll
             for (int v = 0; v < V; ++v) acc[v] += wts[u] * vals[u][v];
         }
-    }
-    if (sh > 0 && warp == 0) {
-        const float wp = p.pref_l[row] * exp2f(p.pref_m[row] - M);
-        den += wp;
-        const float* po = p.pref_o + row * D + lane * V;
-#pragma unroll
-        for (int v = 0; v < V; ++v) acc[v] += wp * po[v];
     }
 #pragma unroll
     for (int v = 0; v < V; ++v) part_acc[warp][lane * V + v] = acc[v];
@@ -754,38 +681,32 @@ cudaError_t set_smem(Kernel kernel, int bytes, int* flags) {
     return cudaSuccess;
 }
 
-template <int D, int BS, bool kCascade>
+template <int D, int BS, bool kSkip>
 cudaError_t launch_partition_kernel(const DecodeParams& p, const CUtensorMap& tmk,
                                     const CUtensorMap& tmv, cudaStream_t stream) {
     using C = Cfg<D>;
     static int grid_ready[64] = {0};
     static int persist_ready[64] = {0};
-    // Persistent CTAs when sequences are split; for the short private tails
-    // of a shared-prefix call, persistent warps that each own whole items
-    // (the copies of the next item stay in flight across item boundaries
-    // and no warp waits for another's merge).
-    const bool persist = (p.max_partitions > 1 || kCascade) && p.num_seqs <= kMaxPersistSeqs;
+    // Persistent CTAs when sequences are split, and when some sequences are
+    // skipped (the compact item list then spends no CTA on them).
+    const bool persist = (p.max_partitions > 1 || kSkip) && p.num_seqs <= kMaxPersistSeqs;
     cudaError_t e;
     if (persist) {
-        constexpr bool kWarp = kCascade;
-        e = set_smem(paged_decode_kernel<D, BS, true, kCascade, kWarp>, C::kSmemPersist,
-                     persist_ready);
+        e = set_smem(paged_decode_kernel<D, BS, true, kSkip>, C::kSmemPersist, persist_ready);
         if (e != cudaSuccess) return e;
         long long per_head = (kTargetCtasPerSM * kNumSMs + p.num_kv_heads - 1) / p.num_kv_heads;
         const long long items = (long long)p.num_seqs * p.max_partitions;
-        const long long streams = kWarp ? (items + kWarps - 1) / kWarps : items;
-        if (per_head > streams) per_head = streams;
+        if (per_head > items) per_head = items;
         if (per_head < 1) per_head = 1;
         dim3 grid((unsigned)p.num_kv_heads, (unsigned)per_head, 1);
-        e = launch_pdl(paged_decode_kernel<D, BS, true, kCascade, kWarp>, grid, dim3(kThreads),
+        e = launch_pdl(paged_decode_kernel<D, BS, true, kSkip>, grid, dim3(kThreads),
                        C::kSmemPersist, stream, tmk, tmv, p);
     } else {
-        e = set_smem(paged_decode_kernel<D, BS, false, kCascade, false>, C::kSmemGrid,
-                     grid_ready);
+        e = set_smem(paged_decode_kernel<D, BS, false, kSkip>, C::kSmemGrid, grid_ready);
         if (e != cudaSuccess) return e;
         dim3 grid((unsigned)p.num_kv_heads, (unsigned)p.max_partitions,
                   (unsigned)p.num_seqs);
-        e = launch_pdl(paged_decode_kernel<D, BS, false, kCascade, false>, grid, dim3(kThreads),
+        e = launch_pdl(paged_decode_kernel<D, BS, false, kSkip>, grid, dim3(kThreads),
                        C::kSmemGrid, stream, tmk, tmv, p);
     }
     count_launch();
@@ -798,8 +719,9 @@ cudaError_t launch_typed(const DecodeParams& p, cudaStream_t stream) {
     if (!encode_pool_map(&tmk, p.k_cache, p.num_blocks, BS, p.num_kv_heads, D) ||
         !encode_pool_map(&tmv, p.v_cache, p.num_blocks, BS, p.num_kv_heads, D))
         return cudaErrorInvalidValue;
-    cudaError_t e = p.cascade ? launch_partition_kernel<D, BS, true>(p, tmk, tmv, stream)
-                              : launch_partition_kernel<D, BS, false>(p, tmk, tmv, stream);
+    cudaError_t e = p.skip_seq != nullptr
+                        ? launch_partition_kernel<D, BS, true>(p, tmk, tmv, stream)
+                        : launch_partition_kernel<D, BS, false>(p, tmk, tmv, stream);
     if (e != cudaSuccess) return e;
     if (p.max_partitions > 1) {
         dim3 rgrid((unsigned)p.num_heads, (unsigned)p.num_seqs);

@@ -28,14 +28,9 @@ struct DecodeParams {
     int max_partitions;          // ceil(max_context_len / partition_size)
     float scale_log2;            // scale * log2(e)
     int block_size;
-    // Shared-prefix call: each sequence starts at its shared length (the
-    // group pass covered the tokens before it) and its result is merged
-    // with the group pass's partial (pref_o = O/l, pref_m, pref_l per row).
-    int cascade;
-    const float* pref_o;         // fp32 [B][Hq][D]
-    const float* pref_m;         // fp32 [B][Hq] (log2 domain)
-    const float* pref_l;         // fp32 [B][Hq]
-    const int32_t* seq_shared;   // int32 [B]: tokens the group pass covered
+    // Shared-prefix call: the group pass answered the sequences with
+    // skip_seq[s] != 0; they have no items here (null: none skipped).
+    const int32_t* skip_seq;     // int32 [B]
 };
 
 // scale * log2(e): logits are kept in the log2 domain (exp2f).

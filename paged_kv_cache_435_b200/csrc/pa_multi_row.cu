@@ -7,9 +7,12 @@
 //    causal within the chunk ("vLLM: Anatomy and Mechanisms of
 //    High-Throughput LLM Inference", "Speculative Decoding");
 //  * the group pass of pa_decode_attention_shared_prefix: the samples of one
-//    prompt times the G heads are the rows, over the prompt blocks they share
-//    ("Memory Sharing via Copy-on-Write (CoW)"), written as partial softmax
-//    results for the decode kernel to merge.
+//    prompt times the G heads are the rows ("Memory Sharing via Copy-on-Write
+//    (CoW)").  An item streams the prompt blocks the samples share once for
+//    all rows, then each sample's private tail for that sample's rows only,
+//    along one virtual token axis: [0, shared end) shared, then the tails,
+//    each padded to 16 tokens; a row sees the shared tokens of its context
+//    and its own tail.
 // With 32 rows over a stream of KV the work is 32 flop per KV byte, far below
 // the tensor roofline: the goal is to read every block once at HBM speed with
 // the math hidden behind it.  A 128-row M tile would waste 3/4 of the tensor
@@ -90,15 +93,18 @@ constexpr int kCmaxOff = kMiscOff;                     // float [32][4]
 // epilogue writes out.
 struct ItemSlot {
     int table_seq, g, range_end, nch;   // nch < 0: no further items
-    int min_lim, pad[3];                // smallest limit over existing rows
-    int lim[32];                        // last visible token of each row
+    int min_lim, nmem, shared_r16, P;   // smallest row limit; members (group
+                                        // mode); end of the shared region
+                                        // rounded to 16; prefix length
+    int lim[32];                        // rows: last visible shared token
+    int tail_lo[32], tail_hi[32];       // rows: their member's tail [lo, hi)
+    int mem_seq[32];                    // members: sequence
+    int mem_v[32], mem_vend[32];        // members: tail pieces [v, vend)
     long long row[32];                  // q / out row of each row (-1: none)
     float red_l[32][4];                 // per-warp partial row sums
-    float m[32];                        // reference max of each row
-    float l[32];                        // row sums
     float inv_l[32];                    // 1 / row sum (0 for an empty row)
 };
-static_assert(sizeof(ItemSlot) == 1312, "slot layout");
+static_assert(sizeof(ItemSlot) == 1696, "slot layout");
 
 constexpr int kSlotOff = kCmaxOff + 512;
 constexpr int kBarOff = kSlotOff + kSlots * (int)sizeof(ItemSlot);
@@ -291,10 +297,15 @@ struct RowItem {
     int unit;       // sequence or group; -1: nothing to do
     int tile;
     int g;
-    int table_seq;  // sequence whose block table is read
-    int range_end;  // tokens [0, range_end) are streamed
+    int table_seq;  // sequence whose block table holds the shared tokens
+    int range_end;  // virtual tokens [0, range_end) are streamed
     int nch;        // 128-token chunks
+    int P;          // group mode: prefix length
+    int shared_end; // group mode: end of the shared region
+    int m0, nmem;   // group mode: first member of the tile, members
 };
+
+__device__ __forceinline__ int round16(int x) { return (x + 15) & ~15; }
 
 __device__ RowItem row_item(const MultiRowParams& p, int idx, bool report_errors) {
     RowItem it;
@@ -323,9 +334,25 @@ __device__ RowItem row_item(const MultiRowParams& p, int idx, bool report_errors
         const int mpt = kN / G;
         const int m0 = a + tile * mpt;
         const int m1 = min(b, m0 + mpt);
-        for (int s = m0; s < m1; ++s)
-            range_end = max(range_end, min(P, clamp_len(p, s, report_errors)));
-        table_seq = a;
+        if (m0 >= m1) return it;
+        // The shared region is read through the table of the member whose
+        // context covers most of it (a shorter member's table may end first).
+        int shared_end = 0, tails = 0;
+        table_seq = m0;
+        for (int s = m0; s < m1; ++s) {
+            const int L = clamp_len(p, s, report_errors);
+            const int sh = min(P, L);
+            if (sh > shared_end) {
+                shared_end = sh;
+                table_seq = s;
+            }
+            tails += round16(L - sh);
+        }
+        range_end = tails > 0 ? round16(shared_end) + tails : shared_end;
+        it.P = P;
+        it.shared_end = shared_end;
+        it.m0 = m0;
+        it.nmem = m1 - m0;
     }
     if (range_end <= 0) return it;
     it.unit = unit;
@@ -350,10 +377,18 @@ __device__ void unit_work(const MultiRowParams& p, int u, bool report_errors, in
     } else {
         const int P = cascade_group_prefix(p.groups, u, p.num_seqs, p.block_size,
                                            p.error_flags, report_errors);
-        const int members = p.groups.group_start[u + 1] - p.groups.group_start[u];
+        const int a = p.groups.group_start[u];
+        const int members = p.groups.group_start[u + 1] - a;
         const int mpt = kN / p.group;
         tiles = P > 0 ? (members + mpt - 1) / mpt : 0;
-        w = (P + kTok - 1) / kTok + 1;
+        long long tails = 0;
+        if (P > 0)
+            for (int s = a; s < a + members; ++s) {
+                const int L = clamp_len(p, s, false);
+                tails += round16(L - min(P, L));
+            }
+        const long long per_tile = tiles > 0 ? tails / tiles : 0;
+        w = (int)((P + per_tile + kTok - 1) / kTok) + 1;
     }
     tiles = min(tiles, p.tiles);
 }
@@ -450,11 +485,6 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
         *abort_flag = 0;
         mbar_init_fence();
     }
-    // V stages start zeroed: the token rows a tail chunk does not load must be
-    // finite (P is 0 there, but 0 x NaN is NaN).
-    for (int i = threadIdx.x; i < kVStages * kStageBytes / 16; i += kThreads)
-        reinterpret_cast<uint4*>(smem + kVOff)[i] = make_uint4(0, 0, 0, 0);
-    fence_proxy_async_smem();
     if (warp == 6) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols)
@@ -470,11 +500,15 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
     if (warp == 7) {
         // -------------------------------------------------------- scheduler
         if (p.shared_prefix_mode) {
-            // Each sequence's shared length, for the per-sequence pass: the
-            // CTAs split the batch.
-            for (int s = blockIdx.x * 32 + lane; s < p.num_seqs; s += gridDim.x * 32)
-                p.seq_shared[s] = cascade_shared_len(p.groups, s, clamp_len(p, s, false),
-                                                     p.num_seqs, p.block_size);
+            // Which sequences this pass answers (members of valid groups with
+            // a prefix), for the per-sequence pass to skip: the CTAs split
+            // the batch.
+            for (int s = blockIdx.x * 32 + lane; s < p.num_seqs; s += gridDim.x * 32) {
+                const int i = cascade_group_of(p.groups, s);
+                p.seq_done[s] = (i >= 0 && cascade_group_prefix(p.groups, i, p.num_seqs,
+                                                                p.block_size, nullptr,
+                                                                false) > 0) ? 1 : 0;
+            }
         }
         int live = 0;
         // Publish item idx (idx < 0: the end marker); false on abort.
@@ -512,12 +546,42 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             int ml = row >= 0 ? lim : 0x7fffffff;
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) ml = min(ml, __shfl_xor_sync(0xffffffffu, ml, o));
+            // Group mode: member `lane`'s private tail on the virtual axis
+            // (after the shared region, each tail padded to 16 tokens), and
+            // every row's own tail interval.
+            const int shared_r16 = p.shared_prefix_mode ? round16(it.shared_end)
+                                                        : round16(it.range_end);
+            int mv = 0, mt = 0, mpad = 0, mseq = -1;
+            if (p.shared_prefix_mode && lane < it.nmem) {
+                mseq = it.m0 + lane;
+                const int L = clamp_len(p, mseq, false);
+                mt = L - min(it.P, L);
+                mpad = round16(mt);
+            }
+            int incl = mpad;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            mv = shared_r16 + incl - mpad;
+            S.mem_seq[lane] = mseq;
+            S.mem_v[lane] = mv;
+            S.mem_vend[lane] = mv + mpad;
+            const int my_m = row >= 0 && p.shared_prefix_mode ? lane / p.group : 0;
+            const int t_lo = __shfl_sync(0xffffffffu, mv, my_m);
+            const int t_len = __shfl_sync(0xffffffffu, mt, my_m);
+            S.tail_lo[lane] = row >= 0 && p.shared_prefix_mode ? t_lo : 0;
+            S.tail_hi[lane] = row >= 0 && p.shared_prefix_mode ? t_lo + t_len : 0;
             if (lane == 0) {
                 S.table_seq = it.table_seq;
                 S.g = it.g;
                 S.range_end = it.range_end;
                 S.nch = it.nch;
                 S.min_lim = ml;
+                S.nmem = p.shared_prefix_mode ? it.nmem : 0;
+                S.shared_r16 = shared_r16;
+                S.P = p.shared_prefix_mode ? it.P : 0;
             }
             // Q^T row `lane` (K-major, 128-byte swizzle; zeros for a missing row).
             const uint32_t qb = smem_u32(smem + kQOff + (live & 1) * kQBytes);
@@ -605,23 +669,38 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 if (lane == 0) set_abort(abort_flag, p.error_flags);
                 break;
             }
-            const int nch = slots[sl].nch;
+            const ItemSlot& SL = slots[sl];
+            const int nch = SL.nch;
             if (nch < 0) break;
-            const int g = slots[sl].g;
-            const int range_end = slots[sl].range_end;
-            const int32_t* bt = p.block_tables + (int64_t)slots[sl].table_seq * p.max_blocks_per_seq;
+            const int g = SL.g;
+            const int range_end = SL.range_end;
+            const int shared_r16 = SL.shared_r16;
             int win = -1;  // lane l: slot of 16-token piece l of chunks c..c+3
             for (int c = 0; c < nch; ++c) {
                 if ((c & 3) == 0) {
-                    const int t0 = (c * 8 + lane) * 16;
+                    // Virtual token v0: shared (the group's table), or a
+                    // member's tail (that member's table, after the prefix).
+                    const int v0 = (c * 8 + lane) * 16;
+                    int seq = -1, tok = v0;
+                    if (v0 < range_end) {
+                        if (v0 < shared_r16) {
+                            seq = SL.table_seq;
+                        } else {
+                            for (int m = 0; m < SL.nmem; ++m)
+                                if (v0 >= SL.mem_v[m] && v0 < SL.mem_vend[m]) {
+                                    seq = SL.mem_seq[m];
+                                    tok = SL.P + (v0 - SL.mem_v[m]);
+                                }
+                        }
+                    }
                     int v = -1;
-                    if (t0 < range_end) {
-                        int id = bt[t0 / BS];
+                    if (seq >= 0) {
+                        int id = p.block_tables[(int64_t)seq * p.max_blocks_per_seq + tok / BS];
                         if (id < 0 || id >= p.num_blocks) {
                             report(p.error_flags, PA_DEVERR_BLOCK_ID);
                             id = 0;
                         }
-                        v = id * BS + t0 % BS;
+                        v = id * BS + tok % BS;
                     }
                     win = v;
                 }
@@ -662,21 +741,18 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
         constexpr uint32_t idesc_s = instr_desc(kTok, kN, false, false);
         constexpr uint32_t idesc_pv = instr_desc(kD, 2 * kN, true, true);
         struct Pending {
-            int n, valid, item;
+            int n, item;
             bool first, last;
         };
-        Pending pend0 = {0, 0, 0, false, false};  // PVs still to issue:
+        Pending pend0 = {0, 0, false, false};     // PVs still to issue:
         Pending pend1 = pend0;                    // pend0 is the older
         int npend = 0;
         bool ok = true;
 
         auto issue_pv = [&](const Pending& pd) -> bool {
             const int vs = pd.n % kVStages;
-            const bool zero_tail = pd.valid % 16 != 0;
-            // Lanes that write into the V stage (tail rows) observe it landing.
             bool good = true;
-            if (lane == 0 || zero_tail) good = wait_bar(&v_full[vs], (pd.n / kVStages) & 1);
-            good = __all_sync(0xffffffffu, good);
+            if (lane == 0) good = wait_bar(&v_full[vs], (pd.n / kVStages) & 1);
             if (good && lane == 0) good = wait_bar(&p_full[pd.n & 1], (pd.n >> 1) & 1);
             if (good && lane == 0 && pd.first && pd.item >= 2)
                 good = wait_bar(&o_empty[pd.item & 1], ((pd.item - 2) >> 1) & 1);
@@ -684,20 +760,6 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             if (!good) {
                 if (lane == 0) set_abort(abort_flag, p.error_flags);
                 return false;
-            }
-            if (zero_tail) {
-                // The last loaded 16-token piece ends past the range: its
-                // extra token rows hold whatever the block holds.
-                unsigned char* vt = smem + kVOff + vs * kStageBytes;
-                const int rows = 16 - pd.valid % 16;
-                for (int e = lane; e < rows * 16; e += 32) {
-                    const int r = pd.valid + (e >> 4);
-                    const int h = (e >> 3) & 1;
-                    *reinterpret_cast<uint4*>(vt + h * kHalf + r * 128 + (e & 7) * 16) =
-                        make_uint4(0, 0, 0, 0);
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
             }
             tc_fence_after();
             if (lane == 0) {
@@ -732,7 +794,6 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             }
             const int nch = slots[sl].nch;
             if (nch < 0) break;
-            const int range_end = slots[sl].range_end;
             const uint32_t q_base = smem_u32(smem + kQOff + (item & 1) * kQBytes);
             for (int c = 0; c < nch; ++c, ++n) {
                 bool good = true;
@@ -772,7 +833,6 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 }
                 Pending pn;
                 pn.n = n;
-                pn.valid = min(kTok, range_end - c * kTok);
                 pn.item = item;
                 pn.first = c == 0;
                 pn.last = c == nch - 1;
@@ -801,7 +861,6 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 ItemSlot& S = slots[sl];
                 const float4 v = *reinterpret_cast<const float4*>(S.red_l[lane]);
                 const float l = (v.x + v.y) + (v.z + v.w);
-                S.l[lane] = l;
                 S.inv_l[lane] = l > 0.f ? 1.f / l : 0.f;
             }
         };
@@ -834,13 +893,6 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                     if (row[e] >= 0)
                         p.out[row[e] * kD + tid] =
                             (__uint_as_float(o[r + e]) + __uint_as_float(olo[r + e])) * inv[e];
-            }
-            if (p.shared_prefix_mode && tid < 32) {
-                const long long row = S.row[tid];
-                if (row >= 0) {
-                    p.out_m[row] = S.m[tid];
-                    p.out_l[row] = S.l[tid];
-                }
             }
             mbar_arrive_plain(&slot_free[sl]);
         };
@@ -891,9 +943,38 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                     for (int r = 0; r < 32; ++r) x[r] = __uint_as_float(raw[r]) * sl2;
                     const int tok = c * kTok + tid;
                     if (c * kTok + kTok - 1 > min_lim) {
+                        // A row sees the shared tokens of its context and
+                        // its own tail (group mode).
+                        bool seen = false;
 #pragma unroll
-                        for (int r = 0; r < 32; ++r)
-                            if (tok > S.lim[r]) x[r] = -INFINITY;
+                        for (int r = 0; r < 32; r += 4) {
+                            const int4 lm = *reinterpret_cast<const int4*>(&S.lim[r]);
+                            const int4 lo = *reinterpret_cast<const int4*>(&S.tail_lo[r]);
+                            const int4 hi = *reinterpret_cast<const int4*>(&S.tail_hi[r]);
+                            const int l4[4] = {lm.x, lm.y, lm.z, lm.w};
+                            const int o4[4] = {lo.x, lo.y, lo.z, lo.w};
+                            const int h4[4] = {hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const bool vis = tok <= l4[e] || (tok >= o4[e] && tok < h4[e]);
+                                if (!vis) x[r + e] = -INFINITY;
+                                seen = seen || vis;
+                            }
+                        }
+                        if (!seen) {
+                            // No row sees this token: its V row may hold
+                            // anything (another block's rows, unwritten
+                            // memory); P is 0 there, but 0 x NaN is NaN.
+                            const int vs = n % kVStages;
+                            if (!wait_bar(&v_full[vs], (n / kVStages) & 1)) fail = true;
+                            unsigned char* vr = smem + kVOff + vs * kStageBytes + tid * 128;
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                *reinterpret_cast<uint4*>(vr + j * 16) = make_uint4(0, 0, 0, 0);
+                                *reinterpret_cast<uint4*>(vr + kHalf + j * 16) =
+                                    make_uint4(0, 0, 0, 0);
+                            }
+                        }
                     }
                 } else {
 #pragma unroll
@@ -990,17 +1071,12 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 }
             }
             if (stop) break;
-            // Item end: per-row partial sums of this warp's 32 tokens, the reference.
+            // Item end: per-row partial sums of this warp's 32 tokens.
             {
                 float v[32];
 #pragma unroll
                 for (int r = 0; r < 32; ++r) v[r] = l_part[r];
                 S.red_l[lane][warp] = transpose_reduce<false>(v, lane);
-                float mine = 0.f;
-#pragma unroll
-                for (int r = 0; r < 32; ++r)
-                    if (r == lane) mine = m_ref[r];
-                if (warp == 0) S.m[lane] = mine;
 #pragma unroll
                 for (int r = 0; r < 32; ++r) {
                     m_ref[r] = kNoMax;

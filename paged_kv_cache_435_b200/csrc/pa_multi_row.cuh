@@ -11,13 +11,9 @@
 namespace pa {
 
 struct MultiRowParams {
-    // Multi-query mode: out fp32 [T][Hq][D], normalised.  Shared-prefix mode:
-    // out fp32 [B][Hq][D] holds each row's partial O / l over its shared
-    // tokens, out_m / out_l fp32 [B][Hq] the matching running max (log2
-    // domain, scaled) and sum.
+    // out fp32 [T][Hq][D] (multi-query mode) or [B][Hq][D] (shared-prefix
+    // mode: the rows of the members of valid groups), normalised.
     float* out;
-    float* out_m;
-    float* out_l;
     const uint16_t* q;               // bf16 [T or B][Hq][D]
     const uint16_t* k_cache;         // bf16 [NB][bs][Hkv][D]
     const uint16_t* v_cache;
@@ -25,8 +21,8 @@ struct MultiRowParams {
     const int32_t* context_lens;     // int32 [B]
     const int32_t* query_start_loc;  // int32 [B+1] (multi-query mode)
     CascadeGroups groups;            // shared-prefix mode
-    int32_t* seq_shared;             // shared-prefix mode: int32 [B], each
-                                     // sequence's shared length (written)
+    int32_t* seq_done;               // shared-prefix mode: int32 [B], written:
+                                     // 1 if this pass answers the sequence
     int* error_flags;                // nullable
     int shared_prefix_mode;
     int num_seqs;

@@ -204,3 +204,12 @@ def test_block_manager_groups_drive_the_shared_prefix_call():
     ref = oracle.paged_decode_attention(q.cpu(), bits(k), bits(v), bt, lens, 0.088, HKV)
     assert_attn_close(out, ref, "block-manager groups")
     assert (plain - out).abs().max().item() <= 2e-5
+
+
+def test_first_member_shorter_than_prefix():
+    """The group's first member ends inside the prefix (its table stops
+    there): the shared blocks are read through a member that covers them."""
+    lens = [40, 300, 256, 9, 511]
+    case = inputs.grouped_case(32, 8, 128, 16, lens, [0, 5], [256], seed=91,
+                               device="cuda")
+    check(case)
