@@ -255,6 +255,48 @@ __device__ __forceinline__ bool aborted(int* flag) {
     return *reinterpret_cast<volatile int*>(flag) != 0;
 }
 
+// One compare-exchange stage of a bitonic network over the warp's 256 keys
+// (8 per lane, element i = lane * 8 + e), sorting blocks of SIZE into
+// descending order at distance STRIDE: below 8 within a lane, else across.
+template <int SIZE, int STRIDE>
+__device__ __forceinline__ void bitonic_stage(long long (&k)[8], int lane) {
+    if (STRIDE >= 8) {
+        constexpr int kL = STRIDE >= 8 ? STRIDE / 8 : 1;
+        const bool lower = (lane & kL) == 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const bool desc = ((lane * 8 + e) & SIZE) == 0;
+            const long long other = __shfl_xor_sync(0xffffffffu, k[e], kL);
+            // the lower index keeps the larger key in a descending block
+            k[e] = (lower == desc) ? max(k[e], other) : min(k[e], other);
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            constexpr int kS = STRIDE < 8 ? STRIDE : 1;
+            if ((e ^ kS) > e) {
+                const bool desc = ((lane * 8 + e) & SIZE) == 0;
+                const long long a = k[e], b = k[e ^ kS];
+                const bool swap = desc ? a < b : a > b;
+                k[e] = swap ? b : a;
+                k[e ^ kS] = swap ? a : b;
+            }
+        }
+    }
+    if constexpr (STRIDE > 1) bitonic_stage<SIZE, STRIDE / 2>(k, lane);
+}
+
+template <int SIZE>
+__device__ __forceinline__ void bitonic_sizes(long long (&k)[8], int lane) {
+    bitonic_stage<SIZE, SIZE / 2>(k, lane);
+    if constexpr (SIZE < 256) bitonic_sizes<SIZE * 2>(k, lane);
+}
+
+// Sorts the warp's 256 keys into descending order.
+__device__ __forceinline__ void warp_sort256_desc(long long (&k)[8], int lane) {
+    bitonic_sizes<2>(k, lane);
+}
+
 // Lane r ends with the reduction over the warp of row r of v (v is consumed).
 template <bool kMax>
 __device__ __forceinline__ float transpose_reduce(float (&v)[32], int lane) {
@@ -367,8 +409,8 @@ __device__ RowItem row_item(const MultiRowParams& p, int idx, bool report_errors
 // Work of unit u (sequence or group) for the item deal: its live row tiles
 // and the weight of each of its items (128-token chunks, plus one for the
 // per-item overhead).  Invalid groups have no tiles.
-__device__ void unit_work(const MultiRowParams& p, int u, bool report_errors, int& tiles,
-                          int& w) {
+__device__ __forceinline__ void unit_work(const MultiRowParams& p, int u,
+                                          bool report_errors, int& tiles, int& w) {
     if (!p.shared_prefix_mode) {
         const int L = clamp_len(p, u, report_errors);
         const int k = clamp_queries(p, u, L, report_errors);
@@ -383,9 +425,13 @@ __device__ void unit_work(const MultiRowParams& p, int u, bool report_errors, in
         tiles = P > 0 ? (members + mpt - 1) / mpt : 0;
         long long tails = 0;
         if (P > 0)
-            for (int s = a; s < a + members; ++s) {
-                const int L = clamp_len(p, s, false);
-                tails += round16(L - min(P, L));
+            for (int s0 = a; s0 < a + members; s0 += 8) {  // 8 loads in flight
+                int Ls[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    Ls[e] = s0 + e < a + members ? clamp_len(p, s0 + e, false) : P;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) tails += round16(Ls[e] - min(P, Ls[e]));
             }
         const long long per_tile = tiles > 0 ? tails / tiles : 0;
         w = (int)((P + per_tile + kTok - 1) / kTok) + 1;
@@ -606,29 +652,94 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
         // head's total T and belongs to the CTA whose share
         // [T*j/per_head, T*(j+1)/per_head) holds that start, so every item
         // has exactly one CTA.
+        // Unit weights are gathered kUnitRounds * 32 units at a time (lane l
+        // takes units base + 32k + l) so that their loads are in flight
+        // together; with at most that many units the second pass reuses them.
         const int Hkv = p.num_kv_heads;
         const int g = blockIdx.x % Hkv;
         const int j = blockIdx.x / Hkv;
         const int per_head = gridDim.x / Hkv;
+        constexpr int kUnitRounds = 8;
+        int tl[kUnitRounds], w[kUnitRounds];
+        auto gather = [&](int base, bool report_errors) {
+#pragma unroll
+            for (int k = 0; k < kUnitRounds; ++k) {
+                const int u = base + k * 32 + lane;
+                tl[k] = 0;
+                w[k] = 0;
+                if (u < p.num_units) unit_work(p, u, report_errors, tl[k], w[k]);
+            }
+        };
         long long T = 0;
-        for (int base = 0; base < p.num_units; base += 32) {
-            const int u = base + lane;
-            int tl = 0, w = 0;
-            if (u < p.num_units) unit_work(p, u, blockIdx.x == 0, tl, w);
-            long long W = (long long)tl * w;
+        for (int base = 0; base < p.num_units; base += kUnitRounds * 32) {
+            gather(base, blockIdx.x == 0);
+            long long W = 0;
+#pragma unroll
+            for (int k = 0; k < kUnitRounds; ++k) W += (long long)tl[k] * w[k];
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
             T += W;
         }
         const long long lo = T * j / per_head;
         const long long hi = T * (j + 1) / per_head;
+        const bool kept = p.num_units <= kUnitRounds * 32;  // tl / w still hold them
         bool stopped = false;
-        long long pos = 0;  // start of the current batch of units
-        for (int base = 0; base < p.num_units && pos < hi && !stopped; base += 32) {
-            const int u = base + lane;
-            int tl = 0, w = 0;
-            if (u < p.num_units) unit_work(p, u, false, tl, w);
-            const long long W = (long long)tl * w;
+        // Longest first when every unit is one item and all fit the warp:
+        // the units sorted by weight go to the head's CTAs in snake order
+        // (0..n-1, then n-1..0, ...), pairing long items with short ones.
+        bool one_tile = true;
+#pragma unroll
+        for (int k = 0; k < kUnitRounds; ++k) one_tile = one_tile && tl[k] <= 1;
+        const bool lpt = kept && __all_sync(0xffffffffu, one_tile);
+        if (lpt) {
+            long long key[8];  // weight << 32 | (~unit): heavier first, then lower unit
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int u = lane * 8 + e;  // sort element u holds unit u
+                int tu = 0, wu = 0;
+#pragma unroll
+                for (int k = 0; k < kUnitRounds; ++k) {  // unit u sits in lane u%32, round u/32
+                    const int src_t = __shfl_sync(0xffffffffu, tl[k], u & 31);
+                    const int src_w = __shfl_sync(0xffffffffu, w[k], u & 31);
+                    if (k == (u >> 5)) {
+                        tu = src_t;
+                        wu = src_w;
+                    }
+                }
+                key[e] = (u < p.num_units && tu > 0)
+                             ? ((long long)wu << 32) | (long long)(0xFFFFFFFFu - (uint32_t)u)
+                             : -1;
+            }
+            warp_sort256_desc(key, lane);
+            int live_units = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) live_units += key[e] >= 0;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) live_units += __shfl_xor_sync(0xffffffffu, live_units, o);
+            for (int r = 0; !stopped; ++r) {
+                const int pos = r * per_head + ((r & 1) ? per_head - 1 - j : j);
+                if (pos >= live_units) break;
+                long long mine = 0;
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if (e == (pos & 7)) mine = key[e];
+                const long long kk = __shfl_sync(0xffffffffu, mine, pos >> 3);
+                const int u = (int)(0xFFFFFFFFu - (uint32_t)(kk & 0xFFFFFFFFll));
+                if (!publish((u * p.tiles) * Hkv + g)) stopped = true;
+            }
+        }
+        long long pos = 0;  // start of the current batch of 32 units
+        for (int base = 0; !lpt && base < p.num_units && pos < hi && !stopped; base += 32) {
+            const int k = (base / 32) % kUnitRounds;
+            if (!kept && k == 0) gather(base, false);
+            int tlk = 0, wk = 0;
+#pragma unroll
+            for (int e = 0; e < kUnitRounds; ++e)
+                if (e == k) {
+                    tlk = tl[e];
+                    wk = w[e];
+                }
+            const long long W = (long long)tlk * wk;
             long long incl = W;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -639,8 +750,8 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             if (pos + total > lo) {
                 for (int i = 0; i < 32 && base + i < p.num_units && !stopped; ++i) {
                     const long long us = pos + __shfl_sync(0xffffffffu, incl - W, i);
-                    const int ti = __shfl_sync(0xffffffffu, tl, i);
-                    const int wi = __shfl_sync(0xffffffffu, w, i);
+                    const int ti = __shfl_sync(0xffffffffu, tlk, i);
+                    const int wi = __shfl_sync(0xffffffffu, wk, i);
                     if (us >= hi) break;
                     if (us + (long long)ti * wi <= lo) continue;
                     for (int t = 0; t < ti && !stopped; ++t) {
