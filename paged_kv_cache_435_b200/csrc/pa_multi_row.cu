@@ -38,21 +38,24 @@
 //   warp 6     TMEM allocation and the MMA issue (one thread), S two chunks
 //              ahead of PV: S(n) needs only that the softmax has loaded
 //              S(n-2) out of its TMEM buffer, PV(n-2) that it wrote P(n-2);
-//   warp 7     scheduler: deals the items to the CTAs by work (a CTA serves
-//              one kv head; among the CTAs of a head, each takes the items
-//              whose cumulative weight starts in its share, computed
-//              identically everywhere; the heads move through the batch in
-//              step, so the head slices of a block are read together), works
-//              out its next
-//              items (token range, block-table row, each row's limit and
-//              output row) into a 4-slot shared-memory ring and copies their
-//              Q rows (cp.async), so no other warp waits on a global load at
-//              an item boundary.
+//   warp 7     scheduler: deals the items to the CTAs by work and publishes
+//              them.  A CTA serves one kv head; the CTAs of a head take the
+//              units (sequences or groups) longest first in snake order when
+//              every unit is one item (a bitonic sort across the warp), else
+//              the items whose cumulative weight starts in their share; all
+//              heads walk the batch in the same order, so the head slices of
+//              a block are read together.  For each item it works out the
+//              token range, block-table rows, each row's visible tokens and
+//              output row into a 4-slot shared-memory ring and copies the Q
+//              rows (cp.async), so no other warp waits on a global load at an
+//              item boundary.
 // Online softmax with a lazy reference: every chunk, one barrier-reduction
 // over the 4 warps (bar.red.popc) asks whether any row's logit exceeds its
 // reference max by more than 2^8; only then is the exact per-row chunk max
 // formed (warp transpose-reduction + shared memory), O^T rescaled in TMEM and
 // the reference moved.  Sums are kept per thread and reduced at item end.
+// A token no row may see (padding, past the range) has its V row zeroed by
+// its own thread once the chunk landed: P is 0 there, but 0 x NaN is NaN.
 // The producers and the MMA warp run ahead across item boundaries; the
 // epilogue of an item runs one chunk into the next item.  Every wait is
 // bounded; the softmax warps decide aborts together at their per-chunk
@@ -429,7 +432,7 @@ __device__ __forceinline__ void unit_work(const MultiRowParams& p, int u,
                 int Ls[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
-                    Ls[e] = s0 + e < a + members ? clamp_len(p, s0 + e, false) : P;
+                    Ls[e] = s0 + e < a + members ? clamp_len(p, s0 + e, report_errors) : P;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) tails += round16(Ls[e] - min(P, Ls[e]));
             }
@@ -1043,6 +1046,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 const int sb = n & 1;
                 bool ok = !fail && __all_sync(0xffffffffu, wait_bar(&s_full[sb], (n >> 1) & 1));
                 float x[32];
+                bool dead = false;  // no row sees this thread's token
                 if (ok) {
                     tc_fence_after();
                     uint32_t raw[32];
@@ -1072,20 +1076,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                                 seen = seen || vis;
                             }
                         }
-                        if (!seen) {
-                            // No row sees this token: its V row may hold
-                            // anything (another block's rows, unwritten
-                            // memory); P is 0 there, but 0 x NaN is NaN.
-                            const int vs = n % kVStages;
-                            if (!wait_bar(&v_full[vs], (n / kVStages) & 1)) fail = true;
-                            unsigned char* vr = smem + kVOff + vs * kStageBytes + tid * 128;
-#pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                *reinterpret_cast<uint4*>(vr + j * 16) = make_uint4(0, 0, 0, 0);
-                                *reinterpret_cast<uint4*>(vr + kHalf + j * 16) =
-                                    make_uint4(0, 0, 0, 0);
-                            }
-                        }
+                        dead = !seen;
                     }
                 } else {
 #pragma unroll
@@ -1169,6 +1160,20 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const uint32_t* src = j < 4 ? &hi[4 * j] : &lo[4 * (j - 4)];
                     *reinterpret_cast<uint4*>(prow + ((j ^ p_sw) << 4)) =
                         make_uint4(src[0], src[1], src[2], src[3]);
+                }
+                if (dead) {
+                    // No row sees this token: its V row may hold anything
+                    // (another block's rows, unwritten memory); P is 0 there,
+                    // but 0 x NaN is NaN.  Cleared once the V chunk landed,
+                    // as late as possible so the wait rarely blocks.
+                    const int vs = n % kVStages;
+                    if (!wait_bar(&v_full[vs], (n / kVStages) & 1)) fail = true;
+                    unsigned char* vr = smem + kVOff + vs * kStageBytes + tid * 128;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        *reinterpret_cast<uint4*>(vr + j * 16) = make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4*>(vr + kHalf + j * 16) = make_uint4(0, 0, 0, 0);
+                    }
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
