@@ -159,3 +159,12 @@ def test_mma_kernel_head128_shapes(monkeypatch, Hq, Hkv, D, bs, lens, qlens):
     case = inputs.multi_query_case(len(lens), Hq, Hkv, D, bs, lens, qlens,
                                    seed=sum(lens) + Hq + 2, device="cuda")
     check(case)
+
+
+def test_multi_row_kernel_long_context(monkeypatch):
+    """A 131072-token sequence (1024 chunks of 128 tokens, piece windows
+    walking 8192 blocks) beside short ones, 4 draft tokens each, G = 8."""
+    monkeypatch.setenv("PA_MULTI_QUERY_KERNEL", "rows")
+    case = inputs.multi_query_case(3, 16, 2, 128, 16, [131072, 300, 17],
+                                   [4, 4, 4], seed=131, device="cuda")
+    check(case)

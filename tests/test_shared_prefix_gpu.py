@@ -213,3 +213,13 @@ def test_first_member_shorter_than_prefix():
     case = inputs.grouped_case(32, 8, 128, 16, lens, [0, 5], [256], seed=91,
                                device="cuda")
     check(case)
+
+
+def test_long_prefix_and_tails():
+    """A 16384-token prefix shared by 6 samples with tails of 0..1000 tokens
+    (G = 4), and a 5000-token prefix shared by 3 samples (bs 16)."""
+    P0, P1 = 16384, 5000 // 16 * 16
+    lens = [P0 + t for t in (0, 1, 999, 1000, 517, 64)] + [P1 + t for t in (3, 700, 0)]
+    case = inputs.grouped_case(32, 8, 128, 16, lens, [0, 6, 9], [P0, P1], seed=16,
+                               device="cuda")
+    check(case)
