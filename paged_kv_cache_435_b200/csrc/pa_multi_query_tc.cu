@@ -5,21 +5,42 @@
 // High-Throughput LLM Inference", "Chunked Prefill"; causal semantics as in
 // pa_multi_query.cu).
 //
-// CTA = (kv head, 128-row tile, sequence), 6 warps:
-//   warps 0-3  softmax and epilogue; thread i owns tile row i, which is TMEM
-//              lane i, so row max / row sum need no shuffles;
-//   warp 4     producer: 64-token K/V chunks of the tile's causal range, as
-//              16-row TMA tensor tiles (128-byte swizzle), into a 2-stage ring;
-//   warp 5     allocates 256 TMEM columns and issues the MMAs (one thread).
-// Per chunk c: S(c) = Q K(c)^T (M=128, N=64, K=128: 8 tcgen05.mma, both
-// operands in shared memory) lands in TMEM buffer c%2; the softmax warps read
-// their rows, write P = bf16(p) and its bf16 residual back into the same
-// buffer, and O += P V(c) runs as 2 x 4 tcgen05.mma with A read from TMEM
-// (M=128, N=128, K=16 each).  S(c+1) is issued before PV(c), so the tensor
-// core computes the next logits while the softmax warps work.  O stays in
-// TMEM (128 columns); it is rescaled only when a row's running max grows by
-// more than 2^8 (the sum and O share the stale reference, so the final O/l is
-// exact).  All waits are bounded; TMEM is released on every exit path.
+// CTA = (kv head, 128-row tile, sequence), one per SM, 12 warps:
+//   warps 0-7  softmax and epilogue in two warpgroups: warp w owns tile rows
+//              32(w%4).. (its TMEM lane quarter); warpgroup 0 takes tokens
+//              0-63 of each 128-token chunk and d 0-63 of the output,
+//              warpgroup 1 tokens 64-127 and d 64-127.  Warps w and w+4 share
+//              rows and agree per chunk through one named barrier (bar.red);
+//   warps 8,10 producers of the K and the V stream: the tile's causal range
+//              in 128-token chunks of 16-row TMA tensor tiles (128-byte
+//              swizzle), one issuing thread per stream, 3- and 4-stage rings;
+//   warp 9     allocates all 512 TMEM columns and issues the S MMAs,
+//   warp 11    issues the PV MMAs (one thread each, descriptors built once).
+//              The tensor pipe queues few MMAs, so a single issuing thread
+//              left it idle during its waits between batches; with two, one
+//              issues while the other waits.
+// The 32 row tiles of a (sequence, kv head) read the same K and V, so the
+// copies keep the default L2 priority (the decode stream's evict-first
+// hint would send every tile back to DRAM).
+//
+// TMEM: S0 | S1 | O | Q (128, 128, 128, 64 columns).  Per chunk c:
+// S(c) = Q K(c)^T (M=128, N=128, K=128: 8 tcgen05.mma, Q read from TMEM so
+// that only K crosses shared memory) lands in buffer c%2; each warpgroup
+// reads its 64 columns and writes P = bf16(p) and its bf16 residual back
+// into them, and O += P V(c) runs as 2 x 8 tcgen05.mma with A read from
+// TMEM (M=128, N=128, K=16 each).  S(c+1) is issued before PV(c), so the
+// tensor core computes the next logits while the softmax warps work; S(c+2)
+// waits until PV(c) has read the P it overwrites.
+//
+// Softmax reference.  The row max is taken exactly on the first chunk only;
+// later chunks exponentiate against that reference and check the chunk's
+// sum instead of taking a max: a sum above 2^16 (or not finite) means the
+// row's max has grown, and only then are the logits (still in TMEM) read
+// again, the exact max taken, O and the running sum rescaled and the chunk
+// exponentiated afresh.  The sum and O share the reference, so the final
+// O / l is exact; p <= 2^16 keeps the fp32 accumulator far from overflow.
+// All waits are bounded, and the two warps of a row pair take every
+// abort decision together; TMEM is released on every exit path.
 #include <cuda.h>
 
 #include <cstdint>
@@ -32,24 +53,37 @@ namespace pa {
 namespace {
 
 constexpr int kRows = 128;        // M: tile rows
-constexpr int kTok = 64;          // tokens per chunk (N of S, K of PV)
+constexpr int kTok = 128;         // tokens per chunk (N of S, K of PV)
 constexpr int kD = 128;           // head size handled by this kernel
-constexpr int kStages = 2;
-constexpr int kThreads = 192;
-constexpr int kQHalf = kRows * 128;                 // 16 KB: 128 rows x 64 d
-constexpr int kKVHalf = kTok * 128;                 // 8 KB: 64 tokens x 64 d
-constexpr int kStageBytes = 4 * kKVHalf;            // K lo/hi, V lo/hi
-constexpr int kQOff = 0;
-constexpr int kRingOff = 2 * kQHalf;                // 32 KB
-constexpr int kBarOff = kRingOff + kStages * kStageBytes;
-// barriers: k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2],
-//           p_full[2], pv_done, o_final, q_ready, then the TMEM base address
-//           and the abort flag.  K and V travel in separate rings: K(c) is
-//           free as soon as S(c) is done, long before PV(c).
-constexpr int kNumBars = 15;
+constexpr int kKStages = 3;
+constexpr int kVStages = 4;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kThreads = (kSoftmaxWarps + 4) * 32;  // + K, S, V, PV warps
+constexpr int kWarpK = kSoftmaxWarps;
+constexpr int kWarpMma = kSoftmaxWarps + 1;         // TMEM owner, S MMAs
+constexpr int kWarpV = kSoftmaxWarps + 2;
+constexpr int kWarpPv = kSoftmaxWarps + 3;
+constexpr int kPiecesPerChunk = kTok / 16;          // 16-token TMA tiles
+constexpr int kKVHalf = kTok * 128;                 // 16 KB: 128 tokens x 64 d
+constexpr int kStageBytes = 2 * kKVHalf;            // one chunk of K or of V
+constexpr int kKOff = 0;
+constexpr int kVOff = kKOff + kKStages * kStageBytes;
+constexpr int kXOff = kVOff + kVStages * kStageBytes;  // float [2][2][128]
+constexpr int kBarOff = kXOff + 2 * 2 * kRows * 4;
+// barriers: k_full[3], k_empty[3], v_full[4], v_empty[4], s_full[2],
+//           p_full[2], pv_done[2] (per S buffer), o_final, q_ready, s_drain,
+//           then the TMEM base address and the abort flag.  K and V travel
+//           in separate rings: K(c) is free as soon as S(c) is done, long
+//           before PV(c).
+constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 9;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16;
-constexpr uint32_t kTmemCols = 256;                 // S0 | S1 | O
-constexpr float kRescaleThreshold = 8.f;            // log2 units
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+// Descriptor start addresses are 14-bit fields of (address >> 4).
+static_assert(kSmemBytes + 1024 <= (1 << 18), "descriptor address range");
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemO = 2 * kTok;
+constexpr uint32_t kTmemQ = kTmemO + kD;
+constexpr float kSumLimit = 65536.f;                // 2^16: see the header
 
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity) {
     return mbar_wait_bounded(bar, parity);
@@ -78,17 +112,6 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo,
 __host__ __device__ constexpr uint32_t instr_desc(int M, int N, bool b_mn_major) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc,
-                                       uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
-        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate),
-        "r"(0u), "r"(0u), "r"(0u), "r"(0u));
 }
 
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem,
@@ -155,6 +178,22 @@ __device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* map,
         : "memory");
 }
 
+// 2^x by the PTX ex2.approx.ftz.f32 instruction (one MUFU operation):
+// relative error about 2^-22, 2^-inf = 0, results below 2^-126 flush to 0
+// (a term that small against the row's reference is invisible in fp32).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// L2 policy with the default (normal) eviction priority.
+__device__ __forceinline__ uint64_t l2_policy_normal() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
 __device__ __forceinline__ void mbar_arrive_plain(uint64_t* bar) {
     asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
                  : "memory");
@@ -167,24 +206,46 @@ __device__ __forceinline__ bool aborted(int* flag) {
     return *reinterpret_cast<volatile int*>(flag) != 0;
 }
 
+// Named barrier over the two warps (w, w + 4) that share tile rows, with an
+// OR of their predicates.
+__device__ __forceinline__ bool pair_any(int id, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.or.pred po, %2, 64, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"(pred ? 1u : 0u), "r"(id)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void pair_sync(int id) {
+    asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
+}
+
 template <int BS>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
 paged_multi_query_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v,
                             const MultiQueryParams p) {
     extern __shared__ __align__(1024) unsigned char smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
-    uint64_t* k_full = bars + 0;
-    uint64_t* k_empty = bars + 2;
-    uint64_t* v_full = bars + 4;
-    uint64_t* v_empty = bars + 6;
-    uint64_t* s_full = bars + 8;
-    uint64_t* p_full = bars + 10;
-    uint64_t* pv_done = bars + 12;
-    uint64_t* o_final = bars + 13;
-    uint64_t* q_ready = bars + 14;
+    uint64_t* k_full = bars;
+    uint64_t* k_empty = k_full + kKStages;
+    uint64_t* v_full = k_empty + kKStages;
+    uint64_t* v_empty = v_full + kVStages;
+    uint64_t* s_full = v_empty + kVStages;
+    uint64_t* p_full = s_full + 2;
+    uint64_t* pv_done = p_full + 2;
+    uint64_t* o_final = pv_done + 2;
+    uint64_t* q_ready = o_final + 1;
+    uint64_t* s_drain = q_ready + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
     int* abort_flag = reinterpret_cast<int*>(smem + kBarOff + kNumBars * 8 + 4);
+    // Per-row exchange between the two warpgroups: [0] maxima, [1] sums.
+    float (*xchg)[2][kRows] = reinterpret_cast<float (*)[2][kRows]>(smem + kXOff);
 
     const int g = blockIdx.x;
     const int rt = blockIdx.y;
@@ -221,21 +282,26 @@ paged_multi_query_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
     const int nch = (range_end + kTok - 1) / kTok;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kKStages; ++i) {
             mbar_init(&k_full[i], 1);
             mbar_init(&k_empty[i], 1);
+        }
+        for (int i = 0; i < kVStages; ++i) {
             mbar_init(&v_full[i], 1);
             mbar_init(&v_empty[i], 1);
-            mbar_init(&s_full[i], 1);
-            mbar_init(&p_full[i], 128);
         }
-        mbar_init(pv_done, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&p_full[i], kSoftmaxWarps * 32);
+            mbar_init(&pv_done[i], 1);
+        }
         mbar_init(o_final, 1);
-        mbar_init(q_ready, 128);
+        mbar_init(q_ready, kSoftmaxWarps * 32);
+        mbar_init(s_drain, 1);
         *abort_flag = 0;
         mbar_init_fence();
     }
-    if (warp == 5) {
+    if (warp == kWarpMma) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols)
                      : "memory");
@@ -245,24 +311,37 @@ paged_multi_query_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tmem_o = tmem + 2 * kTok;          // columns [128, 256)
+    const uint32_t tmem_o = tmem + kTmemO;
+    const uint32_t tmem_q = tmem + kTmemQ;
 
-    const uint64_t pol = l2_policy_evict_first();
-
-    if (warp == 4) {
-        // ---------------------------------------------------------- producer
-        // Order: K(0), K(1), V(0), K(2), V(1), ...: V runs one chunk behind
-        // K, so a K stage is refilled as soon as S has read it.
+    if (warp == kWarpK || warp == kWarpV) {
+        // --------------------------------------------------------- producers
+        const int which = warp == kWarpV;               // 0: K, 1: V
+        const int S = which ? kVStages : kKStages;
+        uint64_t* fulls = which ? v_full : k_full;
+        uint64_t* empties = which ? v_empty : k_empty;
+        const int ring_off = which ? kVOff : kKOff;
+        const uint64_t pol = l2_policy_normal();
         const int32_t* bt = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
-        // Per stream (K, V): lane l holds the slot of 16-token piece l of
-        // chunks base..base+7 (V runs one chunk behind K, so each stream
-        // keeps its own window).
-        int piece_slot[2] = {-1, -1};
-        int slot_base[2] = {-8, -8};
-        auto slots_of = [&](int c, int which, int (&sl)[4]) {
-            if (c >= slot_base[which] + 8) {
-                slot_base[which] = c & ~7;
-                const int t0 = slot_base[which] * kTok + lane * 16;
+        // Lane l holds the slot of 16-token piece l of chunks base..base+3.
+        constexpr int kWindow = 32 / kPiecesPerChunk;   // chunks per window
+        int piece_slot = -1;
+        int slot_base = -kWindow;
+        int issued = 0;
+        for (int c = 0; c < nch; ++c, ++issued) {
+            const int st = c % S;
+            if (c >= S) {
+                bool ok = true;
+                if (lane == 0) ok = wait_bar(&empties[st], (c / S - 1) & 1);
+                if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) {
+                    if (lane == 0) set_abort(abort_flag, p.error_flags);
+                    break;
+                }
+            }
+            if (aborted(abort_flag)) break;
+            if (c >= slot_base + kWindow) {
+                slot_base = c - c % kWindow;
+                const int t0 = slot_base * kTok + lane * 16;
                 int v = -1;
                 if (t0 < range_end) {
                     int id = bt[t0 / BS];
@@ -272,92 +351,102 @@ paged_multi_query_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                     }
                     v = id * BS + t0 % BS;
                 }
-                piece_slot[which] = v;
+                piece_slot = v;
             }
-            const int mine = piece_slot[which];
+            int sl[kPiecesPerChunk];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                sl[i] = __shfl_sync(0xffffffffu, mine, (c - slot_base[which]) * 4 + i);
-        };
-        // Issue K (which = 0) or V (which = 1) of chunk c; false on abort.
-        auto load = [&](int c, int which) -> bool {
-            const int st = c & 1;
-            uint64_t* full = which ? &v_full[st] : &k_full[st];
-            uint64_t* empty = which ? &v_empty[st] : &k_empty[st];
-            if (c >= kStages) {
-                bool ok = true;
-                if (lane == 0) ok = wait_bar(empty, ((c >> 1) - 1) & 1);
-                if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) {
-                    if (lane == 0) set_abort(abort_flag, p.error_flags);
-                    return false;
-                }
-            }
-            if (aborted(abort_flag)) return false;
-            int sl[4];
-            slots_of(c, which, sl);
+            for (int i = 0; i < kPiecesPerChunk; ++i)
+                sl[i] = __shfl_sync(0xffffffffu, piece_slot,
+                                    (c - slot_base) * kPiecesPerChunk + i);
             if (lane == 0) {
                 int pieces = 0;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) pieces += sl[i] >= 0;
-                const uint32_t base = smem_u32(smem + kRingOff + st * kStageBytes +
-                                               which * 2 * kKVHalf);
-                mbar_arrive_expect_tx(full, pieces * 2 * 2048);
+                for (int i = 0; i < kPiecesPerChunk; ++i) pieces += sl[i] >= 0;
+                const uint32_t base = smem_u32(smem + ring_off + st * kStageBytes);
+                mbar_arrive_expect_tx(&fulls[st], pieces * 2 * 2048);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
+                for (int i = 0; i < kPiecesPerChunk; ++i) {
                     if (sl[i] < 0) continue;
 #pragma unroll
                     for (int h = 0; h < 2; ++h)
                         tma_load(base + h * kKVHalf + i * 2048, which ? &tm_v : &tm_k,
-                                 g * 2 + h, sl[i], full, pol);
+                                 g * 2 + h, sl[i], &fulls[st], pol);
                 }
             }
             __syncwarp();
-            return true;
-        };
-        int k_issued = 0, v_issued = 0;
-        for (int c = 0; c <= nch; ++c) {
-            if (c < nch) {
-                if (!load(c, 0)) break;
-                ++k_issued;
-            }
-            if (c >= 1) {
-                if (!load(c - 1, 1)) break;
-                ++v_issued;
-            }
         }
         // Wait for the copies still in flight before the CTA may exit.
-        if (lane == 0) {
-            for (int c = (k_issued > kStages ? k_issued - kStages : 0); c < k_issued; ++c)
-                (void)wait_bar(&k_full[c & 1], (c >> 1) & 1);
-            for (int c = (v_issued > kStages ? v_issued - kStages : 0); c < v_issued; ++c)
-                (void)wait_bar(&v_full[c & 1], (c >> 1) & 1);
-        }
-    } else if (warp == 5) {
-        // --------------------------------------------------------- MMA issuer
+        if (lane == 0)
+            for (int c = (issued > S ? issued - S : 0); c < issued; ++c)
+                (void)wait_bar(&fulls[c % S], (c / S) & 1);
+    } else if (warp == kWarpMma) {
+        // ------------------------------------------------------ S MMA issuer
         constexpr uint32_t idesc_s = instr_desc(kRows, kTok, false);
-        constexpr uint32_t idesc_pv = instr_desc(kRows, kD, true);
-        const uint32_t q_base = smem_u32(smem + kQOff);
+        // K: K-major, its two 64-wide swizzle columns kKVHalf apart, 8-token
+        // groups 1 KB apart; a 16-wide d slice starts 32 B into the 128-byte
+        // row.  Each MMA adds a compile-time offset (16-byte units) to the
+        // start-address field.
+        const uint64_t k_desc0 = smem_desc(smem_u32(smem + kKOff), 16, 1024);
         bool ok = true;
         if (lane == 0) ok = wait_bar(q_ready, 0);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok && lane == 0) set_abort(abort_flag, p.error_flags);
-        int issued_pv = 0;
-        auto issue_pv = [&](int c) -> bool {
+        for (int c = 0; c < nch && ok; ++c) {
+            const int ks_stage = c % kKStages;
+            const int st = c & 1;
+            bool good = true;
+            if (lane == 0) {
+                good = wait_bar(&k_full[ks_stage], (c / kKStages) & 1);
+                // Buffer st holds P(c-2) until PV(c-2) has read it.
+                if (good && c >= 2) good = wait_bar(&pv_done[st], ((c - 2) >> 1) & 1);
+            }
+            good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+            if (!good || aborted(abort_flag)) {
+                if (lane == 0) set_abort(abort_flag, p.error_flags);
+                break;
+            }
+            tc_fence_after();
+            if (lane == 0) {
+                const uint64_t kd = k_desc0 + (uint64_t)((ks_stage * kStageBytes) >> 4);
+#pragma unroll
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    const uint32_t k_off = ((ks >> 2) * kKVHalf + (ks & 3) * 32) >> 4;
+                    mma_ts(tmem + st * kTok, tmem_q + ks * 8, kd + k_off, idesc_s,
+                           ks > 0 ? 1u : 0u);
+                }
+                mma_commit(&s_full[st]);
+                mma_commit(&k_empty[ks_stage]);
+            }
+            __syncwarp();
+        }
+        if (lane == 0) {
+            mma_commit(s_drain);                 // this thread's MMAs retired
+            (void)wait_bar(s_drain, 0);          // before TMEM goes away
+        }
+        __syncwarp();
+    } else if (warp == kWarpPv) {
+        // ----------------------------------------------------- PV MMA issuer
+        constexpr uint32_t idesc_pv = instr_desc(kRows, kD, true);
+        // V: MN-major, its two 64-wide d columns kKVHalf apart (LBO), 8-token
+        // groups 1 KB apart (SBO).
+        const uint64_t v_desc0 = smem_desc(smem_u32(smem + kVOff), kKVHalf, 1024);
+        for (int c = 0; c < nch; ++c) {
+            const int vs = c % kVStages;
             const int st = c & 1;
             // Every lane observes V(c) landing (the tail chunk's lanes write
             // into this stage below).
-            bool good = __all_sync(0xffffffffu, wait_bar(&v_full[st], (c >> 1) & 1));
+            bool good = __all_sync(0xffffffffu, wait_bar(&v_full[vs], (c / kVStages) & 1));
             if (good && lane == 0) good = wait_bar(&p_full[st], (c >> 1) & 1);
             good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
-            if (!good) {
+            if (!good || aborted(abort_flag)) {
                 if (lane == 0) set_abort(abort_flag, p.error_flags);
-                return false;
+                break;
             }
             const int valid = min(kTok, range_end - c * kTok);
             if (valid < kTok) {
                 // Rows past the range hold stale or unwritten data: zero the
                 // V rows (P is 0 there, but 0 x NaN is NaN).
-                unsigned char* vrow = smem + kRingOff + st * kStageBytes + 2 * kKVHalf;
+                unsigned char* vrow = smem + kVOff + vs * kStageBytes;
                 const int rows = kTok - valid;
                 for (int e = lane; e < rows * 2 * 8; e += 32) {
                     const int r = valid + e / 16;
@@ -370,182 +459,192 @@ paged_multi_query_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
             }
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t v_base = smem_u32(smem + kRingOff + st * kStageBytes + 2 * kKVHalf);
-                const uint32_t p_hi = tmem + st * kTok;
-                const uint32_t p_lo = p_hi + kTok / 2;
+                const uint64_t vd = v_desc0 + (uint64_t)((vs * kStageBytes) >> 4);
+                // P of tokens 16kt..16kt+15: warpgroup kt/4's 64 columns,
+                // bf16 pairs at 8(kt%4), residuals 32 columns further.
+                const uint32_t pb = tmem + st * kTok;
 #pragma unroll
-                for (int kt = 0; kt < kTok / 16; ++kt) {
-                    // V rows 16kt..16kt+15 (two 8-row groups), MN-major:
-                    // LBO = the 8 KB between the two 64-column halves.
-                    const uint64_t vd = smem_desc(v_base + kt * 2048, kKVHalf, 1024);
-                    mma_ts(tmem_o, p_hi + kt * 8, vd, idesc_pv, (c > 0 || kt > 0) ? 1u : 0u);
-                }
+                for (int kt = 0; kt < kTok / 16; ++kt)
+                    mma_ts(tmem_o, pb + 64 * (kt >> 2) + 8 * (kt & 3),
+                           vd + (uint64_t)((kt * 2048) >> 4), idesc_pv,
+                           (c > 0 || kt > 0) ? 1u : 0u);
 #pragma unroll
-                for (int kt = 0; kt < kTok / 16; ++kt) {
-                    const uint64_t vd = smem_desc(v_base + kt * 2048, kKVHalf, 1024);
-                    mma_ts(tmem_o, p_lo + kt * 8, vd, idesc_pv, 1u);
-                }
-                mma_commit(&v_empty[st]);
-                mma_commit(pv_done);
+                for (int kt = 0; kt < kTok / 16; ++kt)
+                    mma_ts(tmem_o, pb + 64 * (kt >> 2) + 32 + 8 * (kt & 3),
+                           vd + (uint64_t)((kt * 2048) >> 4), idesc_pv, 1u);
+                mma_commit(&v_empty[vs]);
+                mma_commit(&pv_done[st]);
             }
             __syncwarp();
-            ++issued_pv;
-            return true;
-        };
-        for (int c = 0; c < nch && ok; ++c) {
-            const int st = c & 1;
-            bool good = true;
-            if (lane == 0) good = wait_bar(&k_full[st], (c >> 1) & 1);
-            good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
-            if (!good || aborted(abort_flag)) {
-                if (lane == 0) set_abort(abort_flag, p.error_flags);
-                break;
-            }
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t k_base = smem_u32(smem + kRingOff + st * kStageBytes);
-#pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks) {
-                    const uint32_t off = (ks & 3) * 32;  // K=16 slice in the atom
-                    const uint64_t qd = smem_desc(q_base + (ks >> 2) * kQHalf + off, 16, 1024);
-                    const uint64_t kd = smem_desc(k_base + (ks >> 2) * kKVHalf + off, 16, 1024);
-                    mma_ss(tmem + st * kTok, qd, kd, idesc_s, ks > 0 ? 1u : 0u);
-                }
-                mma_commit(&s_full[st]);
-                mma_commit(&k_empty[st]);
-            }
-            __syncwarp();
-            if (c >= 1 && !issue_pv(c - 1)) break;
         }
-        if (!aborted(abort_flag) && issued_pv == nch - 1 && nch >= 1) issue_pv(nch - 1);
         if (lane == 0) {
-            mma_commit(o_final);                 // everything issued so far
+            mma_commit(o_final);                 // every PV issued so far
             (void)wait_bar(o_final, 0);          // drained before TMEM goes away
         }
         __syncwarp();
     } else {
         // ------------------------------------------------ softmax, epilogue
-        const int r = warp * 32 + lane;          // tile row == TMEM lane
+        const int wg = warp >> 2;                // token half and d half
+        const int qw = warp & 3;                 // TMEM lane quarter
+        const int pair = 1 + qw;                 // named barrier of (w, w+4)
+        const int r = qw * 32 + lane;            // tile row == TMEM lane
         const int R = row0 + r;
         const bool live = R < rows_total;
         const int j = live ? R / G : 0;
         const int gi = live ? R % G : 0;
         const int lim = live ? L - k + j : range_end - 1;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t lane_off = (uint32_t)(qw * 32) << 16;
+        const int col0 = 64 * wg;
 
-        // Q row -> shared memory in the K-major 128-byte-swizzled layout.
+        // This row's half of Q -> TMEM (the S MMA's A operand): column c
+        // holds the bf16 pair (2c, 2c+1), the order of the words in memory.
         {
             const uint4* src = reinterpret_cast<const uint4*>(
-                p.q + ((int64_t)(q0 + j) * Hq + g * G + gi) * kD);
+                p.q + ((int64_t)(q0 + j) * Hq + g * G + gi) * kD + col0);
+            uint32_t w[32];
 #pragma unroll
-            for (int c16 = 0; c16 < 16; ++c16) {
+            for (int c16 = 0; c16 < 8; ++c16) {
                 const uint4 v = live ? src[c16] : make_uint4(0, 0, 0, 0);
-                const int h = c16 >> 3, cc = c16 & 7;
-                *reinterpret_cast<uint4*>(smem + kQOff + h * kQHalf + r * 128 +
-                                          ((cc ^ (r & 7)) << 4)) = v;
+                w[4 * c16] = v.x;
+                w[4 * c16 + 1] = v.y;
+                w[4 * c16 + 2] = v.z;
+                w[4 * c16 + 3] = v.w;
             }
-            fence_proxy_async_smem();
+            tmem_st32(tmem_q + lane_off + 32 * wg, w);
+            tmem_wait_st();
+            tc_fence_before();
             mbar_arrive_plain(q_ready);
         }
 
         const float sl2 = p.scale_log2;
-        float m_ref = -INFINITY;
-        float l_sum = 0.f;
+        float m_ref = 0.f;
+        float l_part = 0.f;
         bool ok = true;
-        for (int c = 0; c < nch; ++c) {
-            const int st = c & 1;
-            ok = wait_bar(&s_full[st], (c >> 1) & 1);
-            if (!__all_sync(0xffffffffu, ok) || aborted(abort_flag)) {
-                if (lane == 0) set_abort(abort_flag, p.error_flags);
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            uint32_t sraw[2][32];
-            tmem_ld32(tmem + lane_off + st * kTok, sraw[0]);
-            tmem_ld32(tmem + lane_off + st * kTok + 32, sraw[1]);
+        // Raw logits of this warpgroup's 64 tokens of chunk c from TMEM,
+        // tokens past the row's causal limit set to -inf.  The scale (log2
+        // domain) folds into one FFMA per exponent; maxima are taken on raw
+        // values and scaled (scale > 0 preserves order).
+        auto load_logits = [&](uint32_t sbase, int ctok, float (&sv)[64]) {
+            uint32_t r0[32], r1[32];
+            tmem_ld32(sbase, r0);
+            tmem_ld32(sbase + 32, r1);
             tmem_wait_ld();
-            // Raw logits; the scale (log2 domain) folds into one FFMA per
-            // exponent below, and the row max is taken on raw values
-            // (scale > 0 preserves order).
-            float sv[64];
-            const int ctok = c * kTok;
 #pragma unroll
-            for (int i = 0; i < 64; ++i) sv[i] = __uint_as_float(sraw[i >> 5][i & 31]);
-            if (ctok + kTok - 1 > min_lim) {
+            for (int i = 0; i < 32; ++i) {
+                sv[i] = __uint_as_float(r0[i]);
+                sv[32 + i] = __uint_as_float(r1[i]);
+            }
+            if (ctok + 63 > min_lim) {
 #pragma unroll
                 for (int i = 0; i < 64; ++i)
                     if (ctok + i > lim) sv[i] = -INFINITY;
             }
+        };
+        auto half_max = [&](const float (&sv)[64]) -> float {
             float mx8[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) mx8[i] = sv[i];
 #pragma unroll
             for (int i = 8; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
-            const float mx = sl2 * fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-            if (c == 0) {
-                m_ref = mx;
-            } else if (__any_sync(0xffffffffu, mx > m_ref + kRescaleThreshold)) {
-                // O must be stable: the previous chunk's PV has to be done.
-                const bool okw = wait_bar(pv_done, (c - 1) & 1);
-                if (!__all_sync(0xffffffffu, okw)) {
-                    if (lane == 0) set_abort(abort_flag, p.error_flags);
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const float m_new = fmaxf(m_ref, mx);
-                const float alpha = exp2f(m_ref - m_new);
-                m_ref = m_new;
-                l_sum *= alpha;
-#pragma unroll
-                for (int part = 0; part < kD / 32; ++part) {
-                    uint32_t o[32];
-                    tmem_ld32(tmem_o + lane_off + part * 32, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    tmem_st32(tmem_o + lane_off + part * 32, o);
-                }
-                tmem_wait_st();
-            }
-            // p = 2^(scale*s - m) (masked logits give 2^-inf = 0) and its bf16
-            // split by truncation: the high half keeps 8 significant bits, the
-            // residual another 8, so P carries ~16 bits into PV.
-            uint32_t hi[32], lo[32];
+            return sl2 * fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        };
+        // In place: sv <- 2^(scale*s - m_ref) (masked logits give 0); the sum.
+        auto exponentiate = [&](float (&sv)[64]) -> float {
             float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             const float neg_m = -m_ref;
 #pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                sv[i] = ex2_approx(fmaf(sv[i], sl2, neg_m));
+                ps8[i & 7] += sv[i];
+            }
+            return ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) +
+                   ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
+        };
+        for (int c = 0; c < nch; ++c) {
+            const int st = c & 1;
+            const bool got = wait_bar(&s_full[st], (c >> 1) & 1);
+            if (pair_any(pair, !got || aborted(abort_flag))) {
+                if (lane == 0) set_abort(abort_flag, p.error_flags);
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t sbase = tmem + lane_off + st * kTok + col0;
+            const int ctok = c * kTok + col0;
+            float sv[64];
+            load_logits(sbase, ctok, sv);
+            if (c == 0) {                        // token 0 is visible to every row
+                xchg[0][wg][r] = half_max(sv);
+                pair_sync(pair);
+                m_ref = fmaxf(xchg[0][0][r], xchg[0][1][r]);
+            }
+            float psum = exponentiate(sv);
+            if (pair_any(pair, !(psum <= kSumLimit))) {
+                // A row's max grew: exact max from the logits still in TMEM,
+                // O and the sums rescaled once the previous PV is done.
+                load_logits(sbase, ctok, sv);
+                xchg[0][wg][r] = half_max(sv);
+                pair_sync(pair);
+                const float m_new = fmaxf(m_ref, fmaxf(xchg[0][0][r], xchg[0][1][r]));
+                if (c > 0) {
+                    const bool okw = wait_bar(&pv_done[(c - 1) & 1], ((c - 1) >> 1) & 1);
+                    if (pair_any(pair, !okw)) {
+                        if (lane == 0) set_abort(abort_flag, p.error_flags);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const float alpha = exp2f(m_ref - m_new);
+                    l_part *= alpha;
+#pragma unroll
+                    for (int part = 0; part < 2; ++part) {
+                        uint32_t o[32];
+                        tmem_ld32(tmem_o + lane_off + col0 + part * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st32(tmem_o + lane_off + col0 + part * 32, o);
+                    }
+                    tmem_wait_st();
+                }
+                m_ref = m_new;
+                psum = exponentiate(sv);
+            }
+            l_part += psum;
+            // bf16 split of p by truncation: the high half keeps 8
+            // significant bits, the residual another 8, so P carries ~16
+            // bits into PV.  Pairs of tokens in the warpgroup's first 32
+            // columns, the residuals in the next 32.
+            uint32_t hi[32], lo[32];
+#pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float a = exp2f(fmaf(sv[2 * i], sl2, neg_m));
-                const float b = exp2f(fmaf(sv[2 * i + 1], sl2, neg_m));
-                ps8[i & 7] += a + b;
+                const float a = sv[2 * i], b = sv[2 * i + 1];
                 const uint32_t ab = __float_as_uint(a), bb = __float_as_uint(b);
                 const float al = a - __uint_as_float(ab & 0xFFFF0000u);
                 const float bl = b - __uint_as_float(bb & 0xFFFF0000u);
                 hi[i] = __byte_perm(ab, bb, 0x7632);
                 lo[i] = __byte_perm(__float_as_uint(al), __float_as_uint(bl), 0x7632);
             }
-            l_sum += ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) +
-                     ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
-            tmem_st32(tmem + lane_off + st * kTok, hi);
-            tmem_st32(tmem + lane_off + st * kTok + 32, lo);
+            tmem_st32(sbase, hi);
+            tmem_st32(sbase + 32, lo);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive_plain(&p_full[st]);
         }
         if (ok) {
+            xchg[1][wg][r] = l_part;
             const bool okw = wait_bar(o_final, 0);
-            if (__all_sync(0xffffffffu, okw)) {
+            // Also orders the partner's sum before the read below.
+            if (!pair_any(pair, !okw)) {
                 tc_fence_after();
-                float* dst = p.out + ((int64_t)(q0 + j) * Hq + g * G + gi) * kD;
-                const float inv = 1.f / l_sum;
+                float* dst = p.out + ((int64_t)(q0 + j) * Hq + g * G + gi) * kD + col0;
+                const float inv = 1.f / (xchg[1][0][r] + xchg[1][1][r]);
 #pragma unroll
-                for (int part = 0; part < kD / 32; ++part) {
+                for (int part = 0; part < 2; ++part) {
                     uint32_t o[32];
-                    tmem_ld32(tmem_o + lane_off + part * 32, o);
+                    tmem_ld32(tmem_o + lane_off + col0 + part * 32, o);
                     tmem_wait_ld();
                     if (live) {
 #pragma unroll
@@ -564,7 +663,7 @@ paged_multi_query_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 5)
+    if (warp == kWarpMma)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
                      ::"r"(tmem), "r"(kTmemCols)
                      : "memory");
