@@ -126,6 +126,9 @@ static_assert(kStageBytes % 1024 == 0 && kQBytes % 1024 == 0 && kPBytes % 1024 =
               "swizzled tiles need 1024-byte alignment");
 static_assert(kSlotOff % 16 == 0 && kBarOff % 8 == 0, "alignment");
 static_assert(kSmemBytes <= 232448, "shared memory");
+// Descriptor start addresses are 14-bit fields of (address >> 4); offsets
+// are added to a base descriptor without a carry out of that field.
+static_assert(kSmemBytes + 1024 <= (1 << 18), "descriptor address range");
 
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity) {
     return mbar_wait_bounded(bar, parity);
@@ -854,6 +857,16 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
         // -------------------------------------------------------- MMA issuer
         constexpr uint32_t idesc_s = instr_desc(kTok, kN, false, false);
         constexpr uint32_t idesc_pv = instr_desc(kD, 2 * kN, true, true);
+        // Base descriptors, built once; each MMA adds its offset in 16-byte
+        // units (stage, buffer and K slice) to the start-address field.
+        // V^T: MN-major, M = d in two 64-wide swizzle columns 16 KB apart
+        // (LBO), 8-token groups 1 KB apart (SBO).  [P_hi^T | P_lo^T]:
+        // MN-major, N = 64 = one swizzle column.  K and Q: K-major, 8-row
+        // groups 1 KB apart; a 16-wide d slice starts 32 B into the row.
+        const uint64_t v_desc0 = smem_desc(smem_u32(smem + kVOff), kHalf, 1024);
+        const uint64_t p_desc0 = smem_desc(smem_u32(smem + kPOff), kPBytes, 1024);
+        const uint64_t k_desc0 = smem_desc(smem_u32(smem + kKOff), 16, 1024);
+        const uint64_t q_desc0 = smem_desc(smem_u32(smem + kQOff), 16, 1024);
         struct Pending {
             int n, item;
             bool first, last;
@@ -877,18 +890,14 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             }
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t v_base = smem_u32(smem + kVOff + vs * kStageBytes);
-                const uint32_t p_base = smem_u32(smem + kPOff + (pd.n & 1) * kPBytes);
+                const uint64_t vd = v_desc0 + (uint64_t)((vs * kStageBytes) >> 4);
+                const uint64_t pdesc = p_desc0 + (uint64_t)(((pd.n & 1) * kPBytes) >> 4);
                 const uint32_t d_tmem = tmem + kTmemO + (pd.item & 1) * 2 * kN;
 #pragma unroll
-                for (int kt = 0; kt < kTok / 16; ++kt) {
-                    // V^T: MN-major, M = d in two 64-wide swizzle columns
-                    // 16 KB apart (LBO), 8-token groups 1 KB apart (SBO).
-                    // [P_hi^T | P_lo^T]: MN-major, N = 64 = one swizzle column.
-                    const uint64_t ad = smem_desc(v_base + kt * 2048, kHalf, 1024);
-                    const uint64_t bd = smem_desc(p_base + kt * 2048, kPBytes, 1024);
-                    mma_ss(d_tmem, ad, bd, idesc_pv, (pd.first && kt == 0) ? 0u : 1u);
-                }
+                for (int kt = 0; kt < kTok / 16; ++kt)
+                    mma_ss(d_tmem, vd + (uint64_t)((kt * 2048) >> 4),
+                           pdesc + (uint64_t)((kt * 2048) >> 4), idesc_pv,
+                           (pd.first && kt == 0) ? 0u : 1u);
                 mma_commit(&v_empty[vs]);
                 mma_commit(&pv_done[pd.n & 1]);
                 if (pd.last) mma_commit(&o_full[pd.item & 1]);
@@ -908,7 +917,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             }
             const int nch = slots[sl].nch;
             if (nch < 0) break;
-            const uint32_t q_base = smem_u32(smem + kQOff + (item & 1) * kQBytes);
+            const uint64_t qd = q_desc0 + (uint64_t)(((item & 1) * kQBytes) >> 4);
             for (int c = 0; c < nch; ++c, ++n) {
                 bool good = true;
                 if (lane == 0) {
@@ -924,13 +933,14 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t k_base = smem_u32(smem + kKOff + (n % kKStages) * kStageBytes);
+                    const uint64_t kd =
+                        k_desc0 + (uint64_t)(((n % kKStages) * kStageBytes) >> 4);
 #pragma unroll
                     for (int ks = 0; ks < kD / 16; ++ks) {
-                        const uint32_t off = (ks & 3) * 32;  // 16-wide d slice in the atom
-                        const uint64_t ad = smem_desc(k_base + (ks >> 2) * kHalf + off, 16, 1024);
-                        const uint64_t bd = smem_desc(q_base + (ks >> 2) * kQHalf + off, 16, 1024);
-                        mma_ss(tmem + (n & 1) * 32, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+                        const uint32_t k_off = ((ks >> 2) * kHalf + (ks & 3) * 32) >> 4;
+                        const uint32_t q_off = ((ks >> 2) * kQHalf + (ks & 3) * 32) >> 4;
+                        mma_ss(tmem + (n & 1) * 32, kd + k_off, qd + q_off, idesc_s,
+                               ks > 0 ? 1u : 0u);
                     }
                     mma_commit(&s_full[n & 1]);
                     mma_commit(&k_empty[n % kKStages]);
