@@ -81,3 +81,21 @@ def test_tc_large_logits_rescale_path():
     out = run(case, "tc")
     assert torch.isfinite(out).all()
     assert_attn_close(out, oracle_out(case), "tcgen05 rescale")
+
+
+@pytest.mark.parametrize("kernel", ["tc", "rows"])
+def test_late_dominant_keys_force_the_rescale(kernel):
+    """Keys of all 64 at token 300 and of all 128 at token 700 (after the
+    first chunk sets the softmax reference) give every row whose query sums
+    to a positive value a logit tens of powers of two above that reference:
+    the tcgen05 kernel's chunk-sum check must take the exact path (max, O and
+    sums rescaled) once or twice per row; the 32-row kernel's rescale too."""
+    case = inputs.multi_query_case(2, 16, 2, 128, 16, [900, 400], [128, 64],
+                                   seed=44, device="cuda")
+    bs = case.workload.block_size
+    for s, t, val in [(0, 300, 64.0), (0, 700, 128.0), (1, 200, 64.0)]:
+        blk = int(case.tables_np[s][t // bs])
+        case.k_cache[blk, t % bs] = val
+    out = run(case, kernel)
+    assert torch.isfinite(out).all()
+    assert_attn_close(out, oracle_out(case), f"{kernel}: late dominant keys")
