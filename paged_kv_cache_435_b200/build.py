@@ -20,7 +20,7 @@ SOURCES = ["pa_api.cu", "pa_decode.cu", "pa_multi_query.cu", "pa_multi_query_tc.
            "pa_multi_row.cu", "pa_cache_ops.cu",
            "pa_swap.cu", "pa_static_ws.cu", "pa_block_manager.cpp"]
 HEADERS = ["pa_common.cuh", "pa_decode.cuh", "pa_multi_query.cuh",
-           "pa_multi_row.cuh", "pa_cascade.cuh", "pa_cache_ops.cuh", "pa_swap.cuh"]
+           "pa_multi_row.cuh", "pa_cascade.cuh", "pa_split.cuh", "pa_cache_ops.cuh", "pa_swap.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

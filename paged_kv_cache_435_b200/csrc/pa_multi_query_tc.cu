@@ -48,6 +48,7 @@
 
 #include "pa_common.cuh"
 #include "pa_multi_query.cuh"
+#include "pa_split.cuh"
 
 namespace pa {
 namespace {
@@ -613,20 +614,12 @@ paged_multi_query_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                 psum = exponentiate(sv);
             }
             l_part += psum;
-            // bf16 split of p by truncation: the high half keeps 8
-            // significant bits, the residual another 8, so P carries ~16
-            // bits into PV.  Pairs of tokens in the warpgroup's first 32
-            // columns, the residuals in the next 32.
+            // p as bf16 plus its bf16 residual, both rounded to nearest (P
+            // carries ~17 bits into PV).  Pairs of tokens in the
+            // warpgroup's first 32 columns, the residuals in the next 32.
             uint32_t hi[32], lo[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float a = sv[2 * i], b = sv[2 * i + 1];
-                const uint32_t ab = __float_as_uint(a), bb = __float_as_uint(b);
-                const float al = a - __uint_as_float(ab & 0xFFFF0000u);
-                const float bl = b - __uint_as_float(bb & 0xFFFF0000u);
-                hi[i] = __byte_perm(ab, bb, 0x7632);
-                lo[i] = __byte_perm(__float_as_uint(al), __float_as_uint(bl), 0x7632);
-            }
+            for (int i = 0; i < 32; ++i) split_bf16x2(sv[2 * i], sv[2 * i + 1], hi[i], lo[i]);
             tmem_st32(sbase, hi);
             tmem_st32(sbase + 32, lo);
             tmem_wait_st();

@@ -49,11 +49,16 @@
 //              output row into a 4-slot shared-memory ring and copies the Q
 //              rows (cp.async), so no other warp waits on a global load at an
 //              item boundary.
-// Online softmax with a lazy reference: every chunk, one barrier-reduction
-// over the 4 warps (bar.red.popc) asks whether any row's logit exceeds its
-// reference max by more than 2^8; only then is the exact per-row chunk max
-// formed (warp transpose-reduction + shared memory), O^T rescaled in TMEM and
-// the reference moved.  Sums are kept per thread and reduced at item end.
+// Online softmax with a lazy reference: an item's rows start from the logit
+// of the item's first token (every row sees it, so each row's sum is at
+// least 1), which thread 0 publishes through shared memory.  Every chunk,
+// one barrier-reduction over the 4 warps (bar.red.popc) asks whether any
+// row's logit exceeds its reference by more than 2^24 (weights stay below
+// 2^24, far from fp32 overflow, and the split of P keeps its relative
+// precision at any scale, so the reference need not be tight); only then is
+// the exact per-row chunk max formed (warp transpose-reduction + shared
+// memory), O^T rescaled in TMEM and the reference moved.  Sums are kept per
+// thread and reduced at item end.
 // A token no row may see (padding, past the range) has its V row zeroed by
 // its own thread once the chunk landed: P is 0 there, but 0 x NaN is NaN.
 // The producers and the MMA warp run ahead across item boundaries; the
@@ -68,6 +73,7 @@
 
 #include "pa_cascade.cuh"
 #include "pa_common.cuh"
+#include "pa_split.cuh"
 #include "pa_multi_row.cuh"
 
 namespace pa {
@@ -118,7 +124,7 @@ constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 15 + 2 * kSlots;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16;
 constexpr uint32_t kTmemCols = 256;       // S0 | S1 | O0 (hi, lo) | O1 (hi, lo)
 constexpr uint32_t kTmemO = 64;           // first O column
-constexpr float kRescaleThreshold = 8.f;  // log2 units
+constexpr float kRescaleThreshold = 24.f;  // log2 units
 constexpr float kNoMax = -FLT_MAX;        // reference of a row with no token yet
 constexpr int kNumSMs = 148;
 
@@ -1093,6 +1099,24 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
 #pragma unroll
                     for (int r = 0; r < 32; ++r) x[r] = -INFINITY;
                 }
+                if (c == 0) {
+                    // References from the item's first token (thread 0).  The
+                    // previous readers of cmax passed the item barrier above.
+                    if (tid == 0) {
+#pragma unroll
+                        for (int r = 0; r < 32; ++r) cmax[r] = x[r];
+                    }
+                    softmax_sync();
+#pragma unroll
+                    for (int r = 0; r < 32; r += 4) {
+                        const float4 c4 = *reinterpret_cast<const float4*>(cmax + r);
+                        const float c0[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)  // -inf: a row that does not exist
+                            m_ref[r + e] = c0[e] > -INFINITY ? c0[e] : 0.f;
+                    }
+                    // cmax is read again only after the vote barrier below.
+                }
                 bool grow = false;
 #pragma unroll
                 for (int r = 0; r < 32; ++r) grow = grow || x[r] > m_ref[r] + kRescaleThreshold;
@@ -1150,8 +1174,8 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 if (n >= 2 && !__all_sync(0xffffffffu,
                                           wait_bar(&pv_done[sb], ((n - 2) >> 1) & 1)))
                     fail = true;
-                // P = 2^(x - m) split by truncation: the high half keeps 8
-                // significant bits, the residual's high half another 8.
+                // P = 2^(x - m) as bf16 plus its bf16 residual, both rounded
+                // to nearest (P carries ~17 bits into PV).
                 uint32_t hi[16], lo[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
@@ -1159,11 +1183,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const float b = exp2f(x[2 * i + 1] - m_ref[2 * i + 1]);
                     l_part[2 * i] += a;
                     l_part[2 * i + 1] += b;
-                    const uint32_t ab = __float_as_uint(a), bb = __float_as_uint(b);
-                    const float al = a - __uint_as_float(ab & 0xFFFF0000u);
-                    const float bl = b - __uint_as_float(bb & 0xFFFF0000u);
-                    hi[i] = __byte_perm(ab, bb, 0x7632);
-                    lo[i] = __byte_perm(__float_as_uint(al), __float_as_uint(bl), 0x7632);
+                    split_bf16x2(a, b, hi[i], lo[i]);
                 }
                 unsigned char* prow = smem + kPOff + sb * kPBytes + p_row;
 #pragma unroll
