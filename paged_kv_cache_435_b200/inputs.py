@@ -406,8 +406,14 @@ def grouped_case(num_heads: int, num_kv_heads: int, head_size: int,
         cursor += n
     w = Workload(f"grouped{seed}", 0, B, num_heads, num_kv_heads, head_size,
                  block_size, "fixed")
+    # Distinct cached positions: each group's shared tokens once (as far as
+    # its longest member reaches into them), every private token.
+    unique = int((lens - shared_of).sum())
+    for i in range(len(pl)):
+        members = shared_of[int(gs[i]):int(gs[i + 1])]
+        unique += int(members.max(initial=0))
     case = _finish(w, lens, tables, NB, np.zeros((0, 2), dtype=np.int64),
-                   device, seed + 1, None, unique_tokens=0)
+                   device, seed + 1, None, unique_tokens=unique)
     dev = torch.device(device)
     mgs = int(np.max(np.diff(gs), initial=1)) if max_group_size is None else max_group_size
     return dataclasses.replace(case, group_start=torch.from_numpy(gs).to(dev),
