@@ -421,6 +421,23 @@ __device__ RowItem row_item(const MultiRowParams& p, int idx, bool report_errors
 // Work of unit u (sequence or group) for the item deal: its live row tiles
 // and the weight of each of its items (128-token chunks, plus one for the
 // per-item overhead).  Invalid groups have no tiles.
+// Multi-query mode: tiles and weight of a sequence from its raw context
+// length and query count, clamped (and reported) as clamp_len and
+// clamp_queries do.
+__device__ __forceinline__ void query_unit_work(const MultiRowParams& p, int L, int k,
+                                                bool report_errors, int& tiles, int& w) {
+    if (L < 0 || L > p.max_context_len) {
+        if (report_errors) report(p.error_flags, PA_DEVERR_CONTEXT_LEN);
+        L = L < 0 ? 0 : p.max_context_len;
+    }
+    if (k < 0 || k > L || k > p.max_query_len) {
+        if (report_errors) report(p.error_flags, PA_DEVERR_QUERY_LEN);
+        k = k < 0 ? 0 : min(k, min(L, p.max_query_len));
+    }
+    tiles = min((k * p.group + kN - 1) / kN, p.tiles);
+    w = (L + kTok - 1) / kTok + 1;
+}
+
 __device__ __forceinline__ void unit_work(const MultiRowParams& p, int u,
                                           bool report_errors, int& tiles, int& w) {
     if (!p.shared_prefix_mode) {
@@ -663,6 +680,28 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
         constexpr int kUnitRounds = 8;
         int tl[kUnitRounds], w[kUnitRounds];
         auto gather = [&](int base, bool report_errors) {
+            if (!p.shared_prefix_mode) {
+                // Every round's lengths first: the error reports below are
+                // atomics on a flag word that may alias the inputs, so loads
+                // after one could not be issued before it.
+                int Lr[kUnitRounds], q0[kUnitRounds], q1[kUnitRounds];
+#pragma unroll
+                for (int k = 0; k < kUnitRounds; ++k) {
+                    const int u = base + k * 32 + lane;
+                    const bool in = u < p.num_units;
+                    Lr[k] = in ? p.context_lens[u] : 0;
+                    q0[k] = in ? p.query_start_loc[u] : 0;
+                    q1[k] = in ? p.query_start_loc[u + 1] : 0;
+                }
+#pragma unroll
+                for (int k = 0; k < kUnitRounds; ++k) {
+                    tl[k] = 0;
+                    w[k] = 0;
+                    if (base + k * 32 + lane < p.num_units)
+                        query_unit_work(p, Lr[k], q1[k] - q0[k], report_errors, tl[k], w[k]);
+                }
+                return;
+            }
 #pragma unroll
             for (int k = 0; k < kUnitRounds; ++k) {
                 const int u = base + k * 32 + lane;
