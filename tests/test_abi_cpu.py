@@ -4,6 +4,8 @@ documented status before any CUDA call."""
 import ctypes
 import os
 import re
+import subprocess
+import sys
 
 import pytest
 
@@ -221,3 +223,32 @@ def test_shared_prefix_workspace_grows_with_rows(lib):
     assert a == nat.pa_decode_workspace_size(8, 32, 8, 128, 16, 1000) + 256
     # no split (short contexts): the flags alone
     assert nat.pa_shared_prefix_workspace_size(8, 32, 8, 128, 16, 300) == 256
+
+
+def test_missing_library_raises_instead_of_falling_back():
+    """No CPU path exists: without the shared library the first call fails."""
+    code = (
+        "import sys; sys.path.insert(0, %r)\n"
+        "from paged_kv_cache_435_b200 import _native\n"
+        "_native.LIB_PATH = '/nonexistent/libpagedattn.so'\n"
+        "try:\n"
+        "    _native.raw()\n"
+        "except ImportError as e:\n"
+        "    print('raised', e)\n"
+        "else:\n"
+        "    print('loaded')\n" % ROOT)
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True,
+                         text=True, timeout=120)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.startswith("raised"), out.stdout
+
+
+def test_cpu_tensors_are_rejected_not_computed():
+    import torch
+    import paged_kv_cache_435_b200 as pa
+    q = torch.zeros(1, 4, 64, dtype=torch.bfloat16)
+    pool = torch.zeros(4, 16, 4, 64, dtype=torch.bfloat16)
+    out = torch.zeros(1, 4, 64, dtype=torch.float32)
+    with pytest.raises(TypeError, match="CUDA"):
+        pa.pa_decode_attention(out, q, pool, pool, torch.zeros(1, 1, dtype=torch.int32),
+                               torch.ones(1, dtype=torch.int32), 1, 0.125)
