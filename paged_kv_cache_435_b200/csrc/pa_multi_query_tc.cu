@@ -188,6 +188,27 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// Pairs of fp32 values in one 64-bit register pair, for the sm_100 packed
+// fp32 arithmetic (same rounding as the scalar instructions).
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpack_f32x2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
 // L2 policy with the default (normal) eviction priority.
 __device__ __forceinline__ uint64_t l2_policy_normal() {
     uint64_t pol;
@@ -551,14 +572,24 @@ paged_multi_query_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         };
         // In place: sv <- 2^(scale*s - m_ref) (masked logits give 0); the sum.
+        // The exponent arguments and the partial sums run on pairs
+        // (fma.rn.f32x2 / add.rn.f32x2: the scalar roundings, half the
+        // instructions).
         auto exponentiate = [&](float (&sv)[64]) -> float {
-            float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            const float neg_m = -m_ref;
+            const uint64_t s2 = pack_f32x2(sl2, sl2);
+            const uint64_t nm2 = pack_f32x2(-m_ref, -m_ref);
+            uint64_t acc[4] = {0, 0, 0, 0};      // four packed pairs of partial sums
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                sv[i] = ex2_approx(fmaf(sv[i], sl2, neg_m));
-                ps8[i & 7] += sv[i];
+            for (int i = 0; i < 32; ++i) {
+                float a, b;
+                unpack_f32x2(fma_f32x2(pack_f32x2(sv[2 * i], sv[2 * i + 1]), s2, nm2), a, b);
+                sv[2 * i] = ex2_approx(a);
+                sv[2 * i + 1] = ex2_approx(b);
+                acc[i & 3] = add_f32x2(acc[i & 3], pack_f32x2(sv[2 * i], sv[2 * i + 1]));
             }
+            float ps8[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) unpack_f32x2(acc[j], ps8[2 * j], ps8[2 * j + 1]);
             return ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) +
                    ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
         };
