@@ -208,6 +208,11 @@ int pa_decode_attention(float* out, const void* q, const void* k_cache,
  *                       PA_DEVERR_QUERY_LEN, PA_DEVERR_TIMEOUT
  * Supports head_size in {64, 128}, block_size in {16, 32},
  * num_heads / num_kv_heads in 1..64.  Returns PA_OK or a negative pa_status.
+ * The kernel follows from the shape (head_size 128: a 128-row tensor-core
+ * kernel when max_query_len * group >= 128, else a 32-row one; head_size
+ * 64: a warp-level MMA kernel); the environment variable
+ * PA_MULTI_QUERY_KERNEL = mma | tc | rows forces one of them (tests,
+ * benchmarks).  Every choice computes the same function.
  */
 int pa_multi_query_attention(float* out, const void* q, const void* k_cache,
                              const void* v_cache, const int32_t* block_tables,
