@@ -47,9 +47,16 @@ METRIC = ("paged decode attn: KV GB/s and % of HBM peak; seq-tokens/s at "
           "batch 256")
 DEFAULT_WORKLOAD = "llama2_70b_gqa_b256"
 FALLBACK_HBM_GBS = 6650.0
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_dram_traffic.txt")
-KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_435_b200", "csrc", f)
-                  for f in ("pa_decode.cu", "pa_common.cuh", "pa_decode.cuh")]
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "dram_traffic_by_workload.txt")
+_CSRC = os.path.join(ROOT, "paged_kv_cache_435_b200", "csrc")
+# Sources whose change invalidates a recorded DRAM-traffic figure, per kernel.
+KERNEL_SOURCES = {
+    "paged_decode_kernel": ["pa_decode.cu", "pa_common.cuh", "pa_decode.cuh"],
+    "paged_multi_row_kernel": ["pa_multi_row.cu", "pa_common.cuh", "pa_split.cuh",
+                               "pa_cascade.cuh", "pa_multi_row.cuh"],
+    "paged_multi_query_tc_kernel": ["pa_multi_query_tc.cu", "pa_common.cuh",
+                                    "pa_split.cuh", "pa_multi_query.cuh"],
+}
 
 
 # ---------------------------------------------------------------- accounting
@@ -92,31 +99,52 @@ def step_bytes(case) -> int:
     return attention_bytes(case) + write + cow
 
 
-def kernel_sha() -> str:
+def kernel_sha(kernel: str = "paged_decode_kernel") -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
-        with open(p, "rb") as f:
-            h.update(f.read())
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(_CSRC, f), "rb") as fh:
+            h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def read_traffic(workload: str):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was
-    taken on the current kernel source for this workload."""
+def dominant_kernel(case, shared_prefix: bool) -> str:
+    """The kernel whose DRAM traffic the roofline line reports."""
+    if case.query_start_loc is not None:
+        k = int(case.query_lens_np.max()) * (case.workload.num_heads //
+                                             case.workload.num_kv_heads)
+        return ("paged_multi_query_tc_kernel" if k >= 128 and case.workload.head_size == 128
+                else "paged_multi_row_kernel")
+    return "paged_multi_row_kernel" if shared_prefix else "paged_decode_kernel"
+
+
+def read_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    summary: records of `key = value` lines separated by blank lines, used
+    only while the record's kernel_sha matches the current kernel sources."""
     if not os.path.exists(PROFILE_TRAFFIC):
         return None
-    kv = {}
+    records, cur = [], {}
     with open(PROFILE_TRAFFIC) as f:
         for line in f:
-            if "=" in line and not line.lstrip().startswith("#"):
+            line = line.strip()
+            if not line:
+                if cur:
+                    records.append(cur)
+                cur = {}
+                continue
+            if "=" in line and not line.startswith("#"):
                 k, v = line.split("=", 1)
-                kv[k.strip()] = v.strip()
-    if kv.get("kernel_sha") != kernel_sha() or kv.get("workload") != workload:
-        return None
-    try:
-        return float(kv["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
+                cur[k.strip()] = v.strip()
+    if cur:
+        records.append(cur)
+    for r in records:
+        if (r.get("workload") == workload and r.get("kernel") == kernel and
+                r.get("kernel_sha") == kernel_sha(kernel)):
+            try:
+                return float(r["dram_bytes_per_launch"])
+            except (KeyError, ValueError):
+                return None
+    return None
 
 
 def hbm_peak():
@@ -151,7 +179,7 @@ class ClockSampler:
         0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.01):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.samples, self.reasons = [], 0
         self.max_mhz = None
         self._stop = threading.Event()
@@ -185,6 +213,13 @@ class ClockSampler:
         self._stop.set()
         if self._nvml is not None:
             self._t.join()
+
+    def absorb(self, other: "ClockSampler"):
+        """Add another sampler's record (a second timed region)."""
+        self.samples.extend(other.samples)
+        self.reasons |= other.reasons
+        if self.max_mhz is None:
+            self.max_mhz = other.max_mhz
 
     def summary(self):
         if not self.samples:
@@ -302,15 +337,22 @@ def run_gpu(args):
     stream = torch.cuda.current_stream(dev)
 
     # in-run copy bandwidth (read + write bytes of a 1 GiB device copy)
-    copy_best = None
+    # and in-run read-only stream bandwidth (a 1 GiB fp32-accumulated sum:
+    # the decode kernel only reads its big operand, which a copy peak, half
+    # of whose bytes are writes, can understate)
+    copy_best = read_best = None
     if not args.kernel_only:
-        a = torch.empty(1 << 29, dtype=torch.bfloat16, device=dev)
+        a = torch.ones(1 << 29, dtype=torch.bfloat16, device=dev)
         b = torch.empty_like(a)
-        copy_best = 0.0
+        copy_best = read_best = 0.0
         for _ in range(6):
             e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
             e0.record(stream); b.copy_(a); e1.record(stream); e1.synchronize()
             copy_best = max(copy_best, 2 * a.numel() * 2 /
+                            (e0.elapsed_time(e1) * 1e-3) / 1e9)
+            e0.record(stream); a.sum(dtype=torch.float32); e1.record(stream)
+            e1.synchronize()
+            read_best = max(read_best, a.numel() * 2 /
                             (e0.elapsed_time(e1) * 1e-3) / 1e9)
         del a, b
 
@@ -340,7 +382,10 @@ def run_gpu(args):
     flags = int(step.flags.item())
 
     # e2e: host buffers through the public API
-    e2e = None if args.kernel_only else run_e2e(case, step, args, dist, dev)
+    e2e = None
+    if not args.kernel_only:
+        e2e, e2e_clk = run_e2e(case, step, args, dist, dev)
+        clk.absorb(e2e_clk)
 
 
     ms_total = max_over_ranks(dist, ms_total, dev)
@@ -356,7 +401,8 @@ def run_gpu(args):
     tensor_bound = flops / ab > ridge
     achieved = ab / (attn_ms_max * 1e-3) / 1e9
     achieved_tflops = flops / (attn_ms_max * 1e-3) / 1e12
-    traffic = read_traffic(args.workload)
+    dom = dominant_kernel(case, step.shared_prefix)
+    traffic = read_traffic(w.name, dom)
     if tensor_bound:
         roof = {"bound": "tensor", "achieved": round(achieved_tflops, 1),
                 "peak": tpeak,
@@ -367,7 +413,7 @@ def run_gpu(args):
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                                if peak_kind == "measured" else "fallback 6.65 TB/s",
                 "unit": "GB/s", "frac": round(achieved / peak, 4)}
-    kernel_name = ("paged_multi_query_kernel" if case.query_start_loc is not None
+    kernel_name = (dom if case.query_start_loc is not None
                    else ("paged_multi_row_kernel (group pass) + " if step.shared_prefix
                          else "") + "paged_decode_kernel" +
                    (" + reduce" if step.partition < case.max_context_len else ""))
@@ -416,11 +462,15 @@ def run_gpu(args):
             "pct_hbm_peak": round(100 * value / (world * peak), 2),
             "step_bytes": sb,
             "in_run_copy_gbs": None if copy_best is None else round(copy_best, 1),
+            "in_run_read_gbs": None if read_best is None else round(read_best, 1),
             "roofline": dict(
                 kernel=kernel_name, **roof,
                 frac_of_in_run_copy=(None if copy_best is None or tensor_bound
                                      else round(achieved / copy_best, 4)),
+                frac_of_in_run_read=(None if read_best is None or tensor_bound
+                                     else round(achieved / read_best, 4)),
                 traffic=traffic,
+                traffic_kernel=dom,
                 algorithmic_bytes_per_launch=ab,
                 flops_per_launch=flops,
                 achieved_gbs=round(achieved, 1),
@@ -440,11 +490,13 @@ def run_gpu(args):
 
 def run_e2e(case, step, args, dist, dev):
     """Per step: pinned host -> device copies of the step's inputs, the
-    library calls, device -> host copy of the output.  Copies run on a second
-    stream, double-buffered, so step i+1's inputs travel while step i
-    computes and step i's output returns while step i+1 computes; every
-    step's copies are inside the timed region.  The KV pool is written and
-    read only on the compute stream, in step order."""
+    library calls, device -> host copy of the output.  Inputs travel on one
+    copy stream and outputs on another (the two directions use separate copy
+    engines and overlap), double-buffered, so step i+1's inputs travel while
+    step i computes and step i's output returns while step i+1 computes;
+    every step's copies are inside the timed region.  The KV pool is written
+    and read only on the compute stream, in step order.  Returns the e2e
+    record and the clock sampler of its timed region."""
     import paged_kv_cache_435_b200 as pa
     c = case
     names = ["q", "new_key", "new_value", "slot_mapping", "block_tables",
@@ -459,7 +511,8 @@ def run_e2e(case, step, args, dist, dev):
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = host_out[0].numel() * host_out[0].element_size()
     comp = torch.cuda.current_stream(dev)
-    copy = torch.cuda.Stream(dev)
+    up = torch.cuda.Stream(dev)     # host -> device
+    down = torch.cuda.Stream(dev)   # device -> host
     ev = lambda: torch.cuda.Event()  # noqa: E731
     in_ready = [ev(), ev()]     # inputs of buffer b landed
     in_free = [ev(), ev()]      # compute finished reading buffer b
@@ -469,11 +522,11 @@ def run_e2e(case, step, args, dist, dev):
         e.record(comp)
 
     def stage_inputs(b):
-        with torch.cuda.stream(copy):
-            copy.wait_event(in_free[b])
+        with torch.cuda.stream(up):
+            up.wait_event(in_free[b])
             for n in names:
                 dev_in[b][n].copy_(host_in[n], non_blocking=True)
-            in_ready[b].record(copy)
+            in_ready[b].record(up)
 
     def compute(b):
         d = dev_in[b]
@@ -509,10 +562,10 @@ def run_e2e(case, step, args, dist, dev):
         out_ready[b].record(comp)
 
     def return_output(b):
-        with torch.cuda.stream(copy):
-            copy.wait_event(out_ready[b])
+        with torch.cuda.stream(down):
+            down.wait_event(out_ready[b])
             host_out[b].copy_(outs[b], non_blocking=True)
-            out_free[b].record(copy)
+            out_free[b].record(down)
 
     def run(n):
         stage_inputs(0)
@@ -526,20 +579,41 @@ def run_e2e(case, step, args, dist, dev):
     torch.cuda.synchronize(dev)
     K = args.steps
     t0, t1 = torch.cuda.Event(True), torch.cuda.Event(True)
-    barrier(dist)
-    torch.cuda.synchronize(dev)
-    t0.record(comp)
-    run(K)
-    comp.wait_stream(copy)  # the last output has reached the host
-    t1.record(comp)
-    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clk:
+        barrier(dist)
+        torch.cuda.synchronize(dev)
+        t0.record(comp)
+        run(K)
+        comp.wait_stream(down)  # the last output has reached the host
+        t1.record(comp)
+        torch.cuda.synchronize(dev)
+        barrier(dist)
     ms = max_over_ranks(dist, t0.elapsed_time(t1), dev) / K
+
+    # Breakdown: each direction's copies alone, K steps' worth, on its stream.
+    def copy_ms(stream, fn):
+        e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for i in range(K):
+                fn(i % 2)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / K
+
+    h2d_ms = copy_ms(up, lambda b: [dev_in[b][n].copy_(host_in[n], non_blocking=True)
+                                    for n in names])
+    d2h_ms = copy_ms(down, lambda b: host_out[b].copy_(outs[b], non_blocking=True))
     world = dist.get_world_size() if dist is not None else 1
     return {"value": round(world * step_bytes(case) / (ms * 1e-3) / 1e9, 2),
             "unit": "GB/s", "ms_per_step": round(ms, 5),
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "overlap": "double-buffered: inputs of step i+1 and output of "
-                       "step i cross PCIe while step i / i+1 compute"}
+            "h2d_ms_per_step_alone": round(h2d_ms, 5),
+            "d2h_ms_per_step_alone": round(d2h_ms, 5),
+            "overlap": "double-buffered on two copy streams (inputs up, "
+                       "outputs down): step i+1's inputs and step i's output "
+                       "cross PCIe while step i / i+1 compute"}, clk
 
 
 # ---------------------------------------------------------------- CPU (oracle)
@@ -588,7 +662,22 @@ def sample_bytes(case, seqs):
     return kv + B * w.num_heads * w.head_size * 6 + tables + B * 4
 
 
-def cpu_baseline(args, budget_s: float = 10.0):
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def cpu_baseline(args, budget_s: float = 10.0, budget_1core_s: float = 8.0):
+    """The fp64 oracle on the host: all threads on a 64-sequence sample for
+    about budget_s, then one thread on the first 8 of those sequences for
+    about budget_1core_s."""
     import oracle
     oracle.build()
     threads = oracle.default_threads()
@@ -599,12 +688,25 @@ def cpu_baseline(args, budget_s: float = 10.0):
         elapsed += time_oracle(case, seqs, threads)
         reps += 1
     n = case.workload.num_seqs if seqs is None else len(seqs)
+
+    case1, seqs1 = oracle_sample(args.workload, 8)
+    nbytes1 = sample_bytes(case1, seqs1)
+    reps1, elapsed1 = 0, 0.0
+    while elapsed1 < budget_1core_s or reps1 == 0:
+        elapsed1 += time_oracle(case1, seqs1, 1)
+        reps1 += 1
+    n1 = case1.workload.num_seqs if seqs1 is None else len(seqs1)
     return {"value": round(reps * nbytes / elapsed / 1e9, 4), "unit": "GB/s",
             "cores": threads, "kind": "oracle",
             "sample": f"{n} sequences of {args.workload} (same shapes and "
                       f"length draw, host-built pool), {reps} passes, "
-                      f"{elapsed:.1f} s, fp64 C oracle on {threads} threads",
-            "seq_tokens_per_s": round(reps * n / elapsed, 2)}
+                      f"{elapsed:.1f} s, fp64 C oracle on {threads} threads; "
+                      f"1 thread: {n1} sequences, {reps1} passes, {elapsed1:.1f} s",
+            "seq_tokens_per_s": round(reps * n / elapsed, 2),
+            "value_1core": round(reps1 * nbytes1 / elapsed1 / 1e9, 4),
+            "seq_tokens_per_s_1core": round(reps1 * n1 / elapsed1, 2),
+            "os_cpu_count": os.cpu_count(),
+            "cpu_model": cpu_model()}
 
 
 def run_reference(args):
@@ -645,6 +747,7 @@ def run_reference(args):
                    "sample_seqs_per_step": n},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s",
                          "cores": threads, "kind": "oracle",
+                         "os_cpu_count": os.cpu_count(), "cpu_model": cpu_model(),
                          "sample": f"{n} sequences of {w.name} per step, fp64 C "
                                    f"oracle on {threads} threads"},
         "e2e": {"value": round(value, 4), "unit": "GB/s",

@@ -151,12 +151,23 @@ size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
  *     k_t = k_cache[block_tables[s][t / block_size]][t % block_size][g][:]
  *     z_t = scale * dot(q[s][h][:], k_t)              for t in [0, L)
  *     out[s][h][:] = sum_t softmax(z)_t * v_t          (fp32)
- * and out[s][h][:] = 0 when L = 0.
+ * and out[s][h][:] = 0 when L = 0.  The gather through the block table is
+ * the one the pages describe: logical block i of a sequence lives in
+ * whichever physical block its table names ("vLLM: Anatomy and Mechanisms of
+ * High-Throughput LLM Inference", "Block-Level Management"; "vLLM
+ * Internals", "The Block Manager"), and the step streams the whole cached
+ * context once, which makes it bandwidth bound (first page, "Prefill vs.
+ * Decode Operations", "The Roofline Model").
  *
- * Work is split into one CTA per (sequence, kv head, KV partition); the CTA
- * reads each of its blocks once for all query heads of the group.  Contexts
- * longer than the partition width are split into partitions whose (max, sum,
- * normalised partial output) are merged by a second kernel.
+ * Work unit: one (sequence, KV partition) for one kv head, which reads each
+ * of its blocks once for all query heads of the group.  Without a split the
+ * grid has one CTA per (kv head, sequence).  When contexts are split into
+ * partitions (partition_size below max_context_len), a persistent grid of
+ * about two CTAs per SM walks the compact list of (sequence, partition)
+ * items of each kv head (no CTA is spent past a sequence's end; above 768
+ * sequences a plain grid of one CTA per (kv head, partition, sequence) with
+ * early exit is used instead), and the partitions' (max, sum, normalised
+ * partial output) are merged by a second kernel.
  *
  *   max_blocks_per_seq   row length of block_tables (>= 1).
  *   max_context_len      host-known upper bound of context_lens
@@ -429,9 +440,16 @@ int pa_bm_shared_prefix_groups(const pa_block_manager* m, const int32_t* seq_ids
  * every GPU that uses the library until the process exits).  It never calls
  * cudaMalloc, cudaFree or any allocating routine.
  *
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and caches it; make
- *     that first call before any stream capture.
+ *   - Every call looks up the array's device address on the current device
+ *     (cudaGetSymbolAddress, which allocates nothing), so the address stays
+ *     right after a context has been torn down and created again.  The
+ *     array itself is committed on a device when the library's device code
+ *     is first loaded there (with CUDA's lazy loading, typically the first
+ *     call of this function on that device); a process whose device memory
+ *     another allocator reserves at start-up should make one call with
+ *     num_seqs = 0 first, which commits the array and enqueues nothing.
+ *     Make that first call before any stream capture.
+ *   - out and the other buffers must be on the current device.
  *   - If pa_decode_workspace_size(...) for these arguments exceeds
  *     PA_STATIC_WORKSPACE_BYTES the call returns PA_ERR_WORKSPACE and
  *     enqueues nothing (use a larger partition_size, or pa_decode_attention

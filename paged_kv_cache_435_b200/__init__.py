@@ -15,7 +15,9 @@ points are bound here under the same names:
   (preemption by swapping);
 * ``pa_decode_attention_shared_prefix``: decode attention that reads the
   prompt blocks shared by a group of sequences (parallel samples, beams)
-  once for the whole group.
+  once for the whole group;
+* ``pa_decode_attention_static_ws``: ``pa_decode_attention`` with scratch
+  built into the library, for callers that cannot allocate device memory.
 
 ``inputs`` builds seeded synthetic workloads.  The library is loaded lazily on
 first use and its absence raises; nothing here computes on the CPU.
@@ -26,6 +28,7 @@ from ._native import (  # noqa: F401
     PA_DEVERR_PREFIX, PA_DEVERR_QUERY_LEN, PA_ERR_UNSUPPORTED,
     PA_ERR_WORKSPACE, PA_OK, PAError, library_path,
     pa_copy_blocks, pa_decode_attention, pa_decode_attention_shared_prefix,
+    pa_decode_attention_static_ws,
     pa_decode_partition_size, pa_shared_prefix_workspace_size,
     pa_decode_workspace_size, pa_launch_count, pa_multi_query_attention,
     pa_reshape_and_cache, pa_swap_blocks, raw, status_string)

@@ -90,6 +90,10 @@ def raw():
         lib.pa_copy_blocks.argtypes = [p, p, i32, p, i32, i32, i32, i32, i32,
                                        p, p]
         lib.pa_copy_blocks.restype = i32
+        lib.pa_decode_attention_static_ws.argtypes = [
+            p, p, p, p, p, i32, p, i32, i32, i32, i32, i32, i32, i32, f32, i32,
+            p, p]
+        lib.pa_decode_attention_static_ws.restype = i32
         _lib = lib
         return lib
 
@@ -363,12 +367,7 @@ def pa_decode_attention_static_ws(out, q, k_cache, v_cache, block_tables,
     """pa_decode_attention with the library's built-in workspace, for callers
     that cannot allocate device memory (see include/pa.h)."""
     import torch
-    lib = raw()
-    f = lib.pa_decode_attention_static_ws
-    p, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
-    f.argtypes = [p, p, p, p, p, i32, p, i32, i32, i32, i32, i32, i32, i32,
-                  f32, i32, p, p]
-    f.restype = i32
+    f = raw().pa_decode_attention_static_ws
     bf = torch.bfloat16
     _cuda(out, "out", torch.float32, 3); _cuda(q, "q", bf, 3)
     _cuda(k_cache, "k_cache", bf, 4); _cuda(v_cache, "v_cache", bf, 4)
@@ -385,6 +384,15 @@ def pa_decode_attention_static_ws(out, q, k_cache, v_cache, block_tables,
         raise ValueError("shape mismatch between q, out and the pools")
     if block_tables.shape[0] != B or context_lens.shape[0] != B:
         raise ValueError("block_tables / context_lens must have B rows")
+    # The built-in scratch is looked up on the current device: every buffer
+    # must live there too.
+    cur = torch.cuda.current_device()
+    for name, t in (("out", out), ("q", q), ("k_cache", k_cache),
+                    ("v_cache", v_cache), ("block_tables", block_tables),
+                    ("context_lens", context_lens), ("error_flags", error_flags)):
+        if t is not None and t.device.index != cur:
+            raise ValueError(f"{name} is on cuda:{t.device.index}, the current "
+                             f"device is cuda:{cur}")
     rc = f(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
            block_tables.shape[1], _ptr(context_lens), int(max_context_len), B,
            Hq, Hkv, D, bs, NB, float(scale), int(partition_size),

@@ -21,9 +21,19 @@ namespace pa {
 static std::atomic<uint64_t> g_launches{0};
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+int device_sm_count() {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        v <= 0) {
+        (void)cudaGetLastError();
+        return 148;
+    }
+    return v;
+}
+
 namespace {
 
-constexpr int kNumSMs = 148;           // B200
 constexpr int kAutoPartition = 512;    // tokens per partition when splitting
 constexpr int kMaxGridYZ = 65535;
 
@@ -61,7 +71,7 @@ int plan_partition(int num_seqs, int num_kv_heads, int block_size,
                                block_size);
     if (max_context_len <= kAutoPartition) return whole;
     const long long units = (long long)num_seqs * num_kv_heads;
-    if (units >= 4LL * kNumSMs) return whole;
+    if (units >= 4LL * device_sm_count()) return whole;
     int part = round_up(kAutoPartition, block_size);
     while ((max_context_len + part - 1) / part > kMaxGridYZ) part *= 2;
     return part;
@@ -72,14 +82,55 @@ int num_partitions(int max_context_len, int part) {
     return n < 1 ? 1 : n;
 }
 
-size_t workspace_bytes_for(int num_seqs, int num_heads, int head_size,
-                           int max_partitions) {
-    if (max_partitions <= 1) return 0;
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Split-KV scratch, each region 256-byte aligned: the partition slots
+// tmp_o [B][Hq][P][D], tmp_m, tmp_l [B][Hq][P]; the persistent grid's
+// straddle rows st_o [Hq][n][D], st_m, st_l [Hq][n] (n = range workers per
+// kv head); the chunk prefix [B+1] and the workers' range starts [n+1].
+struct SplitLayout {
+    size_t o, m, l, st_o, st_m, st_l, prefix, bounds, total;
+    int range_workers;
+};
+
+SplitLayout split_layout(int num_seqs, int num_heads, int num_kv_heads,
+                         int head_size, int max_partitions) {
+    SplitLayout L{};
+    L.range_workers = decode_range_workers(num_kv_heads);
+    if (max_partitions <= 1) return L;
     const size_t rows = (size_t)num_seqs * num_heads * max_partitions;
-    size_t bytes = rows * (size_t)head_size * 4;  // tmp_o
-    bytes = (bytes + 255) & ~(size_t)255;
-    bytes += ((rows * 4 + 255) & ~(size_t)255) * 2;  // tmp_m, tmp_l
-    return bytes;
+    const size_t st_rows = (size_t)num_heads * L.range_workers;
+    size_t off = 0;
+    L.o = off;      off = align256(off + rows * head_size * 4);
+    L.m = off;      off = align256(off + rows * 4);
+    L.l = off;      off = align256(off + rows * 4);
+    L.st_o = off;   off = align256(off + st_rows * head_size * 4);
+    L.st_m = off;   off = align256(off + st_rows * 4);
+    L.st_l = off;   off = align256(off + st_rows * 4);
+    L.prefix = off; off = align256(off + ((size_t)num_seqs + 1) * 4);
+    L.bounds = off; off = align256(off + ((size_t)L.range_workers + 1) * 4);
+    L.total = off;
+    return L;
+}
+
+size_t workspace_bytes_for(int num_seqs, int num_heads, int num_kv_heads,
+                           int head_size, int max_partitions) {
+    return split_layout(num_seqs, num_heads, num_kv_heads, head_size,
+                        max_partitions).total;
+}
+
+// Point the decode parameters at the split scratch inside `ws`.
+void assign_split(DecodeParams& p, unsigned char* ws, const SplitLayout& L) {
+    p.max_range_workers = L.range_workers;
+    if (L.total == 0) return;
+    p.tmp_o = reinterpret_cast<float*>(ws + L.o);
+    p.tmp_m = reinterpret_cast<float*>(ws + L.m);
+    p.tmp_l = reinterpret_cast<float*>(ws + L.l);
+    p.st_o = reinterpret_cast<float*>(ws + L.st_o);
+    p.st_m = reinterpret_cast<float*>(ws + L.st_m);
+    p.st_l = reinterpret_cast<float*>(ws + L.st_l);
+    p.chunk_prefix = reinterpret_cast<int32_t*>(ws + L.prefix);
+    p.worker_bounds = reinterpret_cast<int32_t*>(ws + L.bounds);
 }
 
 // Shared-prefix call: the decode split's scratch, then one flag per
@@ -88,11 +139,11 @@ struct PrefixLayout {
     size_t done_off, total;
 };
 
-PrefixLayout prefix_layout(int num_seqs, int num_heads, int head_size,
-                           int max_partitions) {
+PrefixLayout prefix_layout(int num_seqs, int num_heads, int num_kv_heads,
+                           int head_size, int max_partitions) {
     PrefixLayout L;
-    L.done_off = (workspace_bytes_for(num_seqs, num_heads, head_size,
-                                      max_partitions) + 255) & ~(size_t)255;
+    L.done_off = align256(workspace_bytes_for(num_seqs, num_heads, num_kv_heads,
+                                              head_size, max_partitions));
     L.total = L.done_off + (((size_t)num_seqs * 4 + 255) & ~(size_t)255);
     return L;
 }
@@ -169,7 +220,7 @@ size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
                                               head_size, block_size,
                                               max_context_len, partition_size);
     if (part <= 0 || num_heads <= 0 || head_size <= 0) return 0;
-    return pa::workspace_bytes_for(num_seqs, num_heads, head_size,
+    return pa::workspace_bytes_for(num_seqs, num_heads, num_kv_heads, head_size,
                                    pa::num_partitions(max_context_len, part));
 }
 
@@ -210,8 +261,9 @@ int pa_decode_attention(float* out, const void* q, const void* k_cache,
                                         max_context_len, partition_size);
     const int np = pa::num_partitions(max_context_len, part);
     if (np > pa::kMaxGridYZ) return PA_ERR_INVALID_ARG;
-    const size_t need =
-        pa::workspace_bytes_for(num_seqs, num_heads, head_size, np);
+    const pa::SplitLayout lay =
+        pa::split_layout(num_seqs, num_heads, num_kv_heads, head_size, np);
+    const size_t need = lay.total;
     if (need > 0) {
         if (!workspace || workspace_bytes < need) return PA_ERR_WORKSPACE;
         if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
@@ -225,15 +277,7 @@ int pa_decode_attention(float* out, const void* q, const void* k_cache,
     p.v_cache = static_cast<const uint16_t*>(v_cache);
     p.block_tables = block_tables;
     p.context_lens = context_lens;
-    if (need > 0) {
-        const size_t rows = (size_t)num_seqs * num_heads * np;
-        unsigned char* ws = static_cast<unsigned char*>(workspace);
-        const size_t o_bytes = (rows * head_size * 4 + 255) & ~(size_t)255;
-        const size_t s_bytes = (rows * 4 + 255) & ~(size_t)255;
-        p.tmp_o = reinterpret_cast<float*>(ws);
-        p.tmp_m = reinterpret_cast<float*>(ws + o_bytes);
-        p.tmp_l = reinterpret_cast<float*>(ws + o_bytes + s_bytes);
-    }
+    pa::assign_split(p, static_cast<unsigned char*>(workspace), lay);
     p.error_flags = error_flags;
     p.num_seqs = num_seqs;
     p.max_blocks_per_seq = max_blocks_per_seq;
@@ -363,7 +407,7 @@ size_t pa_shared_prefix_workspace_size(int num_seqs, int num_heads,
                                               head_size, block_size,
                                               max_context_len, partition_size);
     if (part <= 0 || num_heads <= 0 || head_size <= 0) return 0;
-    return pa::prefix_layout(num_seqs, num_heads, head_size,
+    return pa::prefix_layout(num_seqs, num_heads, num_kv_heads, head_size,
                              pa::num_partitions(max_context_len, part)).total;
 }
 
@@ -409,7 +453,8 @@ int pa_decode_attention_shared_prefix(
                                         max_context_len, partition_size);
     const int np = pa::num_partitions(max_context_len, part);
     if (np > pa::kMaxGridYZ) return PA_ERR_INVALID_ARG;
-    const pa::PrefixLayout lay = pa::prefix_layout(num_seqs, num_heads, head_size, np);
+    const pa::PrefixLayout lay =
+        pa::prefix_layout(num_seqs, num_heads, num_kv_heads, head_size, np);
     if (!workspace || workspace_bytes < lay.total) return PA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PA_ERR_INVALID_ARG;
     unsigned char* ws = static_cast<unsigned char*>(workspace);
@@ -456,14 +501,8 @@ int pa_decode_attention_shared_prefix(
     p.v_cache = static_cast<const uint16_t*>(v_cache);
     p.block_tables = block_tables;
     p.context_lens = context_lens;
-    if (np > 1) {
-        const size_t rows = (size_t)num_seqs * num_heads * np;
-        const size_t o_bytes = (rows * head_size * 4 + 255) & ~(size_t)255;
-        const size_t s_bytes = (rows * 4 + 255) & ~(size_t)255;
-        p.tmp_o = reinterpret_cast<float*>(ws);
-        p.tmp_m = reinterpret_cast<float*>(ws + o_bytes);
-        p.tmp_l = reinterpret_cast<float*>(ws + o_bytes + s_bytes);
-    }
+    pa::assign_split(p, ws, pa::split_layout(num_seqs, num_heads, num_kv_heads,
+                                              head_size, np));
     p.error_flags = error_flags;
     p.num_seqs = num_seqs;
     p.max_blocks_per_seq = max_blocks_per_seq;

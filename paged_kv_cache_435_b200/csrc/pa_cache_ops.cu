@@ -112,7 +112,7 @@ cudaError_t launch_reshape_and_cache(const void* key, const void* value,
                          (vec ? head_size / 8 : head_size);
     const int threads = 256;
     int64_t blocks = (work + threads - 1) / threads;
-    const int64_t cap = 148LL * 8;  // grid-stride beyond 8 CTAs per SM
+    const int64_t cap = 8LL * device_sm_count();  // grid-stride beyond 8 CTAs per SM
     if (blocks > cap) blocks = cap;
     const int64_t num_slots = (int64_t)num_blocks * block_size;
     auto* k = static_cast<const uint16_t*>(key);

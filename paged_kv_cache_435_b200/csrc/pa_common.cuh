@@ -20,6 +20,11 @@ namespace pa {
 // Process-wide launch counter (pa_api.cu).
 void count_launch();
 
+// Streaming multiprocessors of the current device (cudaDevAttrMultiProcessorCount;
+// 148 on B200, the value assumed when no device answers, e.g. on a host
+// without a GPU asking for a plan).  pa_api.cu.
+int device_sm_count();
+
 // Upper bound on a single mbarrier wait before the kernel gives up and
 // reports PA_DEVERR_TIMEOUT (nanoseconds of %globaltimer).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
@@ -72,14 +77,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for phase `parity` of `bar`.  Returns false after
-// kWaitLimitNs without completion (the caller reports and bails out).
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar,
-                                                  uint32_t parity) {
+// `limit_ns` without completion (the caller reports and bails out).
+__device__ __forceinline__ bool mbar_wait_bounded(
+    uint64_t* bar, uint32_t parity,
+    unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0u && global_timer_ns() - t0 > kWaitLimitNs)
+        if ((it & 63u) == 0u && global_timer_ns() - t0 > limit_ns)
             return false;
     }
 }

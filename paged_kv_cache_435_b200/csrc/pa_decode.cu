@@ -52,8 +52,17 @@ constexpr int kChunk = 16;          // tokens per pipeline stage
 constexpr int kMaxGroup = 8;
 constexpr int kMaxPersistSeqs = 768;
 constexpr int kTargetCtasPerSM = 2;
-constexpr int kNumSMs = 148;
 constexpr float kLog2e = 1.4426950408889634f;
+
+#ifdef PA_TEST_UNSIGNALLED_FIRST_WAIT
+// Test build only (libpagedattn_waittest.so, never the product library):
+// every warp's first chunk wait polls a spare barrier that nothing arrives
+// on, so it runs out after this limit and the kernel takes its timeout path
+// (report PA_DEVERR_TIMEOUT, skip the rest, drain the copies already issued
+// with the full limit).  This is how a test makes a bounded wait expire
+// without any GPU fault.
+constexpr unsigned long long kTestWaitLimitNs = 20000000ull;  // 20 ms
+#endif
 
 template <int D>
 struct Cfg {
@@ -63,12 +72,15 @@ struct Cfg {
     static constexpr int kStageBytes = 2 * kKVBytes;
     static constexpr int kStages = D == 128 ? 3 : 5;
     static constexpr int kRingBytes = kWarps * kStages * kStageBytes;
+    // Item-end exchange: warps 1..3 post their partial O rows for warp 0.
     static constexpr int kRedStride = D + 8;                // floats per row
     static constexpr int kRedOBytes = (kWarps - 1) * kMaxGroup * kRedStride * 4;
     static constexpr int kRedMLBytes = kWarps * kMaxGroup * 2 * 4;
     static constexpr int kRedOff = kRingBytes;
     static constexpr int kBarOff = kRedOff + kRedOBytes + kRedMLBytes;
-    static constexpr int kBarBytes = (kWarps * kStages * 8 + 127) / 128 * 128;
+    // One barrier per stage and warp, plus one spare per warp (used only by
+    // the wait-timeout test build, below).
+    static constexpr int kBarBytes = (kWarps * (kStages + 1) * 8 + 127) / 128 * 128;
     static constexpr int kPrefixOff = kBarOff + kBarBytes;
     static constexpr int kSmemGrid = kPrefixOff;
     static constexpr int kSmemPersist = kPrefixOff + (kMaxPersistSeqs + 1) * 4;
@@ -77,13 +89,19 @@ struct Cfg {
                   "two CTAs per SM must fit");
 };
 
+// A piece of work: tokens [tok0, tok1) of sequence s for one kv head, and
+// where its result goes.
+enum PieceKind { kWhole = 0, kSlot = 1, kStraddle = 2 };
+
 struct Item {
     int s;       // sequence; -1 = no item
-    int part;    // partition index
     int L;       // context length (clamped)
-    int tok0;    // first token of the partition
-    int tok1;    // one past its last token
-    int nparts;  // partitions of this sequence
+    int tok0;    // first token
+    int tok1;    // one past the last token
+    int x1;      // persistent grid: chunk position one past the piece
+    int kind;    // kWhole: the sequence's output; kSlot: partition idx's
+                 // partial; kStraddle: the partial in this CTA's straddle row
+    int idx;
 };
 
 __device__ __forceinline__ int clamped_len(const DecodeParams& p, int s) {
@@ -105,47 +123,115 @@ __device__ __forceinline__ bool skipped(const DecodeParams& p, int s) {
     return kSkip && p.skip_seq[s] != 0;
 }
 
-// Item k of this CTA (k = 0, 1, ...).
-template <bool kPersist, bool kSkip>
-__device__ __forceinline__ Item get_item(const DecodeParams& p,
-                                         const int* prefix, int k) {
+// ---------------------------------------------------------------- plain grid
+// One CTA per (kv head, partition, sequence); a partition past the
+// sequence's end has no item.
+__device__ __forceinline__ Item grid_item(const DecodeParams& p, int s, int part,
+                                          bool skip) {
     Item it;
     it.s = -1;
-    int s, part;
-    if (kPersist) {
-        const int j = blockIdx.y + k * gridDim.y;
-        if (j >= prefix[p.num_seqs]) return it;
-        int lo = 0, hi = p.num_seqs - 1;  // largest s with prefix[s] <= j
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (prefix[mid] <= j) lo = mid; else hi = mid - 1;
-        }
-        s = lo;
-        part = j - prefix[s];
-    } else {
-        if (k > 0) return it;
-        s = blockIdx.z;
-        part = blockIdx.y;
-    }
-    if (skipped<kSkip>(p, s)) return it;
+    if (skip) return it;
     const int L = clamped_len(p, s);
     const int np = parts_of(L, p.partition_size);
     if (part >= np) return it;
     it.s = s;
-    it.part = part;
     it.L = L;
-    it.nparts = np;
     it.tok0 = part * p.partition_size;
     it.tok1 = min(L, it.tok0 + p.partition_size);
+    it.x1 = 0;
+    it.kind = np == 1 ? kWhole : kSlot;
+    it.idx = part;
     return it;
 }
 
-// Chunks of `it` that warp w owns.
+// ---------------------------------------------------------- persistent grid
+// Per kv head the 16-token chunks of all (not skipped) sequences lie end to
+// end: sequence s occupies chunk positions [X[s], X[s+1]), T = X[B] in all.
+// Split (max_partitions > 1): each warp of the head's CTAs is a range worker;
+// worker i of the head's n takes positions [floor(i T/n), floor((i+1) T/n)),
+// so every worker streams the same amount to within one chunk, and streams
+// it alone: no warp of the CTA ever waits for another.  Its range is cut
+// into pieces at sequence ends and at partition starts (every partition_size
+// tokens of a sequence), so a partial never spans two partitions: a piece
+// that starts a partition writes that partition's slot, the piece a worker
+// starts in the middle of a partition writes the worker's straddle row, and
+// a piece holding a whole sequence writes the output.  No split (the
+// shared-prefix call's per-sequence pass): each CTA is one worker whose four
+// warps share its items, and its range is the sequences whose first chunk
+// lies in [floor(b T/n), floor((b+1) T/n)), taken whole.
+struct Range {
+    int r0, r1;   // chunk positions [r0, r1)
+    int q;        // chunks per partition
+    int worker;   // straddle row of a piece that starts mid-partition
+};
+
+// Largest s with X[s] <= x (x < X[B]): the sequence holding chunk x.
+__device__ __forceinline__ int seq_at(const int* X, int B, int x) {
+    int lo = 0, hi = B - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (X[mid] <= x) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Smallest sequence start X[s] >= x (X[B] if none).
+__device__ __forceinline__ int seq_start_at_or_after(const int* X, int B, int x) {
+    int lo = 0, hi = B;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (X[mid] >= x) hi = mid; else lo = mid + 1;
+    }
+    return X[lo];
+}
+
+__device__ __forceinline__ Item piece_at(const DecodeParams& p, const int* X,
+                                         const Range& r, int x0) {
+    Item it;
+    it.s = -1;
+    if (x0 >= r.r1) return it;
+    const int s = seq_at(X, p.num_seqs, x0);
+    const int xs = X[s];
+    const int cs = X[s + 1] - xs;
+    const int o0 = x0 - xs;
+    const int k = o0 / r.q;
+    const int pend = xs + min(cs, (k + 1) * r.q);
+    it.s = s;
+    it.L = clamped_len(p, s);
+    it.x1 = min(pend, r.r1);
+    it.tok0 = o0 * kChunk;
+    it.tok1 = min(it.L, (it.x1 - xs) * kChunk);
+    if (o0 == 0 && it.x1 == xs + cs) {
+        it.kind = kWhole;
+        it.idx = 0;
+    } else if (o0 % r.q == 0) {
+        it.kind = kSlot;
+        it.idx = k;
+    } else {
+        it.kind = kStraddle;  // only a range's first piece starts mid-partition
+        it.idx = r.worker;
+    }
+    return it;
+}
+
+// Chunks of `it` that warp w owns: all of them when the warp is a range
+// worker, else chunks w, w+4, w+8, ... (the CTA's four warps share the item).
+template <bool kWarpRanges>
 __device__ __forceinline__ int warp_chunks(const Item& it, int warp) {
     if (it.s < 0) return 0;
     const int n = (it.tok1 - it.tok0 + kChunk - 1) / kChunk;
+    if (kWarpRanges) return n;
     return n > warp ? (n - warp + kWarps - 1) / kWarps : 0;
 }
+
+// First token of the i-th chunk that warp w owns in `it`.
+template <bool kWarpRanges>
+__device__ __forceinline__ int chunk_token(const Item& it, int warp, int i) {
+    return it.tok0 + (kWarpRanges ? i : warp + kWarps * i) * kChunk;
+}
+
+// Grid shapes of the partition kernel.
+enum DecodeMode { kModeGrid = 0, kModeCtaRanges = 1, kModeWarpRanges = 2 };
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map,
                                             int c0, int c1, int c2,
@@ -165,19 +251,21 @@ __device__ __forceinline__ void named_bar_arrive(int id) {
     asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(kThreads) : "memory");
 }
 
-template <int D, int BS, bool kPersist, bool kSkip>
+template <int D, int BS, int kMode, bool kSkip>
 __global__ void __launch_bounds__(kThreads, kTargetCtasPerSM)
 paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
                     const DecodeParams p) {
     using C = Cfg<D>;
+    constexpr bool kPersist = kMode != kModeGrid;
+    constexpr bool kWarpRanges = kMode == kModeWarpRanges;
     extern __shared__ __align__(1024) unsigned char smem[];
     unsigned char* ring = smem;
     float* red_o = reinterpret_cast<float*>(smem + C::kRedOff);
     float* red_m = red_o + (kWarps - 1) * kMaxGroup * C::kRedStride;
     float* red_l = red_m + kWarps * kMaxGroup;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
-    int* prefix = reinterpret_cast<int*>(smem + C::kPrefixOff);
+    int* X = reinterpret_cast<int*>(smem + C::kPrefixOff);
 
     const int g = blockIdx.x;  // kv head
     const int warp = threadIdx.x >> 5;
@@ -195,17 +283,18 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
     pdl_wait();
     pdl_launch_dependents();
 
+    Range rg{0, 0, 1, 0};
     if (kPersist) {
-        // prefix[s] = partitions of sequences 0..s-1 (block-wide scan).  The
+        // X[s] = 16-token chunks of sequences 0..s-1 (block-wide scan).  The
         // merge area is free until the first item ends; it holds the warp sums.
         int* warp_tot = reinterpret_cast<int*>(red_l);
         int running = 0;
-        if (threadIdx.x == 0) prefix[0] = 0;
+        if (threadIdx.x == 0) X[0] = 0;
         for (int base = 0; base < p.num_seqs; base += kThreads) {
             const int s = base + threadIdx.x;
             int v = 0;
             if (s < p.num_seqs && !skipped<kSkip>(p, s))
-                v = parts_of(clamped_len(p, s), p.partition_size);
+                v = (clamped_len(p, s) + kChunk - 1) / kChunk;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int t = __shfl_up_sync(0xffffffffu, v, o);
@@ -215,16 +304,53 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
             __syncthreads();
             int before = running;
             for (int w = 0; w < warp; ++w) before += warp_tot[w];
-            if (s < p.num_seqs) prefix[s + 1] = before + v;
+            if (s < p.num_seqs) X[s + 1] = before + v;
             for (int w = 0; w < kWarps; ++w) running += warp_tot[w];
             __syncthreads();
         }
+        const long long T = X[p.num_seqs];
+        rg.q = p.partition_size / kChunk;
+        if (kWarpRanges) {
+            const long long n = (long long)gridDim.y * kWarps;
+            rg.worker = blockIdx.y * kWarps + warp;
+            rg.r0 = (int)(rg.worker * T / n);
+            rg.r1 = (int)((rg.worker + 1) * T / n);
+            // The merge kernel finds the pieces of a sequence from the same
+            // scan and the same ranges.
+            if (g == 0 && blockIdx.y == 0) {
+                for (int s = threadIdx.x; s <= p.num_seqs; s += kThreads)
+                    p.chunk_prefix[s] = X[s];
+                for (int i = threadIdx.x; i <= n; i += kThreads)
+                    p.worker_bounds[i] = (int)(i * T / n);
+            }
+        } else {
+            const long long n = gridDim.y;
+            const int b = blockIdx.y;
+            rg.worker = b;
+            rg.r0 = seq_start_at_or_after(X, p.num_seqs, (int)(b * T / n));
+            rg.r1 = seq_start_at_or_after(X, p.num_seqs, (int)((b + 1) * T / n));
+        }
     }
+    // Items of this CTA, as a chain: key = chunk position of the piece's
+    // start (persistent grid) or 0 / 1 = the CTA's one item / none (plain
+    // grid).
+    auto item_at = [&](int key) -> Item {
+        if (kPersist) return piece_at(p, X, rg, key);
+        Item none;
+        none.s = -1;
+        if (key != 0) return none;
+        return grid_item(p, blockIdx.z, blockIdx.y, skipped<kSkip>(p, blockIdx.z));
+    };
+    auto next_key = [&](const Item& it) -> int { return kPersist ? it.x1 : 1; };
+    const int first_key = kPersist ? rg.r0 : 0;
 
     uint64_t* my_bars = bars + warp * C::kStages;
     unsigned char* my_ring = ring + warp * C::kStages * C::kStageBytes;
     if (lane == 0) {
         for (int i = 0; i < C::kStages; ++i) mbar_init(&my_bars[i], 1);
+#ifdef PA_TEST_UNSIGNALLED_FIRST_WAIT
+        mbar_init(&bars[kWarps * C::kStages + warp], 1);
+#endif
         mbar_init_fence();
     }
     __syncthreads();  // barriers initialised, prefix visible
@@ -239,30 +365,30 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
     const float sl2 = p.scale_log2;
 
     // ---------------- producer state (this warp's chunk stream) ----------
-    int prod_k = 0;        // item of the next chunk to look up
-    int prod_i = 0;        // warp-chunk index within that item
-    int prod_count = 0;    // chunks issued so far
-    int ids_base = 0;      // prod_count at the last refill
-    int ids = -1;          // lane l: slot coordinate of chunk ids_base + l
+    int prod_key = first_key;  // item of the next chunk to look up
+    int prod_i = 0;            // warp-chunk index within that item
+    int prod_count = 0;        // chunks issued so far
+    int ids_base = 0;          // prod_count at the last refill
+    int ids = -1;              // lane l: slot coordinate of chunk ids_base + l
     bool prod_done = false;
 
     // Lane l finds the (ids_base + l)-th chunk of the stream and its slot.
     auto refill = [&]() {
-        int k = prod_k, i = prod_i, n = lane;
-        Item it = get_item<kPersist, kSkip>(p, prefix, k);
+        int key = prod_key, i = prod_i, n = lane;
+        Item it = item_at(key);
         for (;;) {
             if (it.s < 0) break;
-            const int rem = warp_chunks(it, warp) - i;
+            const int rem = warp_chunks<kWarpRanges>(it, warp) - i;
             if (rem > n) break;
             n -= rem > 0 ? rem : 0;
-            ++k;
+            key = next_key(it);
             i = 0;
-            it = get_item<kPersist, kSkip>(p, prefix, k);
+            it = item_at(key);
         }
         int slot = -1;
         if (it.s >= 0) {
             i += n;
-            const int ctok = it.tok0 + (warp + kWarps * i) * kChunk;
+            const int ctok = chunk_token<kWarpRanges>(it, warp, i);
             int id = tables[(int64_t)it.s * p.max_blocks_per_seq + ctok / BS];
             if (id < 0 || id >= p.num_blocks) {
                 report(p.error_flags, PA_DEVERR_BLOCK_ID);
@@ -273,7 +399,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         }
         ids = slot;
         ids_base = prod_count;
-        prod_k = __shfl_sync(0xffffffffu, k, 31);
+        prod_key = __shfl_sync(0xffffffffu, key, 31);
         prod_i = __shfl_sync(0xffffffffu, i, 31);
         prod_done = __shfl_sync(0xffffffffu, slot, 31) < 0;
     };
@@ -311,7 +437,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
     int cons_count = 0;
     bool aborted = false;
     int drain_from = 0;  // first chunk whose wait gave up
-    int k = 0;
+    int items_done = 0;
     // Q fragments of an item (A operand): rows = heads of the group, rows >= G
     // zero.  The next item's are fetched while the current one streams.
     auto load_q = [&](const Item& it, uint32_t (&dst)[D / 16][2]) {
@@ -324,20 +450,20 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
             dst[ks][1] = live ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8 + qc) : 0u;
         }
     };
-    Item next_it = get_item<kPersist, kSkip>(p, prefix, 0);
+    Item next_it = item_at(first_key);
     uint32_t qnext[D / 16][2];
     load_q(next_it, qnext);
-    for (;; ++k) {
+    for (;;) {
         const Item it = next_it;
         if (it.s < 0) break;
-        const int my_n = warp_chunks(it, warp);
+        const int my_n = warp_chunks<kWarpRanges>(it, warp);
         uint32_t qa[D / 16][2];
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
             qa[ks][0] = qnext[ks][0];
             qa[ks][1] = qnext[ks][1];
         }
-        next_it = get_item<kPersist, kSkip>(p, prefix, k + 1);
+        next_it = item_at(next_key(it));
         load_q(next_it, qnext);
 
         float o[D / 8][4];
@@ -349,8 +475,16 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         for (int i = 0; i < my_n; ++i) {
             const int stage = cons_count % C::kStages;
             if (!aborted) {
+#ifdef PA_TEST_UNSIGNALLED_FIRST_WAIT
+                const bool ok =
+                    cons_count == 0
+                        ? mbar_wait_bounded(&bars[kWarps * C::kStages + warp], 0,
+                                            kTestWaitLimitNs)
+                        : mbar_wait_bounded(&my_bars[stage], (cons_count / C::kStages) & 1);
+#else
                 const bool ok = mbar_wait_bounded(&my_bars[stage],
                                                   (cons_count / C::kStages) & 1);
+#endif
                 if (!__all_sync(0xffffffffu, ok)) {
                     aborted = true;
                     drain_from = cons_count;
@@ -360,7 +494,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
             ++cons_count;
             if (aborted) continue;
 
-            const int ctok = it.tok0 + (warp + kWarps * i) * kChunk;
+            const int ctok = chunk_token<kWarpRanges>(it, warp, i);
             const int valid = min(kChunk, it.tok1 - ctok);
             const uint32_t kaddr = smem_u32(my_ring + stage * C::kStageBytes);
             const uint32_t vaddr = kaddr + C::kKVBytes;
@@ -457,11 +591,45 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
             if (!prod_done || prod_count < ids_base + 32) issue();
         }
 
-        // ---------------- item end: merge the four warps ----------------
         l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
         l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+        if (kWarpRanges) {
+            // ------------- item end of a range worker: its own result ---
+            // Rows qr (the head) and qr + 8 (the P residual's share) add up;
+            // the quad's lanes hold the row's columns 8j + qc, +1.
+            if (qr < G) {
+                const int h = g * G + qr;
+                const int64_t row = (int64_t)it.s * Hq + h;
+                int64_t pidx = 0;
+                float* dst;
+                if (it.kind == kWhole) {
+                    dst = p.out + row * D;
+                } else if (it.kind == kSlot) {
+                    pidx = row * p.max_partitions + it.idx;
+                    dst = p.tmp_o + pidx * D;
+                } else {
+                    pidx = (int64_t)h * p.max_range_workers + it.idx;
+                    dst = p.st_o + pidx * D;
+                }
+                const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll
+                for (int j = 0; j < D / 8; ++j)
+                    *reinterpret_cast<float2*>(dst + 8 * j + qc) =
+                        make_float2((o[j][0] + o[j][2]) * inv, (o[j][1] + o[j][3]) * inv);
+                if (it.kind != kWhole && (lane & 3) == 0) {
+                    float* dm = it.kind == kSlot ? p.tmp_m : p.st_m;
+                    float* dl = it.kind == kSlot ? p.tmp_l : p.st_l;
+                    dm[pidx] = m_run;
+                    dl[pidx] = l_run;
+                }
+            }
+            continue;
+        }
+        // ---------------- item end: merge the four warps ----------------
+        // Warps 1..3 post (max, sum, O) and go on streaming; warp 0 merges
+        // and writes the result, so only warp 0 pauses its copy ring.
         if (warp != 0) {
-            if (k > 0) named_bar_sync(2);  // warp 0 has read the previous item
+            if (items_done > 0) named_bar_sync(2);  // warp 0 has read the previous item
             float* dst = red_o + ((warp - 1) * kMaxGroup + qr) * C::kRedStride + qc;
 #pragma unroll
             for (int j = 0; j < D / 8; ++j)
@@ -487,10 +655,18 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
             }
             if (qr < G) {
                 const int h = g * G + qr;
-                const bool direct = it.nparts == 1;
                 const int64_t row = (int64_t)it.s * Hq + h;
-                const int64_t idx = row * p.max_partitions + it.part;
-                float* dst = direct ? p.out + row * D : p.tmp_o + idx * D;
+                int64_t pidx = 0;
+                float* dst;
+                if (it.kind == kWhole) {
+                    dst = p.out + row * D;
+                } else if (it.kind == kSlot) {
+                    pidx = row * p.max_partitions + it.idx;
+                    dst = p.tmp_o + pidx * D;
+                } else {
+                    pidx = (int64_t)h * p.max_range_workers + it.idx;
+                    dst = p.st_o + pidx * D;
+                }
 #pragma unroll
                 for (int j = 0; j < D / 8; ++j) {
                     float v[2];
@@ -504,16 +680,29 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                     }
                     *reinterpret_cast<float2*>(dst + 8 * j + qc) = make_float2(v[0], v[1]);
                 }
-                if (!direct && (lane & 3) == 0) {
-                    p.tmp_m[idx] = M;
-                    p.tmp_l[idx] = den;
+                if (it.kind != kWhole && (lane & 3) == 0) {
+                    float* dm = it.kind == kSlot ? p.tmp_m : p.st_m;
+                    float* dl = it.kind == kSlot ? p.tmp_l : p.st_l;
+                    dm[pidx] = M;
+                    dl[pidx] = den;
                 }
             }
             named_bar_arrive(2);
         }
+        ++items_done;
     }
     // Consume warp 0's last "merged" arrival so no barrier is left pending.
-    if (warp != 0 && k > 0) named_bar_sync(2);
+    if (warp != 0 && items_done > 0) named_bar_sync(2);
+
+    if (kPersist) {
+        // Sequences with an empty context (not skipped) own no chunk: their
+        // output is zero, written by the CTAs of the head in turn.
+        for (int s = blockIdx.y; s < p.num_seqs; s += gridDim.y) {
+            if (skipped<kSkip>(p, s) || X[s + 1] != X[s]) continue;
+            for (int e = threadIdx.x; e < G * D; e += kThreads)
+                p.out[((int64_t)s * Hq + g * G) * D + e] = 0.f;
+        }
+    }
 
     if (aborted) {
         // Drain copies still in flight on this warp's ring (bounded) before
@@ -523,12 +712,17 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
     }
 }
 
-// Merge of the per-partition results: out = sum_p w_p o_p / sum_p w_p with
-// w_p = l_p * 2^(m_p - max_p m_p).  One CTA of 8 warps per (query head,
-// sequence); warp w takes partitions w, w+8, ... with 8 partitions' rows in
-// flight per round, each lane holding D/32 consecutive columns.
+// Merge of the pieces of a split sequence: out = sum_i w_i o_i / sum_i w_i
+// with w_i = l_i * 2^(m_i - max_j m_j), over the sequence's partition slots
+// and, on the persistent grid, the straddle rows of the range workers whose
+// ranges begin inside one of its partitions.  One CTA of 8 warps per (query head,
+// sequence); warp w takes pieces w, w+8, ..., 16 pieces' rows in flight per
+// round, each lane holding D/32 consecutive columns, with a running max so
+// every round is one memory round trip; the warps combine through shared
+// memory.  Sequences held whole by one piece were written by the partition
+// kernel.
 constexpr int kReduceWarps = 8;
-constexpr int kReduceUnroll = 8;
+constexpr int kReduceUnroll = 16;
 
 template <int D>
 __global__ void __launch_bounds__(kReduceWarps * 32)
@@ -539,73 +733,122 @@ paged_decode_reduce_kernel(const DecodeParams p) {
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     pdl_wait();  // the partials come from the grid launched just before
+    if (p.skip_seq != nullptr && p.skip_seq[s] != 0) return;  // answered elsewhere
     int L = p.context_lens[s];
     L = L < 0 ? 0 : (L > p.max_context_len ? p.max_context_len : L);
-    if (p.skip_seq != nullptr && p.skip_seq[s] != 0) return;  // answered elsewhere
-    const int np = (L + p.partition_size - 1) / p.partition_size;
-    if (np <= 1) return;  // written directly by the partition kernel
-    const int64_t base = ((int64_t)s * p.num_heads + h) * p.max_partitions;
 
-    __shared__ float warp_max[kReduceWarps];
-    __shared__ float part_acc[kReduceWarps][D];
+    // Pieces: partition slots 0..nslot-1, then candidate straddle rows
+    // b_lo..b_lo+ncand-1 (persistent grid only): the range boundaries
+    // strictly inside the sequence's chunks.  A candidate holds a piece when
+    // its boundary is not a partition start and it is the last worker
+    // starting at that position (earlier ones have empty ranges).
+    int nslot, b_lo = 0, ncand = 0, xs = 0, q = 1;
+    const int32_t* E = p.worker_bounds;
+    if (p.range_workers > 0) {
+        const int cs = (L + kChunk - 1) / kChunk;
+        if (cs == 0) return;  // empty: zeros written by the partition kernel
+        q = p.partition_size / kChunk;
+        nslot = (cs + q - 1) / q;
+        xs = p.chunk_prefix[s];
+        const long long T = p.chunk_prefix[p.num_seqs];
+        const long long n = p.range_workers;
+        // floor(b T / n) > xs  <=>  b >= ceil((xs + 1) n / T);
+        // floor(b T / n) < xs + cs  <=>  b <= ceil((xs + cs) n / T) - 1.
+        const long long lo = ((xs + 1) * n + T - 1) / T;
+        const long long hi = ((xs + cs) * n + T - 1) / T - 1;
+        b_lo = (int)max(1LL, lo);
+        ncand = max(0, (int)min(n - 1, hi) - b_lo + 1);
+    } else {
+        nslot = (L + p.partition_size - 1) / p.partition_size;
+    }
+    auto straddle = [&](int b) -> bool {
+        const int e = E[b];
+        return (e - xs) % q != 0 && E[b + 1] > e;
+    };
+    int nstr = 0;
+    for (int c = lane; c < ncand; c += 32)
+        nstr += straddle(b_lo + c) ? 1 : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) nstr += __shfl_xor_sync(0xffffffffu, nstr, o);
+    if (nslot + nstr <= 1) return;  // written directly by the partition kernel
+    const int total = nslot + ncand;
+
+    __shared__ float part_m[kReduceWarps];
     __shared__ float part_den[kReduceWarps];
+    __shared__ float part_acc[kReduceWarps][D];
 
-    float M = -INFINITY;
-    for (int i = threadIdx.x; i < np; i += kReduceWarps * 32)
-        M = fmaxf(M, p.tmp_m[base + i]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    if (lane == 0) warp_max[warp] = M;
-    __syncthreads();
-    M = warp_max[0];
-#pragma unroll
-    for (int w = 1; w < kReduceWarps; ++w) M = fmaxf(M, warp_max[w]);
-
+    const int64_t slot_base = ((int64_t)s * p.num_heads + h) * p.max_partitions;
+    const int64_t st_base = (int64_t)h * p.max_range_workers;
+    float M = -INFINITY, den = 0.f;
     float acc[V];
 #pragma unroll
     for (int v = 0; v < V; ++v) acc[v] = 0.f;
-    float den = 0.f;
-    for (int i0 = warp; i0 < np; i0 += kReduceWarps * kReduceUnroll) {
-        float wts[kReduceUnroll];
-        float vals[kReduceUnroll][V];
-        float lv[kReduceUnroll], mv[kReduceUnroll];
+    for (int i0 = warp; i0 < total; i0 += kReduceWarps * kReduceUnroll) {
+        // Every load of the round is issued before any is used; a row that
+        // is not a piece is read from a valid address and then ignored (the
+        // straddle region may hold an earlier call's values).
+        float mv[kReduceUnroll], lv[kReduceUnroll], vals[kReduceUnroll][V];
+        bool live[kReduceUnroll];
 #pragma unroll
         for (int u = 0; u < kReduceUnroll; ++u) {
-            // Rows past np re-read the last row with weight 0, so every load
-            // of the round is unconditional and in flight together.
-            const int i = min(i0 + u * kReduceWarps, np - 1);
-            lv[u] = p.tmp_l[base + i];
-            mv[u] = p.tmp_m[base + i];
-            const float* row = p.tmp_o + (base + i) * D + lane * V;
+            const int i = i0 + u * kReduceWarps;
+            const bool in_slots = i < nslot;
+            const int b = b_lo + (in_slots ? 0 : min(i - nslot, max(ncand - 1, 0)));
+            live[u] = i < total && (in_slots || straddle(b));
+            const int64_t r = in_slots ? slot_base + i : st_base + b;
+            const float* mrow = in_slots ? p.tmp_m : p.st_m;
+            const float* lrow = in_slots ? p.tmp_l : p.st_l;
+            const float* orow = (in_slots ? p.tmp_o : p.st_o) + r * D + lane * V;
+            const bool ok = i < total;
+            mv[u] = ok ? mrow[r] : -INFINITY;
+            lv[u] = ok ? lrow[r] : 0.f;
             if (V == 4) {
-                const float4 t = *reinterpret_cast<const float4*>(row);
+                const float4 t = ok ? *reinterpret_cast<const float4*>(orow)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
                 vals[u][0] = t.x; vals[u][V > 1 ? 1 : 0] = t.y;
                 vals[u][V > 2 ? 2 : 0] = t.z; vals[u][V > 3 ? 3 : 0] = t.w;
             } else {
-                const float2 t = *reinterpret_cast<const float2*>(row);
+                const float2 t = ok ? *reinterpret_cast<const float2*>(orow)
+                                    : make_float2(0.f, 0.f);
                 vals[u][0] = t.x; vals[u][V > 1 ? 1 : 0] = t.y;
             }
         }
+        float Mr = M;
 #pragma unroll
         for (int u = 0; u < kReduceUnroll; ++u)
-            wts[u] = i0 + u * kReduceWarps < np ? lv[u] * exp2f(mv[u] - M) : 0.f;
+            if (live[u]) Mr = fmaxf(Mr, mv[u]);
+        if (Mr == -INFINITY) continue;
+        const float keep = M == -INFINITY ? 0.f : exp2f(M - Mr);
+        den *= keep;
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[v] *= keep;
 #pragma unroll
         for (int u = 0; u < kReduceUnroll; ++u) {
-            den += wts[u];
+            if (!live[u] || mv[u] == -INFINITY) continue;
+            const float w = lv[u] * exp2f(mv[u] - Mr);
+            den += w;
 #pragma unroll
-            for (int v = 0; v < V; ++v) acc[v] += wts[u] * vals[u][v];
+            for (int v = 0; v < V; ++v) acc[v] += w * vals[u][v];
         }
+        M = Mr;
+    }
+    if (lane == 0) {
+        part_m[warp] = M;
+        part_den[warp] = den;
     }
 #pragma unroll
     for (int v = 0; v < V; ++v) part_acc[warp][lane * V + v] = acc[v];
-    if (lane == 0) part_den[warp] = den;
     __syncthreads();
+    float Mall = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kReduceWarps; ++w) Mall = fmaxf(Mall, part_m[w]);
     for (int d = threadIdx.x; d < D; d += kReduceWarps * 32) {
         float a = 0.f, dn = 0.f;
 #pragma unroll
         for (int w = 0; w < kReduceWarps; ++w) {
-            a += part_acc[w][d];
-            dn += part_den[w];
+            const float sc = part_m[w] == -INFINITY ? 0.f : exp2f(part_m[w] - Mall);
+            a += sc * part_acc[w][d];
+            dn += sc * part_den[w];
         }
         p.out[((int64_t)s * p.num_heads + h) * D + d] = a / dn;
     }
@@ -681,44 +924,56 @@ cudaError_t set_smem(Kernel kernel, int bytes, int* flags) {
     return cudaSuccess;
 }
 
-template <int D, int BS, bool kSkip>
-cudaError_t launch_partition_kernel(const DecodeParams& p, const CUtensorMap& tmk,
-                                    const CUtensorMap& tmv, cudaStream_t stream) {
-    using C = Cfg<D>;
-    static int grid_ready[64] = {0};
-    static int persist_ready[64] = {0};
-    // Persistent CTAs when sequences are split, and when some sequences are
-    // skipped (the compact item list then spends no CTA on them).
-    const bool persist = (p.max_partitions > 1 || kSkip) && p.num_seqs <= kMaxPersistSeqs;
-    cudaError_t e;
-    if (persist) {
-        e = set_smem(paged_decode_kernel<D, BS, true, kSkip>, C::kSmemPersist, persist_ready);
-        if (e != cudaSuccess) return e;
-        long long per_head = (kTargetCtasPerSM * kNumSMs + p.num_kv_heads - 1) / p.num_kv_heads;
-        const long long items = (long long)p.num_seqs * p.max_partitions;
-        if (per_head > items) per_head = items;
-        if (per_head < 1) per_head = 1;
-        dim3 grid((unsigned)p.num_kv_heads, (unsigned)per_head, 1);
-        e = launch_pdl(paged_decode_kernel<D, BS, true, kSkip>, grid, dim3(kThreads),
-                       C::kSmemPersist, stream, tmk, tmv, p);
-    } else {
-        e = set_smem(paged_decode_kernel<D, BS, false, kSkip>, C::kSmemGrid, grid_ready);
-        if (e != cudaSuccess) return e;
-        dim3 grid((unsigned)p.num_kv_heads, (unsigned)p.max_partitions,
-                  (unsigned)p.num_seqs);
-        e = launch_pdl(paged_decode_kernel<D, BS, false, kSkip>, grid, dim3(kThreads),
-                       C::kSmemGrid, stream, tmk, tmv, p);
-    }
+template <int D, int BS, int kMode, bool kSkip>
+cudaError_t launch_mode(const DecodeParams& p, const CUtensorMap& tmk,
+                        const CUtensorMap& tmv, dim3 grid, int smem,
+                        cudaStream_t stream) {
+    static int ready[64] = {0};
+    cudaError_t e = set_smem(paged_decode_kernel<D, BS, kMode, kSkip>, smem, ready);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(paged_decode_kernel<D, BS, kMode, kSkip>, grid, dim3(kThreads),
+                   smem, stream, tmk, tmv, p);
     count_launch();
     return e;
 }
 
+// Persistent CTAs when sequences are split (balanced chunk ranges per warp),
+// and when some sequences are skipped (no CTA is spent on them); up to
+// kMaxPersistSeqs sequences, whose chunk prefix fits in shared memory.
+template <int D, int BS, bool kSkip>
+cudaError_t launch_partition_kernel(DecodeParams& p, const CUtensorMap& tmk,
+                                    const CUtensorMap& tmv, cudaStream_t stream) {
+    using C = Cfg<D>;
+    p.range_workers = 0;
+    const bool split = p.max_partitions > 1;
+    if ((split || kSkip) && p.num_seqs <= kMaxPersistSeqs) {
+        long long per_head = decode_ctas_per_head(p.num_kv_heads);
+        const long long items = (long long)p.num_seqs * p.max_partitions;
+        if (per_head > items) per_head = items;
+        if (split && per_head * kWarps > p.max_range_workers)
+            per_head = p.max_range_workers / kWarps;  // the straddle region's rows
+        if (per_head < 1) per_head = 1;
+        const dim3 grid((unsigned)p.num_kv_heads, (unsigned)per_head, 1);
+        if (split) {
+            p.range_workers = (int)per_head * kWarps;
+            return launch_mode<D, BS, kModeWarpRanges, kSkip>(p, tmk, tmv, grid,
+                                                             C::kSmemPersist, stream);
+        }
+        return launch_mode<D, BS, kModeCtaRanges, kSkip>(p, tmk, tmv, grid,
+                                                        C::kSmemPersist, stream);
+    }
+    const dim3 grid((unsigned)p.num_kv_heads, (unsigned)p.max_partitions,
+                    (unsigned)p.num_seqs);
+    return launch_mode<D, BS, kModeGrid, kSkip>(p, tmk, tmv, grid, C::kSmemGrid, stream);
+}
+
 template <int D, int BS>
-cudaError_t launch_typed(const DecodeParams& p, cudaStream_t stream) {
+cudaError_t launch_typed(const DecodeParams& params, cudaStream_t stream) {
     CUtensorMap tmk, tmv;
-    if (!encode_pool_map(&tmk, p.k_cache, p.num_blocks, BS, p.num_kv_heads, D) ||
-        !encode_pool_map(&tmv, p.v_cache, p.num_blocks, BS, p.num_kv_heads, D))
+    if (!encode_pool_map(&tmk, params.k_cache, params.num_blocks, BS, params.num_kv_heads, D) ||
+        !encode_pool_map(&tmv, params.v_cache, params.num_blocks, BS, params.num_kv_heads, D))
         return cudaErrorInvalidValue;
+    DecodeParams p = params;
     cudaError_t e = p.skip_seq != nullptr
                         ? launch_partition_kernel<D, BS, true>(p, tmk, tmv, stream)
                         : launch_partition_kernel<D, BS, false>(p, tmk, tmv, stream);
@@ -735,6 +990,15 @@ cudaError_t launch_typed(const DecodeParams& p, cudaStream_t stream) {
 }  // namespace
 
 float log2e_scale(float scale) { return scale * kLog2e; }
+
+int decode_ctas_per_head(int num_kv_heads) {
+    if (num_kv_heads <= 0) return 1;
+    return (kTargetCtasPerSM * device_sm_count() + num_kv_heads - 1) / num_kv_heads;
+}
+
+int decode_range_workers(int num_kv_heads) {
+    return kWarps * decode_ctas_per_head(num_kv_heads);
+}
 
 cudaError_t launch_paged_decode(const DecodeParams& p, int head_size,
                                 int block_size, cudaStream_t stream) {

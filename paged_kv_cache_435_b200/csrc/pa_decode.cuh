@@ -16,6 +16,16 @@ struct DecodeParams {
     float* tmp_o;                // fp32 [B][Hq][max_partitions][D]
     float* tmp_m;                // fp32 [B][Hq][max_partitions] (log2 domain)
     float* tmp_l;                // fp32 [B][Hq][max_partitions]
+    // Persistent split grid: every warp streams its own range of chunks
+    // (a "range worker"); the piece a worker starts in the middle of a
+    // partition goes to the worker's straddle row.
+    float* st_o;                 // fp32 [Hq][max_range_workers][D]
+    float* st_m;                 // fp32 [Hq][max_range_workers]
+    float* st_l;                 // fp32 [Hq][max_range_workers]
+    int32_t* chunk_prefix;       // int32 [B+1]: 16-token chunks before each
+                                 // sequence (written by the partition kernel)
+    int32_t* worker_bounds;      // int32 [max_range_workers+1]: first chunk
+                                 // position of each worker's range (likewise)
     int* error_flags;            // nullable
     int num_seqs;
     int max_blocks_per_seq;
@@ -28,6 +38,9 @@ struct DecodeParams {
     int max_partitions;          // ceil(max_context_len / partition_size)
     float scale_log2;            // scale * log2(e)
     int block_size;
+    int max_range_workers;       // rows of the straddle region per query head
+    int range_workers;           // split on the persistent grid: range workers
+                                 // (warps) per kv head; 0 otherwise
     // Shared-prefix call: the group pass answered the sequences with
     // skip_seq[s] != 0; they have no items here (null: none skipped).
     const int32_t* skip_seq;     // int32 [B]
@@ -35,6 +48,12 @@ struct DecodeParams {
 
 // scale * log2(e): logits are kept in the log2 domain (exp2f).
 float log2e_scale(float scale);
+
+// CTAs per kv head of the persistent grid on the current device (about two
+// per SM over all kv heads), and the range workers (warps) they hold, which
+// size the straddle region.
+int decode_ctas_per_head(int num_kv_heads);
+int decode_range_workers(int num_kv_heads);
 
 // Enqueue the partition kernel (and the merge kernel when
 // max_partitions > 1).  head_size in {64,128}, block_size in {16,32};

@@ -126,7 +126,6 @@ constexpr uint32_t kTmemCols = 256;       // S0 | S1 | O0 (hi, lo) | O1 (hi, lo)
 constexpr uint32_t kTmemO = 64;           // first O column
 constexpr float kRescaleThreshold = 24.f;  // log2 units
 constexpr float kNoMax = -FLT_MAX;        // reference of a row with no token yet
-constexpr int kNumSMs = 148;
 
 static_assert(kStageBytes % 1024 == 0 && kQBytes % 1024 == 0 && kPBytes % 1024 == 0,
               "swizzled tiles need 1024-byte alignment");
@@ -1326,19 +1325,7 @@ bool mr_encode_map(CUtensorMap* map, const void* pool, int num_blocks, int block
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int num_sms() {
-    static int sms[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return kNumSMs;
-    if (sms[dev] == 0) {
-        int v = 0;
-        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            v <= 0)
-            v = kNumSMs;
-        sms[dev] = v;
-    }
-    return sms[dev];
-}
+int num_sms() { return device_sm_count(); }
 
 template <int BS>
 cudaError_t mr_launch_typed(const MultiRowParams& p, cudaStream_t stream) {

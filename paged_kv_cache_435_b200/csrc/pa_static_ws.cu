@@ -11,9 +11,10 @@
 // The array is a file-scope __device__ variable, so every GPU on which the
 // library is used holds PA_STATIC_WORKSPACE_BYTES of it until the process
 // exits.  Host code cannot pass the variable's name to a kernel (on the host
-// it is only a stand-in for the symbol); its device address is looked up
-// once per device with cudaGetSymbolAddress, with that device current, on the
-// first call made on that device, and cached.
+// it is only a stand-in for the symbol); its device address is looked up on
+// every call with cudaGetSymbolAddress on the current device.  The lookup
+// allocates nothing and is cheap, and it stays right when a context is torn
+// down and created again (the module then reloads, possibly elsewhere).
 //
 // All calls share the array and it keeps whatever the last call left in it.
 // The decode kernels write every scratch value before they read it within a
@@ -23,7 +24,6 @@
 #include <cuda_runtime.h>
 
 #include <cstddef>
-#include <mutex>
 
 #include "pa.h"
 
@@ -31,24 +31,12 @@ namespace {
 
 __device__ __align__(256) unsigned char g_decode_scratch[PA_STATIC_WORKSPACE_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of g_decode_scratch on the current device (looked up once).
+// Device address of g_decode_scratch on the current device.
 cudaError_t scratch_address(void** addr) {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (g_scratch_addr[dev] == nullptr) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_decode_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_addr[dev] = p;
-    }
-    *addr = g_scratch_addr[dev];
+    *addr = p;
     return cudaSuccess;
 }
 

@@ -84,18 +84,3 @@ def oracle_attention(case, k_bits, v_bits, seqs=None):
     return oracle.paged_decode_attention(q, k_bits, v_bits, tables, lens,
                                          case.scale,
                                          case.workload.num_kv_heads)
-
-
-def sample_seqs(lens: np.ndarray, n: int, seed: int = 0) -> np.ndarray:
-    """Sequence indices: the longest, the shortest and n-2 random others."""
-    B = len(lens)
-    if B <= n:
-        return np.arange(B)
-    rng = np.random.default_rng(seed)
-    pick = {int(np.argmax(lens)), int(np.argmin(lens))}
-    rest = rng.permutation(B)
-    for s in rest:
-        if len(pick) >= n:
-            break
-        pick.add(int(s))
-    return np.array(sorted(pick))

@@ -62,19 +62,26 @@ def test_multi_query_flops_count_causal_pairs():
 
 
 def test_traffic_is_used_only_for_its_kernel_source_and_workload(tmp_path, monkeypatch):
+    dk, mk = "paged_decode_kernel", "paged_multi_row_kernel"
     good = tmp_path / "traffic.txt"
-    good.write_text(f"# note\nworkload = w1\nkernel_sha = {bench.kernel_sha()}\n"
-                    "dram_bytes_per_launch = 1234.5\n")
+    good.write_text(f"# note\nworkload = w1\nkernel = {dk}\nkernel_sha = {bench.kernel_sha(dk)}\n"
+                    "dram_bytes_per_launch = 1234.5\n\n"
+                    f"workload = w2\nkernel = {mk}\nkernel_sha = {bench.kernel_sha(mk)}\n"
+                    "dram_bytes_per_launch = 99\n")
     monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(good))
-    assert bench.read_traffic("w1") == 1234.5
-    assert bench.read_traffic("w2") is None
+    assert bench.read_traffic("w1", dk) == 1234.5
+    assert bench.read_traffic("w2", mk) == 99.0
+    assert bench.read_traffic("w2", dk) is None   # another kernel's record
+    assert bench.read_traffic("w3", dk) is None
     stale = tmp_path / "stale.txt"
-    stale.write_text("workload = w1\nkernel_sha = 0000000000000000\n"
+    stale.write_text(f"workload = w1\nkernel = {dk}\nkernel_sha = 0000000000000000\n"
                      "dram_bytes_per_launch = 1234.5\n")
     monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(stale))
-    assert bench.read_traffic("w1") is None
-    assert len(bench.kernel_sha()) == 16 and np.all([c in "0123456789abcdef"
-                                                     for c in bench.kernel_sha()])
+    assert bench.read_traffic("w1", dk) is None
+    for k in bench.KERNEL_SOURCES:
+        sha = bench.kernel_sha(k)
+        assert len(sha) == 16 and all(c in "0123456789abcdef" for c in sha)
+    assert bench.kernel_sha(dk) != bench.kernel_sha(mk)
 
 
 def test_shared_prefix_workload_unique_tokens():

@@ -103,6 +103,48 @@ def test_prefix_hash_chains_on_the_parent():
     assert prefix_block_hash(h1, toks(16)) != prefix_block_hash(s ^ 1, toks(16))
 
 
+_FNV64_PRIME = 0x100000001b3
+_FNV64_BASIS = 0xcbf29ce484222325
+
+
+def _fnv1a64(h, data: bytes) -> int:
+    """FNV-1a, 64 bit: for each byte, xor it in, then multiply by the prime."""
+    for c in data:
+        h = ((h ^ c) * _FNV64_PRIME) & ((1 << 64) - 1)
+    return h
+
+
+def test_fnv1a_reference_matches_published_vectors():
+    # Test vectors of the FNV-1a 64-bit hash as published with the algorithm.
+    assert _fnv1a64(_FNV64_BASIS, b"") == 0xcbf29ce484222325
+    assert _fnv1a64(_FNV64_BASIS, b"a") == 0xaf63dc4c8601ec8c
+    assert _fnv1a64(_FNV64_BASIS, b"foobar") == 0x85944171f73967e8
+
+
+@pytest.mark.parametrize("tokens", [
+    [], [0x61], [0x626f6f66, 0x7261], [1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12,
+                                       13, 14, 15, 16], [-1, 2**31 - 1, 0]])
+def test_prefix_hash_known_answers(tokens):
+    # The block hash is FNV-1a over the block's token ids (little-endian
+    # int32 bytes) started from the parent hash, xor the parent times the
+    # prime; the seed of a first block is the FNV offset basis.
+    assert prefix_hash_seed() == _FNV64_BASIS
+    t = np.asarray(tokens, dtype=np.int32)
+    for parent in (_FNV64_BASIS, 0, 0x0123456789abcdef):
+        want = _fnv1a64(parent, t.astype("<i4").tobytes()) ^ \
+            ((parent * _FNV64_PRIME) & ((1 << 64) - 1))
+        assert prefix_block_hash(parent, t) == want
+
+
+def test_prefix_hash_of_ascii_tokens_is_published_fnv1a():
+    # "a" as one token id 0x61 hashes the bytes 61 00 00 00: the published
+    # value of "a" continued over three zero bytes.
+    h_a = _fnv1a64(_FNV64_BASIS, b"a")
+    assert h_a == 0xaf63dc4c8601ec8c
+    want = _fnv1a64(h_a, b"\0\0\0") ^ ((_FNV64_BASIS * _FNV64_PRIME) & ((1 << 64) - 1))
+    assert prefix_block_hash(_FNV64_BASIS, np.array([0x61], np.int32)) == want
+
+
 def test_out_of_blocks_changes_nothing():
     m = BlockManager(4, 16)
     a, _, _ = m.add_sequence(toks(48))

@@ -223,3 +223,21 @@ def test_long_prefix_and_tails():
     case = inputs.grouped_case(32, 8, 128, 16, lens, [0, 6, 9], [P0, P1], seed=16,
                                device="cuda")
     check(case)
+
+
+@pytest.mark.parametrize("partition_size", [0, 256])
+def test_more_than_768_sequences(partition_size):
+    """800 sequences: 96 groups of 8 samples sharing a 512-token prefix, then
+    32 sequences outside every group.  Past 768 sequences the per-sequence
+    pass skips the groups' members on the plain grid (one CTA per kv head,
+    partition and sequence) instead of the persistent compact-item grid; with
+    256-token partitions the ungrouped sequences are split and merged."""
+    rng = np.random.default_rng(768)
+    grouped = 512 + rng.integers(0, 201, size=768)
+    lone = rng.integers(1, 1500, size=32)
+    lens = np.concatenate([grouped, lone])
+    gs = np.arange(0, 769, 8)
+    pl = np.full(96, 512)
+    case = inputs.grouped_case(32, 8, 128, 16, lens, gs, pl, seed=800,
+                               device="cuda")
+    check(case, partition_size=partition_size)
