@@ -268,8 +268,14 @@ int pa_multi_query_attention(float* out, const void* q, const void* k_cache,
  *                   without the group pass.
  *   workspace       device buffer of at least
  *                   pa_shared_prefix_workspace_size(...) bytes, 256-byte
- *                   aligned; scratch, needs no initialisation.
+ *                   aligned (NULL allowed when that size is 0); scratch,
+ *                   needs no initialisation.  It holds the per-sequence
+ *                   pass's split-KV scratch only.
  *   other arguments as for pa_decode_attention.
+ * The group pass and the per-sequence pass write disjoint outputs and
+ * classify every sequence with the same rule from group_start / prefix_lens,
+ * so the per-sequence pass may run while the group pass is still running
+ * (on the SMs that pass leaves free).
  * Supports head_size 128, block_size in {16, 32}, num_heads / num_kv_heads
  * in 1..8 (head_size 64 returns PA_ERR_UNSUPPORTED).  Returns PA_OK or a
  * negative pa_status; run-to-run results are bitwise deterministic.

@@ -274,7 +274,8 @@ def pa_decode_attention_shared_prefix(out, q, k_cache, v_cache, block_tables,
     _cuda(context_lens, "context_lens", torch.int32, 1)
     _cuda(group_start, "group_start", torch.int32, 1)
     _cuda(prefix_lens, "prefix_lens", torch.int32, 1)
-    _cuda(workspace, "workspace")
+    if workspace is not None:
+        _cuda(workspace, "workspace")
     for name, t in (("out", out), ("q", q), ("k_cache", k_cache),
                     ("v_cache", v_cache), ("block_tables", block_tables),
                     ("context_lens", context_lens),
@@ -290,7 +291,7 @@ def pa_decode_attention_shared_prefix(out, q, k_cache, v_cache, block_tables,
         raise ValueError("block_tables / context_lens must have B rows")
     if group_start.shape[0] != G + 1:
         raise ValueError("group_start must have one more entry than prefix_lens")
-    ws_bytes = workspace.numel() * workspace.element_size()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     rc = raw().pa_decode_attention_shared_prefix(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
         block_tables.shape[1], _ptr(context_lens), int(max_context_len),

@@ -133,21 +133,6 @@ void assign_split(DecodeParams& p, unsigned char* ws, const SplitLayout& L) {
     p.worker_bounds = reinterpret_cast<int32_t*>(ws + L.bounds);
 }
 
-// Shared-prefix call: the decode split's scratch, then one flag per
-// sequence (the group pass answered it).
-struct PrefixLayout {
-    size_t done_off, total;
-};
-
-PrefixLayout prefix_layout(int num_seqs, int num_heads, int num_kv_heads,
-                           int head_size, int max_partitions) {
-    PrefixLayout L;
-    L.done_off = align256(workspace_bytes_for(num_seqs, num_heads, num_kv_heads,
-                                              head_size, max_partitions));
-    L.total = L.done_off + (((size_t)num_seqs * 4 + 255) & ~(size_t)255);
-    return L;
-}
-
 }  // namespace
 }  // namespace pa
 
@@ -407,8 +392,8 @@ size_t pa_shared_prefix_workspace_size(int num_seqs, int num_heads,
                                               head_size, block_size,
                                               max_context_len, partition_size);
     if (part <= 0 || num_heads <= 0 || head_size <= 0) return 0;
-    return pa::prefix_layout(num_seqs, num_heads, num_kv_heads, head_size,
-                             pa::num_partitions(max_context_len, part)).total;
+    return pa::workspace_bytes_for(num_seqs, num_heads, num_kv_heads, head_size,
+                                   pa::num_partitions(max_context_len, part));
 }
 
 int pa_decode_attention_shared_prefix(
@@ -453,10 +438,12 @@ int pa_decode_attention_shared_prefix(
                                         max_context_len, partition_size);
     const int np = pa::num_partitions(max_context_len, part);
     if (np > pa::kMaxGridYZ) return PA_ERR_INVALID_ARG;
-    const pa::PrefixLayout lay =
-        pa::prefix_layout(num_seqs, num_heads, num_kv_heads, head_size, np);
-    if (!workspace || workspace_bytes < lay.total) return PA_ERR_WORKSPACE;
-    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PA_ERR_INVALID_ARG;
+    const pa::SplitLayout lay =
+        pa::split_layout(num_seqs, num_heads, num_kv_heads, head_size, np);
+    if (lay.total > 0) {
+        if (!workspace || workspace_bytes < lay.total) return PA_ERR_WORKSPACE;
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PA_ERR_INVALID_ARG;
+    }
     unsigned char* ws = static_cast<unsigned char*>(workspace);
     const int G = num_heads / num_kv_heads;
     // A group cannot hold more than num_seqs sequences: the bound changes
@@ -475,7 +462,6 @@ int pa_decode_attention_shared_prefix(
         r.block_tables = block_tables;
         r.context_lens = context_lens;
         r.groups = groups;
-        r.seq_done = reinterpret_cast<int32_t*>(ws + lay.done_off);
         r.error_flags = error_flags;
         r.shared_prefix_mode = 1;
         r.num_seqs = num_seqs;
@@ -501,8 +487,7 @@ int pa_decode_attention_shared_prefix(
     p.v_cache = static_cast<const uint16_t*>(v_cache);
     p.block_tables = block_tables;
     p.context_lens = context_lens;
-    pa::assign_split(p, ws, pa::split_layout(num_seqs, num_heads, num_kv_heads,
-                                              head_size, np));
+    pa::assign_split(p, ws, lay);
     p.error_flags = error_flags;
     p.num_seqs = num_seqs;
     p.max_blocks_per_seq = max_blocks_per_seq;
@@ -515,8 +500,8 @@ int pa_decode_attention_shared_prefix(
     p.max_partitions = np;
     p.scale_log2 = pa::log2e_scale(scale);
     p.block_size = block_size;
-    p.skip_seq = num_groups > 0 ? reinterpret_cast<const int32_t*>(ws + lay.done_off)
-                                : nullptr;
+    p.has_groups = num_groups > 0;
+    p.groups = groups;
     cudaError_t e = pa::launch_paged_decode(p, head_size, block_size, st);
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

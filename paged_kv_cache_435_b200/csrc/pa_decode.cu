@@ -83,7 +83,10 @@ struct Cfg {
     static constexpr int kBarBytes = (kWarps * (kStages + 1) * 8 + 127) / 128 * 128;
     static constexpr int kPrefixOff = kBarOff + kBarBytes;
     static constexpr int kSmemGrid = kPrefixOff;
-    static constexpr int kSmemPersist = kPrefixOff + (kMaxPersistSeqs + 1) * 4;
+    // Persistent grid: the chunk prefix, then (shared-prefix call) one bit
+    // per sequence marking the grouped ones.
+    static constexpr int kGroupedOff = kPrefixOff + (kMaxPersistSeqs + 1) * 4;
+    static constexpr int kSmemPersist = kGroupedOff + (kMaxPersistSeqs + 31) / 32 * 4;
     static_assert(kRingBytes % 1024 == 0, "ring tiles must stay 1024-aligned");
     static_assert(kSmemPersist + 1024 <= 232448 / kTargetCtasPerSM,
                   "two CTAs per SM must fit");
@@ -117,10 +120,21 @@ __device__ __forceinline__ int parts_of(int L, int P) {
     return L <= 0 ? 1 : (L + P - 1) / P;  // an empty context still owns one item
 }
 
-// Sequence s has no items here: a shared-prefix group pass answered it.
+// Sequence s has no items here: a shared-prefix group pass answers it (it
+// belongs to a valid group with a prefix).
+__device__ __forceinline__ bool grouped(const DecodeParams& p, int s) {
+    const int i = cascade_group_of(p.groups, s);
+    return i >= 0 && cascade_group_prefix(p.groups, i, p.num_seqs, p.block_size,
+                                          nullptr, false) > 0;
+}
 template <bool kSkip>
 __device__ __forceinline__ bool skipped(const DecodeParams& p, int s) {
-    return kSkip && p.skip_seq[s] != 0;
+    return kSkip && grouped(p, s);
+}
+// The same from the CTA's bitmap of grouped sequences (persistent grid).
+template <bool kSkip>
+__device__ __forceinline__ bool skipped_bit(const uint32_t* bits, int s) {
+    return kSkip && ((bits[s >> 5] >> (s & 31)) & 1u);
 }
 
 // ---------------------------------------------------------------- plain grid
@@ -279,11 +293,31 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         return;
     }
     // Launched behind the cache write: nothing global is read before the
-    // preceding grid has completed.
-    pdl_wait();
+    // preceding grid has completed.  In the shared-prefix call the
+    // preceding grid is the group pass, which this pass needs nothing from
+    // (the outputs are disjoint, the grouping is recomputed here); it may
+    // run beside it, since the group pass lets it launch only after its own
+    // wait for the cache write.
+    if (!kSkip) pdl_wait();
     pdl_launch_dependents();
 
     Range rg{0, 0, 1, 0};
+    uint32_t* grouped_bits = reinterpret_cast<uint32_t*>(smem + C::kGroupedOff);
+    if (kPersist && kSkip) {
+        // Mark the members of every valid group with a prefix: a thread per
+        // group, one round of loads (the same rule as cascade_group_prefix).
+        for (int w = threadIdx.x; w < (p.num_seqs + 31) / 32; w += kThreads)
+            grouped_bits[w] = 0u;
+        __syncthreads();
+        for (int i = threadIdx.x; i < p.groups.num_groups; i += kThreads) {
+            if (cascade_group_prefix(p.groups, i, p.num_seqs, p.block_size, nullptr,
+                                     false) <= 0)
+                continue;
+            const int a = p.groups.group_start[i], b = p.groups.group_start[i + 1];
+            for (int s = a; s < b; ++s) atomicOr(&grouped_bits[s >> 5], 1u << (s & 31));
+        }
+        __syncthreads();
+    }
     if (kPersist) {
         // X[s] = 16-token chunks of sequences 0..s-1 (block-wide scan).  The
         // merge area is free until the first item ends; it holds the warp sums.
@@ -293,7 +327,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         for (int base = 0; base < p.num_seqs; base += kThreads) {
             const int s = base + threadIdx.x;
             int v = 0;
-            if (s < p.num_seqs && !skipped<kSkip>(p, s))
+            if (s < p.num_seqs && !skipped_bit<kSkip>(grouped_bits, s))
                 v = (clamped_len(p, s) + kChunk - 1) / kChunk;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -698,7 +732,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         // Sequences with an empty context (not skipped) own no chunk: their
         // output is zero, written by the CTAs of the head in turn.
         for (int s = blockIdx.y; s < p.num_seqs; s += gridDim.y) {
-            if (skipped<kSkip>(p, s) || X[s + 1] != X[s]) continue;
+            if (skipped_bit<kSkip>(grouped_bits, s) || X[s + 1] != X[s]) continue;
             for (int e = threadIdx.x; e < G * D; e += kThreads)
                 p.out[((int64_t)s * Hq + g * G) * D + e] = 0.f;
         }
@@ -722,10 +756,13 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
 // memory.  Sequences held whole by one piece were written by the partition
 // kernel.
 constexpr int kReduceWarps = 8;
-constexpr int kReduceUnroll = 16;
+constexpr int kReduceUnroll = 8;
+// Most of the grid's CTAs find a sequence held whole and leave at once; with
+// three CTAs resident per SM the whole grid is in flight in a few waves.
+constexpr int kReduceCtasPerSM = 3;
 
 template <int D>
-__global__ void __launch_bounds__(kReduceWarps * 32)
+__global__ void __launch_bounds__(kReduceWarps * 32, kReduceCtasPerSM)
 paged_decode_reduce_kernel(const DecodeParams p) {
     constexpr int V = D / 32;  // columns per lane
     const int h = blockIdx.x;
@@ -733,8 +770,16 @@ paged_decode_reduce_kernel(const DecodeParams p) {
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     pdl_wait();  // the partials come from the grid launched just before
-    if (p.skip_seq != nullptr && p.skip_seq[s] != 0) return;  // answered elsewhere
+    // Every scalar this CTA needs, loaded together (one round trip).  On the
+    // range grid the partition kernel's published chunk prefix says which
+    // sequences it streamed: a grouped (skipped) or empty sequence has no
+    // chunks, so both kernels classify it the same way by construction.
+    const bool ranges = p.range_workers > 0;
     int L = p.context_lens[s];
+    const int xs_raw = ranges ? p.chunk_prefix[s] : 0;
+    const int xe_raw = ranges ? p.chunk_prefix[s + 1] : 0;
+    const int T_raw = ranges ? p.chunk_prefix[p.num_seqs] : 1;
+    if (!ranges && p.has_groups && grouped(p, s)) return;  // answered elsewhere
     L = L < 0 ? 0 : (L > p.max_context_len ? p.max_context_len : L);
 
     // Pieces: partition slots 0..nslot-1, then candidate straddle rows
@@ -744,13 +789,13 @@ paged_decode_reduce_kernel(const DecodeParams p) {
     // starting at that position (earlier ones have empty ranges).
     int nslot, b_lo = 0, ncand = 0, xs = 0, q = 1;
     const int32_t* E = p.worker_bounds;
-    if (p.range_workers > 0) {
-        const int cs = (L + kChunk - 1) / kChunk;
-        if (cs == 0) return;  // empty: zeros written by the partition kernel
+    if (ranges) {
+        const int cs = xe_raw - xs_raw;
+        if (cs <= 0) return;  // grouped, or empty (zeros written by the partition kernel)
         q = p.partition_size / kChunk;
         nslot = (cs + q - 1) / q;
-        xs = p.chunk_prefix[s];
-        const long long T = p.chunk_prefix[p.num_seqs];
+        xs = xs_raw;
+        const long long T = T_raw;
         const long long n = p.range_workers;
         // floor(b T / n) > xs  <=>  b >= ceil((xs + 1) n / T);
         // floor(b T / n) < xs + cs  <=>  b <= ceil((xs + cs) n / T) - 1.
@@ -765,12 +810,15 @@ paged_decode_reduce_kernel(const DecodeParams p) {
         const int e = E[b];
         return (e - xs) % q != 0 && E[b + 1] > e;
     };
-    int nstr = 0;
-    for (int c = lane; c < ncand; c += 32)
-        nstr += straddle(b_lo + c) ? 1 : 0;
+    if (nslot <= 1) {
+        // One partition: split only if a range starts inside it.
+        int nstr = 0;
+        for (int c = lane; c < ncand; c += 32)
+            nstr += straddle(b_lo + c) ? 1 : 0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) nstr += __shfl_xor_sync(0xffffffffu, nstr, o);
-    if (nslot + nstr <= 1) return;  // written directly by the partition kernel
+        for (int o = 16; o > 0; o >>= 1) nstr += __shfl_xor_sync(0xffffffffu, nstr, o);
+        if (nslot + nstr <= 1) return;  // written directly by the partition kernel
+    }
     const int total = nslot + ncand;
 
     __shared__ float part_m[kReduceWarps];
@@ -974,7 +1022,7 @@ cudaError_t launch_typed(const DecodeParams& params, cudaStream_t stream) {
         !encode_pool_map(&tmv, params.v_cache, params.num_blocks, BS, params.num_kv_heads, D))
         return cudaErrorInvalidValue;
     DecodeParams p = params;
-    cudaError_t e = p.skip_seq != nullptr
+    cudaError_t e = p.has_groups
                         ? launch_partition_kernel<D, BS, true>(p, tmk, tmv, stream)
                         : launch_partition_kernel<D, BS, false>(p, tmk, tmv, stream);
     if (e != cudaSuccess) return e;

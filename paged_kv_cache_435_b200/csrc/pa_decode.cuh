@@ -4,6 +4,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "pa_cascade.cuh"
+
 namespace pa {
 
 struct DecodeParams {
@@ -41,9 +43,11 @@ struct DecodeParams {
     int max_range_workers;       // rows of the straddle region per query head
     int range_workers;           // split on the persistent grid: range workers
                                  // (warps) per kv head; 0 otherwise
-    // Shared-prefix call: the group pass answered the sequences with
-    // skip_seq[s] != 0; they have no items here (null: none skipped).
-    const int32_t* skip_seq;     // int32 [B]
+    // Shared-prefix call: the members of valid groups with a prefix are
+    // answered by the group pass and have no items here; both passes
+    // classify a sequence with the same functions (pa_cascade.cuh).
+    bool has_groups;
+    CascadeGroups groups;
 };
 
 // scale * log2(e): logits are kept in the log2 domain (exp2f).

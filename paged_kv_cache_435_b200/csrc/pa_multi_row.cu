@@ -803,18 +803,6 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             pos += total;
         }
         if (!stopped) (void)publish(-1);
-        if (p.shared_prefix_mode) {
-            // Which sequences this pass answers (members of valid groups with
-            // a prefix), for the per-sequence pass to skip: the CTAs split
-            // the batch.  Only the next launch reads them, after this grid
-            // has completed, so they are written once the items are out.
-            for (int s = blockIdx.x * 32 + lane; s < p.num_seqs; s += gridDim.x * 32) {
-                const int i = cascade_group_of(p.groups, s);
-                p.seq_done[s] = (i >= 0 && cascade_group_prefix(p.groups, i, p.num_seqs,
-                                                                p.block_size, nullptr,
-                                                                false) > 0) ? 1 : 0;
-            }
-        }
     } else if (warp == 4 || warp == 5) {
         // ------------------------------------------------ K / V producers
         const bool is_v = warp == 5;

@@ -21,8 +21,6 @@ struct MultiRowParams {
     const int32_t* context_lens;     // int32 [B]
     const int32_t* query_start_loc;  // int32 [B+1] (multi-query mode)
     CascadeGroups groups;            // shared-prefix mode
-    int32_t* seq_done;               // shared-prefix mode: int32 [B], written:
-                                     // 1 if this pass answers the sequence
     int* error_flags;                // nullable
     int shared_prefix_mode;
     int num_seqs;

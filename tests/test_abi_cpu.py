@@ -209,20 +209,22 @@ def test_shared_prefix_host_validation(lib):
     assert call(a9=FAKE + 2) == nat.PA_ERR_INVALID_ARG     # prefix_lens misaligned
     assert call(a15=64) == nat.PA_ERR_UNSUPPORTED          # head size 64
     assert call(a13=128) == nat.PA_ERR_UNSUPPORTED         # 128 q / 8 kv: group 16
-    assert call(a20=None) == nat.PA_ERR_WORKSPACE          # no workspace
-    assert call(a21=16) == nat.PA_ERR_WORKSPACE            # too small
-    assert call(a20=FAKE + 16) == nat.PA_ERR_INVALID_ARG   # workspace not 256-aligned
+    # 64-token partitions split the 100-token contexts: scratch is needed
+    assert call(a19=64, a20=None) == nat.PA_ERR_WORKSPACE          # no workspace
+    assert call(a19=64, a21=16) == nat.PA_ERR_WORKSPACE            # too small
+    assert call(a19=64, a20=FAKE + 16) == nat.PA_ERR_INVALID_ARG   # not 256-aligned
     assert call(a12=0, a0=None, a1=None) == nat.PA_OK      # empty batch
 
 
 def test_shared_prefix_workspace_grows_with_rows(lib):
+    # The shared-prefix call needs only the per-sequence pass's split scratch.
+    for B in (8, 16):
+        for part in (0, 64):
+            assert (nat.pa_shared_prefix_workspace_size(B, 32, 8, 128, 16, 1000, part) ==
+                    nat.pa_decode_workspace_size(B, 32, 8, 128, 16, 1000, part))
     a = nat.pa_shared_prefix_workspace_size(8, 32, 8, 128, 16, 1000)
     b = nat.pa_shared_prefix_workspace_size(16, 32, 8, 128, 16, 1000)
-    assert b > a >= nat.pa_decode_workspace_size(8, 32, 8, 128, 16, 1000) + 8 * 4
-    # one flag per sequence beside the decode split's scratch
-    assert a == nat.pa_decode_workspace_size(8, 32, 8, 128, 16, 1000) + 256
-    # no split (short contexts): the flags alone
-    assert nat.pa_shared_prefix_workspace_size(8, 32, 8, 128, 16, 300) == 256
+    assert b > a > 0
 
 
 def test_missing_library_raises_instead_of_falling_back():
