@@ -87,10 +87,13 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 // Split-KV scratch, each region 256-byte aligned: the partition slots
 // tmp_o [B][Hq][P][D], tmp_m, tmp_l [B][Hq][P]; the persistent grid's
 // straddle rows st_o [Hq][n][D], st_m, st_l [Hq][n] (n = range workers per
-// kv head); the chunk prefix [B+1] and the workers' range starts [n+1].
+// kv head); the chunk prefix [B+1] and the workers' range starts [n+1];
+// the range merge's arrival counters [B][Hq] and slice partials
+// sub_o [B][Hq][S][D], sub_m, sub_l [B][Hq][S].
 struct SplitLayout {
-    size_t o, m, l, st_o, st_m, st_l, prefix, bounds, total;
-    int range_workers;
+    size_t o, m, l, st_o, st_m, st_l, prefix, bounds, count, sub_o, sub_m, sub_l,
+        total;
+    int range_workers, max_slices;
 };
 
 SplitLayout split_layout(int num_seqs, int num_heads, int num_kv_heads,
@@ -109,6 +112,14 @@ SplitLayout split_layout(int num_seqs, int num_heads, int num_kv_heads,
     L.st_l = off;   off = align256(off + st_rows * 4);
     L.prefix = off; off = align256(off + ((size_t)num_seqs + 1) * 4);
     L.bounds = off; off = align256(off + ((size_t)L.range_workers + 1) * 4);
+    // A sequence's candidate rows: its partition slots plus the range
+    // boundaries inside it.
+    L.max_slices = (max_partitions + L.range_workers + kMergeRows - 1) / kMergeRows;
+    const size_t sub_rows = (size_t)num_seqs * num_heads * L.max_slices;
+    L.count = off;  off = align256(off + (size_t)num_seqs * num_heads * 4);
+    L.sub_o = off;  off = align256(off + sub_rows * head_size * 4);
+    L.sub_m = off;  off = align256(off + sub_rows * 4);
+    L.sub_l = off;  off = align256(off + sub_rows * 4);
     L.total = off;
     return L;
 }
@@ -131,6 +142,11 @@ void assign_split(DecodeParams& p, unsigned char* ws, const SplitLayout& L) {
     p.st_l = reinterpret_cast<float*>(ws + L.st_l);
     p.chunk_prefix = reinterpret_cast<int32_t*>(ws + L.prefix);
     p.worker_bounds = reinterpret_cast<int32_t*>(ws + L.bounds);
+    p.merge_count = reinterpret_cast<int32_t*>(ws + L.count);
+    p.sub_o = reinterpret_cast<float*>(ws + L.sub_o);
+    p.sub_m = reinterpret_cast<float*>(ws + L.sub_m);
+    p.sub_l = reinterpret_cast<float*>(ws + L.sub_l);
+    p.max_slices = L.max_slices;
 }
 
 }  // namespace

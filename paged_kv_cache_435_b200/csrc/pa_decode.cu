@@ -357,6 +357,16 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                 for (int i = threadIdx.x; i <= n; i += kThreads)
                     p.worker_bounds[i] = (int)(i * T / n);
             }
+            // Arrival counters of the merge, zeroed here: the merge kernel
+            // starts only after this grid has completed.  Each CTA clears a
+            // contiguous share.
+            {
+                const long long total = (long long)p.num_seqs * p.num_heads;
+                const long long ctas = (long long)gridDim.x * gridDim.y;
+                const long long me = (long long)blockIdx.y * gridDim.x + blockIdx.x;
+                const long long c0 = total * me / ctas, c1 = total * (me + 1) / ctas;
+                for (long long c = c0 + threadIdx.x; c < c1; c += kThreads) p.merge_count[c] = 0;
+            }
         } else {
             const long long n = gridDim.y;
             const int b = blockIdx.y;
@@ -746,126 +756,31 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
     }
 }
 
-// Merge of the pieces of a split sequence: out = sum_i w_i o_i / sum_i w_i
-// with w_i = l_i * 2^(m_i - max_j m_j), over the sequence's partition slots
-// and, on the persistent grid, the straddle rows of the range workers whose
-// ranges begin inside one of its partitions.  One CTA of 8 warps per (query head,
-// sequence); warp w takes pieces w, w+8, ..., 16 pieces' rows in flight per
-// round, each lane holding D/32 consecutive columns, with a running max so
-// every round is one memory round trip; the warps combine through shared
-// memory.  Sequences held whole by one piece were written by the partition
-// kernel.
+// ---------------------------------------------------------------- merges
+// Merge of a split sequence's pieces: out = sum_i w_i o_i / sum_i w_i with
+// w_i = l_i * 2^(m_i - max_j m_j).  A row of (m, l, o) of D floats per piece;
+// rows are read 8 per warp per round, all loads of a round issued before any
+// value is used, with a running max so a round is one memory round trip.
 constexpr int kReduceWarps = 8;
 constexpr int kReduceUnroll = 8;
-// Most of the grid's CTAs find a sequence held whole and leave at once; with
-// three CTAs resident per SM the whole grid is in flight in a few waves.
-constexpr int kReduceCtasPerSM = 3;
+static_assert(kReduceWarps * kReduceUnroll == kMergeRows, "one round per merge slice");
 
 template <int D>
-__global__ void __launch_bounds__(kReduceWarps * 32, kReduceCtasPerSM)
-paged_decode_reduce_kernel(const DecodeParams p) {
-    constexpr int V = D / 32;  // columns per lane
-    const int h = blockIdx.x;
-    const int s = blockIdx.y;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    pdl_wait();  // the partials come from the grid launched just before
-    // Every scalar this CTA needs, loaded together (one round trip).  On the
-    // range grid the partition kernel's published chunk prefix says which
-    // sequences it streamed: a grouped (skipped) or empty sequence has no
-    // chunks, so both kernels classify it the same way by construction.
-    const bool ranges = p.range_workers > 0;
-    int L = p.context_lens[s];
-    const int xs_raw = ranges ? p.chunk_prefix[s] : 0;
-    const int xe_raw = ranges ? p.chunk_prefix[s + 1] : 0;
-    const int T_raw = ranges ? p.chunk_prefix[p.num_seqs] : 1;
-    if (!ranges && p.has_groups && grouped(p, s)) return;  // answered elsewhere
-    L = L < 0 ? 0 : (L > p.max_context_len ? p.max_context_len : L);
-
-    // Pieces: partition slots 0..nslot-1, then candidate straddle rows
-    // b_lo..b_lo+ncand-1 (persistent grid only): the range boundaries
-    // strictly inside the sequence's chunks.  A candidate holds a piece when
-    // its boundary is not a partition start and it is the last worker
-    // starting at that position (earlier ones have empty ranges).
-    int nslot, b_lo = 0, ncand = 0, xs = 0, q = 1;
-    const int32_t* E = p.worker_bounds;
-    if (ranges) {
-        const int cs = xe_raw - xs_raw;
-        if (cs <= 0) return;  // grouped, or empty (zeros written by the partition kernel)
-        q = p.partition_size / kChunk;
-        nslot = (cs + q - 1) / q;
-        xs = xs_raw;
-        const long long T = T_raw;
-        const long long n = p.range_workers;
-        // floor(b T / n) > xs  <=>  b >= ceil((xs + 1) n / T);
-        // floor(b T / n) < xs + cs  <=>  b <= ceil((xs + cs) n / T) - 1.
-        const long long lo = ((xs + 1) * n + T - 1) / T;
-        const long long hi = ((xs + cs) * n + T - 1) / T - 1;
-        b_lo = (int)max(1LL, lo);
-        ncand = max(0, (int)min(n - 1, hi) - b_lo + 1);
-    } else {
-        nslot = (L + p.partition_size - 1) / p.partition_size;
-    }
-    auto straddle = [&](int b) -> bool {
-        const int e = E[b];
-        return (e - xs) % q != 0 && E[b + 1] > e;
-    };
-    if (nslot <= 1) {
-        // One partition: split only if a range starts inside it.
-        int nstr = 0;
-        for (int c = lane; c < ncand; c += 32)
-            nstr += straddle(b_lo + c) ? 1 : 0;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) nstr += __shfl_xor_sync(0xffffffffu, nstr, o);
-        if (nslot + nstr <= 1) return;  // written directly by the partition kernel
-    }
-    const int total = nslot + ncand;
-
-    __shared__ float part_m[kReduceWarps];
-    __shared__ float part_den[kReduceWarps];
-    __shared__ float part_acc[kReduceWarps][D];
-
-    const int64_t slot_base = ((int64_t)s * p.num_heads + h) * p.max_partitions;
-    const int64_t st_base = (int64_t)h * p.max_range_workers;
+struct MergeAcc {
+    static constexpr int V = D / 32;  // columns per lane
     float M = -INFINITY, den = 0.f;
-    float acc[V];
-#pragma unroll
-    for (int v = 0; v < V; ++v) acc[v] = 0.f;
-    for (int i0 = warp; i0 < total; i0 += kReduceWarps * kReduceUnroll) {
-        // Every load of the round is issued before any is used; a row that
-        // is not a piece is read from a valid address and then ignored (the
-        // straddle region may hold an earlier call's values).
-        float mv[kReduceUnroll], lv[kReduceUnroll], vals[kReduceUnroll][V];
-        bool live[kReduceUnroll];
-#pragma unroll
-        for (int u = 0; u < kReduceUnroll; ++u) {
-            const int i = i0 + u * kReduceWarps;
-            const bool in_slots = i < nslot;
-            const int b = b_lo + (in_slots ? 0 : min(i - nslot, max(ncand - 1, 0)));
-            live[u] = i < total && (in_slots || straddle(b));
-            const int64_t r = in_slots ? slot_base + i : st_base + b;
-            const float* mrow = in_slots ? p.tmp_m : p.st_m;
-            const float* lrow = in_slots ? p.tmp_l : p.st_l;
-            const float* orow = (in_slots ? p.tmp_o : p.st_o) + r * D + lane * V;
-            const bool ok = i < total;
-            mv[u] = ok ? mrow[r] : -INFINITY;
-            lv[u] = ok ? lrow[r] : 0.f;
-            if (V == 4) {
-                const float4 t = ok ? *reinterpret_cast<const float4*>(orow)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-                vals[u][0] = t.x; vals[u][V > 1 ? 1 : 0] = t.y;
-                vals[u][V > 2 ? 2 : 0] = t.z; vals[u][V > 3 ? 3 : 0] = t.w;
-            } else {
-                const float2 t = ok ? *reinterpret_cast<const float2*>(orow)
-                                    : make_float2(0.f, 0.f);
-                vals[u][0] = t.x; vals[u][V > 1 ? 1 : 0] = t.y;
-            }
-        }
+    float acc[V] = {};
+
+    // Fold a round of up to kReduceUnroll rows (live[u] false: ignored).
+    __device__ __forceinline__ void fold(const float (&mv)[kReduceUnroll],
+                                         const float (&lv)[kReduceUnroll],
+                                         const float (&vals)[kReduceUnroll][V],
+                                         const bool (&live)[kReduceUnroll]) {
         float Mr = M;
 #pragma unroll
         for (int u = 0; u < kReduceUnroll; ++u)
             if (live[u]) Mr = fmaxf(Mr, mv[u]);
-        if (Mr == -INFINITY) continue;
+        if (Mr == -INFINITY) return;
         const float keep = M == -INFINITY ? 0.f : exp2f(M - Mr);
         den *= keep;
 #pragma unroll
@@ -880,25 +795,256 @@ paged_decode_reduce_kernel(const DecodeParams p) {
         }
         M = Mr;
     }
+};
+
+template <int D>
+__device__ __forceinline__ void load_row(const float* row, bool ok, float (&dst)[D / 32]) {
+    constexpr int V = D / 32;
+    if (V == 4) {
+        const float4 t = ok ? *reinterpret_cast<const float4*>(row) : make_float4(0.f, 0.f, 0.f, 0.f);
+        dst[0] = t.x; dst[V > 1 ? 1 : 0] = t.y; dst[V > 2 ? 2 : 0] = t.z; dst[V > 3 ? 3 : 0] = t.w;
+    } else {
+        const float2 t = ok ? *reinterpret_cast<const float2*>(row) : make_float2(0.f, 0.f);
+        dst[0] = t.x; dst[V > 1 ? 1 : 0] = t.y;
+    }
+}
+
+// Combine the 8 warps' accumulators through shared memory; every thread
+// returns the CTA's max and sum, and thread d's column d of the sum of O.
+template <int D>
+struct MergeSmem {
+    float m[kReduceWarps];
+    float den[kReduceWarps];
+    float acc[kReduceWarps][D];
+};
+
+template <int D>
+__device__ __forceinline__ void combine_warps(const MergeAcc<D>& a, MergeSmem<D>& sm,
+                                              float& M, float& den) {
+    constexpr int V = D / 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (lane == 0) {
-        part_m[warp] = M;
-        part_den[warp] = den;
+        sm.m[warp] = a.M;
+        sm.den[warp] = a.den;
     }
 #pragma unroll
-    for (int v = 0; v < V; ++v) part_acc[warp][lane * V + v] = acc[v];
+    for (int v = 0; v < V; ++v) sm.acc[warp][lane * V + v] = a.acc[v];
     __syncthreads();
-    float Mall = -INFINITY;
+    M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kReduceWarps; ++w) Mall = fmaxf(Mall, part_m[w]);
-    for (int d = threadIdx.x; d < D; d += kReduceWarps * 32) {
-        float a = 0.f, dn = 0.f;
+    for (int w = 0; w < kReduceWarps; ++w) M = fmaxf(M, sm.m[w]);
+    den = 0.f;
 #pragma unroll
-        for (int w = 0; w < kReduceWarps; ++w) {
-            const float sc = part_m[w] == -INFINITY ? 0.f : exp2f(part_m[w] - Mall);
-            a += sc * part_acc[w][d];
-            dn += sc * part_den[w];
+    for (int w = 0; w < kReduceWarps; ++w)
+        den += sm.m[w] == -INFINITY ? 0.f : sm.den[w] * exp2f(sm.m[w] - M);
+}
+
+template <int D>
+__device__ __forceinline__ float combined_column(const MergeSmem<D>& sm, float M, int d) {
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < kReduceWarps; ++w)
+        a += sm.m[w] == -INFINITY ? 0.f : sm.acc[w][d] * exp2f(sm.m[w] - M);
+    return a;
+}
+
+// Plain grid (more than kMaxPersistSeqs sequences): one CTA of 8 warps per
+// (query head, sequence) merges the sequence's partition slots.  Sequences
+// held by one partition were written by the partition kernel.
+template <int D>
+__global__ void __launch_bounds__(kReduceWarps * 32, 3)
+paged_decode_reduce_kernel(const DecodeParams p) {
+    constexpr int V = D / 32;
+    const int h = blockIdx.x;
+    const int s = blockIdx.y;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    pdl_wait();  // the partials come from the grid launched just before
+    int L = p.context_lens[s];
+    if (p.has_groups && grouped(p, s)) return;  // answered by the group pass
+    L = L < 0 ? 0 : (L > p.max_context_len ? p.max_context_len : L);
+    const int nslot = (L + p.partition_size - 1) / p.partition_size;
+    if (nslot <= 1) return;
+    __shared__ MergeSmem<D> sm;
+    const int64_t base = ((int64_t)s * p.num_heads + h) * p.max_partitions;
+    MergeAcc<D> a;
+    for (int i0 = warp; i0 < nslot; i0 += kReduceWarps * kReduceUnroll) {
+        float mv[kReduceUnroll], lv[kReduceUnroll], vals[kReduceUnroll][V];
+        bool live[kReduceUnroll];
+#pragma unroll
+        for (int u = 0; u < kReduceUnroll; ++u) {
+            const int i = i0 + u * kReduceWarps;
+            live[u] = i < nslot;
+            const int64_t r = base + (live[u] ? i : 0);
+            mv[u] = live[u] ? p.tmp_m[r] : -INFINITY;
+            lv[u] = live[u] ? p.tmp_l[r] : 0.f;
+            load_row<D>(p.tmp_o + r * D + lane * V, live[u], vals[u]);
         }
-        p.out[((int64_t)s * p.num_heads + h) * D + d] = a / dn;
+        a.fold(mv, lv, vals, live);
+    }
+    float M, den;
+    combine_warps<D>(a, sm, M, den);
+    for (int d = threadIdx.x; d < D; d += kReduceWarps * 32)
+        p.out[((int64_t)s * p.num_heads + h) * D + d] = combined_column<D>(sm, M, d) / den;
+}
+
+// Range-worker grid: a persistent grid over work items (sequence, query
+// head, slice of kMergeRows candidate rows).  A sequence's candidate rows
+// are its partition slots, then the range boundaries strictly inside it
+// (live when the boundary is no partition start and is the last worker
+// starting there).  Each CTA scans the published slice counts into a work
+// list; an item merges its slice in one round; a sequence with one slice is
+// written at once, otherwise each slice writes its (max, sum, normalised O)
+// and the last of the sequence's slices to arrive (an arrival counter the
+// partition kernel zeroed) merges them.  No CTA waits on another.
+template <int D>
+__global__ void __launch_bounds__(kReduceWarps * 32, 2)
+paged_decode_merge_kernel(const DecodeParams p) {
+    constexpr int V = D / 32;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int Hq = p.num_heads;
+    // Per sequence, computed once by the CTA: merge slices (as a prefix over
+    // sequences: the work list), partition slots, first boundary candidate,
+    // candidate count and first chunk.
+    __shared__ int work[kMaxPersistSeqs + 1];
+    __shared__ int g_nslot[kMaxPersistSeqs], g_blo[kMaxPersistSeqs];
+    __shared__ int g_total[kMaxPersistSeqs], g_xs[kMaxPersistSeqs];
+    __shared__ MergeSmem<D> sm;
+    __shared__ int is_last;
+    pdl_wait();  // the partials come from the grid launched just before
+
+    const long long T = p.chunk_prefix[p.num_seqs];
+    const long long nw = p.range_workers;
+    const int q = p.partition_size / kChunk;
+    const int32_t* E = p.worker_bounds;
+    int running = 0;
+    if (threadIdx.x == 0) work[0] = 0;
+    for (int base = 0; base < p.num_seqs; base += kReduceWarps * 32) {
+        const int s = base + threadIdx.x;
+        int v = 0;
+        if (s < p.num_seqs) {
+            const long long xs = p.chunk_prefix[s];
+            const long long cs = p.chunk_prefix[s + 1] - xs;
+            int nslot = 0, b_lo = 1, ncand = 0;
+            if (cs > 0) {
+                nslot = (int)((cs + q - 1) / q);
+                const long long lo = max(1LL, ((xs + 1) * nw + T - 1) / T);
+                const long long hi = min(nw - 1, ((xs + cs) * nw + T - 1) / T - 1);
+                b_lo = (int)lo;
+                ncand = hi >= lo ? (int)(hi - lo + 1) : 0;
+                // Two slots, or one slot and a boundary inside: split.
+                if (nslot >= 2 || ncand >= 1) v = (nslot + ncand + kMergeRows - 1) / kMergeRows;
+            }
+            g_nslot[s] = nslot;
+            g_blo[s] = b_lo;
+            g_total[s] = nslot + ncand;
+            g_xs[s] = (int)xs;
+        }
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += t;
+        }
+        if (lane == 31) sm.m[warp] = __int_as_float(v);
+        __syncthreads();
+        int before = running;
+        for (int w = 0; w < warp; ++w) before += __float_as_int(sm.m[w]);
+        if (s < p.num_seqs) work[s + 1] = before + v;
+        for (int w = 0; w < kReduceWarps; ++w) running += __float_as_int(sm.m[w]);
+        __syncthreads();
+    }
+    const int total_items = running * Hq;
+
+    for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
+        const int h = item % Hq;
+        const int gsl = item / Hq;
+        int lo = 0, hi = p.num_seqs - 1;  // largest s with work[s] <= gsl
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (work[mid] <= gsl) lo = mid; else hi = mid - 1;
+        }
+        const int s = lo;
+        const int sl = gsl - work[s];
+        const int nsl = work[s + 1] - work[s];
+        const int nslot = g_nslot[s], b_lo = g_blo[s], total = g_total[s];
+        const int xs = g_xs[s];
+        const int64_t slot_base = ((int64_t)s * Hq + h) * p.max_partitions;
+        const int64_t st_base = (int64_t)h * p.max_range_workers;
+
+        // First level: candidate rows [sl * kMergeRows, +kMergeRows), one round.
+        MergeAcc<D> a;
+        {
+            float mv[kReduceUnroll], lv[kReduceUnroll], vals[kReduceUnroll][V];
+            int e0[kReduceUnroll], e1[kReduceUnroll];
+            bool live[kReduceUnroll], in_slots[kReduceUnroll];
+#pragma unroll
+            for (int u = 0; u < kReduceUnroll; ++u) {
+                const int i = sl * kMergeRows + warp + u * kReduceWarps;
+                const bool ok = i < total;
+                in_slots[u] = i < nslot;
+                const int b = min(max(b_lo + i - nslot, 0), (int)nw - 1);
+                const int64_t r = in_slots[u] ? slot_base + i : st_base + b;
+                e0[u] = (ok && !in_slots[u]) ? E[b] : 0;
+                e1[u] = (ok && !in_slots[u]) ? E[b + 1] : 0;
+                mv[u] = ok ? (in_slots[u] ? p.tmp_m : p.st_m)[r] : -INFINITY;
+                lv[u] = ok ? (in_slots[u] ? p.tmp_l : p.st_l)[r] : 0.f;
+                load_row<D>((in_slots[u] ? p.tmp_o : p.st_o) + r * D + lane * V, ok, vals[u]);
+                live[u] = ok;
+            }
+#pragma unroll
+            for (int u = 0; u < kReduceUnroll; ++u)
+                live[u] = live[u] && (in_slots[u] ||
+                                      ((e0[u] - xs) % q != 0 && e1[u] > e0[u]));
+            a.fold(mv, lv, vals, live);
+        }
+        float M, den;
+        combine_warps<D>(a, sm, M, den);
+        float* out_row = p.out + ((int64_t)s * Hq + h) * D;
+        if (nsl == 1) {
+            for (int d = threadIdx.x; d < D; d += kReduceWarps * 32)
+                out_row[d] = combined_column<D>(sm, M, d) / den;
+            __syncthreads();  // sm is reused by the next item
+            continue;
+        }
+        const int64_t sub = ((int64_t)s * Hq + h) * p.max_slices;
+        for (int d = threadIdx.x; d < D; d += kReduceWarps * 32)
+            p.sub_o[(sub + sl) * D + d] =
+                den > 0.f ? combined_column<D>(sm, M, d) / den : 0.f;
+        if (threadIdx.x == 0) {
+            p.sub_m[sub + sl] = den > 0.f ? M : -INFINITY;
+            p.sub_l[sub + sl] = den;
+        }
+        // Publish the slice, then count it; the last slice to arrive merges.
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0)
+            is_last = atomicAdd(&p.merge_count[(int64_t)s * Hq + h], 1) == nsl - 1;
+        __syncthreads();
+        if (!is_last) continue;
+        __threadfence();
+        MergeAcc<D> b;
+        for (int i0 = warp; i0 < nsl; i0 += kReduceWarps * kReduceUnroll) {
+            float mv[kReduceUnroll], lv[kReduceUnroll], vals[kReduceUnroll][V];
+            bool live[kReduceUnroll];
+#pragma unroll
+            for (int u = 0; u < kReduceUnroll; ++u) {
+                const int i = i0 + u * kReduceWarps;
+                live[u] = i < nsl;
+                const int64_t r = sub + (live[u] ? i : 0);
+                // Written by other CTAs of this grid: read through L2.
+                mv[u] = live[u] ? __ldcg(p.sub_m + r) : -INFINITY;
+                lv[u] = live[u] ? __ldcg(p.sub_l + r) : 0.f;
+                const float* row = p.sub_o + r * D + lane * V;
+#pragma unroll
+                for (int v = 0; v < V; ++v) vals[u][v] = live[u] ? __ldcg(row + v) : 0.f;
+            }
+            b.fold(mv, lv, vals, live);
+        }
+        combine_warps<D>(b, sm, M, den);
+        for (int d = threadIdx.x; d < D; d += kReduceWarps * 32)
+            out_row[d] = combined_column<D>(sm, M, d) / den;
+        __syncthreads();
     }
 }
 
@@ -1027,9 +1173,16 @@ cudaError_t launch_typed(const DecodeParams& params, cudaStream_t stream) {
                         : launch_partition_kernel<D, BS, false>(p, tmk, tmv, stream);
     if (e != cudaSuccess) return e;
     if (p.max_partitions > 1) {
-        dim3 rgrid((unsigned)p.num_heads, (unsigned)p.num_seqs);
-        e = launch_pdl(paged_decode_reduce_kernel<D>, rgrid,
-                       dim3(kReduceWarps * 32), 0, stream, p);
+        if (p.range_workers > 0) {
+            // Persistent over the work list the partition kernel published.
+            const dim3 mgrid((unsigned)(2 * device_sm_count()));
+            e = launch_pdl(paged_decode_merge_kernel<D>, mgrid, dim3(kReduceWarps * 32), 0,
+                           stream, p);
+        } else {
+            const dim3 rgrid((unsigned)p.num_heads, (unsigned)p.num_seqs);
+            e = launch_pdl(paged_decode_reduce_kernel<D>, rgrid, dim3(kReduceWarps * 32), 0,
+                           stream, p);
+        }
         count_launch();
     }
     return e;

@@ -28,6 +28,14 @@ struct DecodeParams {
                                  // sequence (written by the partition kernel)
     int32_t* worker_bounds;      // int32 [max_range_workers+1]: first chunk
                                  // position of each worker's range (likewise)
+    // Merge of the range workers' pieces, in slices of kMergeRows candidate
+    // rows: per (sequence, query head) an arrival counter that the partition
+    // kernel zeroes, and each slice's (max, sum, normalised O).
+    int32_t* merge_count;        // int32 [B][Hq]
+    float* sub_o;                // fp32 [B][Hq][max_slices][D]
+    float* sub_m;                // fp32 [B][Hq][max_slices]
+    float* sub_l;                // fp32 [B][Hq][max_slices]
+    int max_slices;
     int* error_flags;            // nullable
     int num_seqs;
     int max_blocks_per_seq;
@@ -58,6 +66,9 @@ float log2e_scale(float scale);
 // size the straddle region.
 int decode_ctas_per_head(int num_kv_heads);
 int decode_range_workers(int num_kv_heads);
+
+// Candidate rows merged by one work item of the range merge.
+constexpr int kMergeRows = 64;
 
 // Enqueue the partition kernel (and the merge kernel when
 // max_partitions > 1).  head_size in {64,128}, block_size in {16,32};

@@ -97,6 +97,9 @@ constexpr int kQOff = kVOff + kVStages * kStageBytes;  // 2 item buffers
 constexpr int kPOff = kQOff + 2 * kQBytes;             // 2 chunk buffers x (hi | lo)
 constexpr int kMiscOff = kPOff + 2 * kPBytes;
 constexpr int kCmaxOff = kMiscOff;                     // float [32][4]
+// Largest unit weight the scheduler's counting sort handles (its histogram
+// and order live in the P buffers before the first item is published).
+constexpr int kCountSortMaxWeight = 2048;
 
 // One published item: what every role needs, and the per-row results the
 // epilogue writes out.
@@ -127,6 +130,8 @@ constexpr uint32_t kTmemO = 64;           // first O column
 constexpr float kRescaleThreshold = 24.f;  // log2 units
 constexpr float kNoMax = -FLT_MAX;        // reference of a row with no token yet
 
+static_assert((kCountSortMaxWeight + 1 + 256) * 4 <= 2 * kPBytes,
+              "the scheduler's counting sort fits in the P buffers");
 static_assert(kStageBytes % 1024 == 0 && kQBytes % 1024 == 0 && kPBytes % 1024 == 0,
               "swizzled tiles need 1024-byte alignment");
 static_assert(kSlotOff % 16 == 0 && kBarOff % 8 == 0, "alignment");
@@ -356,6 +361,7 @@ struct RowItem {
     int P;          // group mode: prefix length
     int shared_end; // group mode: end of the shared region
     int m0, nmem;   // group mode: first member of the tile, members
+    int lane_len;   // group mode: context length of member m0 + lane (lane < nmem)
 };
 
 __device__ __forceinline__ int round16(int x) { return (x + 15) & ~15; }
@@ -389,23 +395,34 @@ __device__ RowItem row_item(const MultiRowParams& p, int idx, bool report_errors
         const int m1 = min(b, m0 + mpt);
         if (m0 >= m1) return it;
         // The shared region is read through the table of the member whose
-        // context covers most of it (a shorter member's table may end first).
-        int shared_end = 0, tails = 0;
-        table_seq = m0;
-        for (int s = m0; s < m1; ++s) {
-            const int L = clamp_len(p, s, report_errors);
-            const int sh = min(P, L);
-            if (sh > shared_end) {
-                shared_end = sh;
-                table_seq = s;
+        // context covers most of it (a shorter member's table may end first;
+        // ties go to the first member).  Called by a whole warp with the same
+        // idx: lane m loads member m0 + m's length (at most 32 members per
+        // tile), and warp reductions combine them.
+        const int lane = threadIdx.x & 31;
+        const bool mem = m0 + lane < m1;
+        const int L = mem ? clamp_len(p, m0 + lane, report_errors) : 0;
+        const int sh = mem ? min(P, L) : -1;
+        int best = sh, best_s = mem ? m0 + lane : 0x7fffffff;
+        int tails = mem ? round16(L - sh) : 0;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const int ob = __shfl_xor_sync(0xffffffffu, best, o);
+            const int os = __shfl_xor_sync(0xffffffffu, best_s, o);
+            if (ob > best || (ob == best && os < best_s)) {
+                best = ob;
+                best_s = os;
             }
-            tails += round16(L - sh);
+            tails += __shfl_xor_sync(0xffffffffu, tails, o);
         }
+        const int shared_end = best;
+        table_seq = best_s;
         range_end = tails > 0 ? round16(shared_end) + tails : shared_end;
         it.P = P;
         it.shared_end = shared_end;
         it.m0 = m0;
         it.nmem = m1 - m0;
+        it.lane_len = L;
     }
     if (range_end <= 0) return it;
     it.unit = unit;
@@ -485,14 +502,14 @@ __device__ void row_of(const MultiRowParams& p, const RowItem& it, int r, int& l
         lim = L - k + j;
         row = (long long)(p.query_start_loc[s] + j) * Hq + it.g * G + R % G;
     } else {
+        // Called by the whole warp, lane = r: member m = r / G's length is
+        // in lane m of it.lane_len.
         const int mpt = kN / G;
         const int m = r / G;
-        if (m >= mpt) return;
-        const int s = p.groups.group_start[it.unit] + it.tile * mpt + m;
-        if (s >= p.groups.group_start[it.unit + 1]) return;
-        const int P = cascade_group_prefix(p.groups, it.unit, p.num_seqs, p.block_size,
-                                           nullptr, false);
-        lim = min(P, clamp_len(p, s, false)) - 1;
+        const int Lm = __shfl_sync(0xffffffffu, it.lane_len, m < 32 ? m : 0);
+        if (m >= mpt || m >= it.nmem) return;
+        const int s = it.m0 + m;
+        lim = min(it.P, Lm) - 1;
         row = (long long)s * Hq + it.g * G + r % G;
     }
 }
@@ -617,7 +634,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             int mv = 0, mt = 0, mpad = 0, mseq = -1;
             if (p.shared_prefix_mode && lane < it.nmem) {
                 mseq = it.m0 + lane;
-                const int L = clamp_len(p, mseq, false);
+                const int L = it.lane_len;
                 mt = L - min(it.P, L);
                 mpad = round16(mt);
             }
@@ -730,7 +747,86 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
 #pragma unroll
         for (int k = 0; k < kUnitRounds; ++k) one_tile = one_tile && tl[k] <= 1;
         const bool lpt = kept && __all_sync(0xffffffffu, one_tile);
-        if (lpt) {
+        int max_weight = 0;  // of the units with work
+#pragma unroll
+        for (int k = 0; k < kUnitRounds; ++k) max_weight = max(max_weight, tl[k] > 0 ? w[k] : 0);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1)
+            max_weight = max(max_weight, __shfl_xor_sync(0xffffffffu, max_weight, o));
+        if (lpt && p.num_units <= 32) {
+            // One key per lane (unit = lane): a 15-stage bitonic sort across
+            // the warp, descending; the sorted key at position pos is in
+            // lane pos.
+            long long k1 = (lane < p.num_units && tl[0] > 0)
+                               ? ((long long)w[0] << 32) | (long long)(0xFFFFFFFFu - (uint32_t)lane)
+                               : -1;
+#pragma unroll
+            for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+                for (int stride = size >> 1; stride >= 1; stride >>= 1) {
+                    const long long other = __shfl_xor_sync(0xffffffffu, k1, stride);
+                    const bool desc = (lane & size) == 0;
+                    const bool lower = (lane & stride) == 0;
+                    k1 = (lower == desc) ? max(k1, other) : min(k1, other);
+                }
+            }
+            const int live_units = __popc(__ballot_sync(0xffffffffu, k1 >= 0));
+            for (int r = 0; !stopped; ++r) {
+                const int pos = r * per_head + ((r & 1) ? per_head - 1 - j : j);
+                if (pos >= live_units) break;
+                const long long kk = __shfl_sync(0xffffffffu, k1, pos);
+                const int u = (int)(0xFFFFFFFFu - (uint32_t)(kk & 0xFFFFFFFFll));
+                if (!publish((u * p.tiles) * Hkv + g)) stopped = true;
+            }
+        } else if (lpt && max_weight <= kCountSortMaxWeight) {
+            // Counting sort by weight, heavier first and lower unit first on
+            // ties (the bitonic order below), in the P buffers, which are
+            // idle until the first item is published: a histogram of the
+            // weights, its descending prefix as start positions, then the
+            // units placed in unit order.  Unit u = k * 32 + lane.
+            int* start = reinterpret_cast<int*>(smem + kPOff);      // [weight]
+            int* order = start + kCountSortMaxWeight + 1;           // [position]
+            for (int v = lane; v <= max_weight; v += 32) start[v] = 0;
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < kUnitRounds; ++k)
+                if (k * 32 + lane < p.num_units && tl[k] > 0) atomicAdd(&start[w[k]], 1);
+            __syncwarp();
+            int live_units = 0;
+            for (int top = max_weight; top >= 0; top -= 32) {
+                const int v = top - lane;  // lane 0 holds the heaviest weight of the block
+                const int c = v >= 0 ? start[v] : 0;
+                int incl = c;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += t;
+                }
+                __syncwarp();
+                if (v >= 0) start[v] = live_units + incl - c;
+                live_units += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            __syncwarp();
+            const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+            for (int k = 0; k < kUnitRounds; ++k) {
+                const bool live = k * 32 + lane < p.num_units && tl[k] > 0;
+                const int key = live ? w[k] : -1;
+                const unsigned same = __match_any_sync(0xffffffffu, key);
+                if (live) order[start[key] + __popc(same & lt)] = k * 32 + lane;
+                __syncwarp();
+                if (live && (same & lt) == 0) start[key] += __popc(same);
+                __syncwarp();
+            }
+            for (int r = 0; !stopped; ++r) {
+                const int pos = r * per_head + ((r & 1) ? per_head - 1 - j : j);
+                if (pos >= live_units) break;
+                const int u = order[pos];
+                if (!publish((u * p.tiles) * Hkv + g)) stopped = true;
+            }
+        } else if (lpt) {
+            // Weights too large for the counting sort: bitonic sort of
+            // 64-bit keys across the warp.
             long long key[8];  // weight << 32 | (~unit): heavier first, then lower unit
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
