@@ -272,10 +272,9 @@ int pa_multi_query_attention(float* out, const void* q, const void* k_cache,
  *                   needs no initialisation.  It holds the per-sequence
  *                   pass's split-KV scratch only.
  *   other arguments as for pa_decode_attention.
- * The group pass and the per-sequence pass write disjoint outputs and
- * classify every sequence with the same rule from group_start / prefix_lens,
- * so the per-sequence pass may run while the group pass is still running
- * (on the SMs that pass leaves free).
+ * The per-sequence pass runs first, then the group pass; they write
+ * disjoint outputs and classify every sequence with the same rule from
+ * group_start / prefix_lens, so neither reads what the other writes.
  * Supports head_size 128, block_size in {16, 32}, num_heads / num_kv_heads
  * in 1..8 (head_size 64 returns PA_ERR_UNSUPPORTED).  Returns PA_OK or a
  * negative pa_status; run-to-run results are bitwise deterministic.

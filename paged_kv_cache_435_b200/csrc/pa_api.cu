@@ -468,9 +468,9 @@ int pa_decode_attention_shared_prefix(
     const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
     pa::CascadeGroups groups{group_start, prefix_lens, num_groups, mgs};
+    pa::MultiRowParams r{};
     if (num_groups > 0) {
         const int per_tile = pa::kMultiRowTile / G;
-        pa::MultiRowParams r{};
         r.out = out;
         r.q = static_cast<const uint16_t*>(q);
         r.k_cache = static_cast<const uint16_t*>(k_cache);
@@ -493,7 +493,6 @@ int pa_decode_attention_shared_prefix(
         r.scale_log2 = pa::log2e_scale(scale);
         if ((long long)num_groups * r.tiles * num_kv_heads > 0x7fffffffLL)
             return PA_ERR_UNSUPPORTED;
-        if (pa::launch_paged_multi_row(r, st) != cudaSuccess) return PA_ERR_CUDA;
     }
 
     pa::DecodeParams p{};
@@ -518,8 +517,14 @@ int pa_decode_attention_shared_prefix(
     p.block_size = block_size;
     p.has_groups = num_groups > 0;
     p.groups = groups;
-    cudaError_t e = pa::launch_paged_decode(p, head_size, block_size, st);
-    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    // The per-sequence pass first: it attends the sequences outside every
+    // group and has little to do when every sequence is grouped; the group
+    // pass, launched behind it, writes the other outputs.
+    if (pa::launch_paged_decode(p, head_size, block_size, st) != cudaSuccess)
+        return PA_ERR_CUDA;
+    if (num_groups > 0 && pa::launch_paged_multi_row(r, st) != cudaSuccess)
+        return PA_ERR_CUDA;
+    return PA_OK;
 }
 
 int pa_swap_blocks(const void* const* src_caches, void* const* dst_caches,

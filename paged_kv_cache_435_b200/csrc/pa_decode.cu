@@ -293,12 +293,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         return;
     }
     // Launched behind the cache write: nothing global is read before the
-    // preceding grid has completed.  In the shared-prefix call the
-    // preceding grid is the group pass, which this pass needs nothing from
-    // (the outputs are disjoint, the grouping is recomputed here); it may
-    // run beside it, since the group pass lets it launch only after its own
-    // wait for the cache write.
-    if (!kSkip) pdl_wait();
+    // preceding grid has completed.
+    pdl_wait();
     pdl_launch_dependents();
 
     Range rg{0, 0, 1, 0};

@@ -783,7 +783,8 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             // ties (the bitonic order below), in the P buffers, which are
             // idle until the first item is published: a histogram of the
             // weights, its descending prefix as start positions, then the
-            // units placed in unit order.  Unit u = k * 32 + lane.
+            // units placed in unit order.  Unit u = k * 32 + lane.  Nothing
+            // reads the buffers after the first publication (below).
             int* start = reinterpret_cast<int*>(smem + kPOff);      // [weight]
             int* order = start + kCountSortMaxWeight + 1;           // [position]
             for (int v = lane; v <= max_weight; v += 32) start[v] = 0;
@@ -818,10 +819,26 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 if (live && (same & lt) == 0) start[key] += __popc(same);
                 __syncwarp();
             }
-            for (int r = 0; !stopped; ++r) {
-                const int pos = r * per_head + ((r & 1) ? per_head - 1 - j : j);
-                if (pos >= live_units) break;
-                const int u = order[pos];
+            // This CTA's units in snake order, taken into registers before
+            // the first publication: the softmax warps write P into these
+            // buffers as soon as an item is out.  The CTA's r-th item
+            // (r = e * 32 + lane) is position r * per_head + (r odd ?
+            // per_head - 1 - j : j); at most 256 units.
+            int mine[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int r = e * 32 + lane;
+                const long long pos = (long long)r * per_head + ((r & 1) ? per_head - 1 - j : j);
+                mine[e] = pos < live_units ? order[pos] : -1;
+            }
+            __syncwarp();
+            for (int r = 0; r < 256 && !stopped; ++r) {
+                int own = -1;
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if (e == (r >> 5)) own = mine[e];
+                const int u = __shfl_sync(0xffffffffu, own, r & 31);
+                if (u < 0) break;
                 if (!publish((u * p.tiles) * Hkv + g)) stopped = true;
             }
         } else if (lpt) {
