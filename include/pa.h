@@ -253,9 +253,14 @@ int pa_multi_query_attention(float* out, const void* q, const void* k_cache,
  * for all members' query rows, then each member's private tail for that
  * member's rows only: sequence s with context length L attends its first
  * min(prefix_lens[i], L) tokens through the shared blocks and the rest
- * through its own table, in one online softmax.  Sequences outside every
- * group, and groups whose description is invalid (reported with
- * PA_DEVERR_PREFIX), are attended by the decode kernel as by
+ * through its own table, in one online softmax.  When there are at most 256
+ * groups, each fits one pass (at most 32 / (num_heads / num_kv_heads)
+ * members) and one pass alone is longer than 1.5 times an SM's even share
+ * of the kv head's work, the passes are dealt to the SMs by 128-token
+ * chunks: a long pass is cut into pieces on several SMs, whose partial (max,
+ * sum, output) rows are merged by the piece that finishes last.  Sequences
+ * outside every group, and groups whose description is invalid (reported
+ * with PA_DEVERR_PREFIX), are attended by the decode kernel as by
  * pa_decode_attention.
  *
  *   group_start     int32 [num_groups + 1], device, non-decreasing, in
@@ -268,13 +273,19 @@ int pa_multi_query_attention(float* out, const void* q, const void* k_cache,
  *                   without the group pass.
  *   workspace       device buffer of at least
  *                   pa_shared_prefix_workspace_size(...) bytes, 256-byte
- *                   aligned (NULL allowed when that size is 0); scratch,
- *                   needs no initialisation.  It holds the per-sequence
- *                   pass's split-KV scratch only.
+ *                   aligned; scratch, needs no initialisation.  It holds
+ *                   the per-sequence pass's split-KV scratch, then the
+ *                   group pass's pieces: (num_seqs + SMs / num_kv_heads)
+ *                   x num_kv_heads x 32 rows of head_size + 2 floats, and
+ *                   num_seqs x num_kv_heads arrival counters, which the
+ *                   per-sequence pass clears.  The size depends on the
+ *                   current device's SM count: query it on the device the
+ *                   call runs on.
  *   other arguments as for pa_decode_attention.
  * The per-sequence pass runs first, then the group pass; they write
  * disjoint outputs and classify every sequence with the same rule from
- * group_start / prefix_lens, so neither reads what the other writes.
+ * group_start / prefix_lens, so the group pass reads nothing of the
+ * per-sequence pass's but the cleared counters.
  * Supports head_size 128, block_size in {16, 32}, num_heads / num_kv_heads
  * in 1..8 (head_size 64 returns PA_ERR_UNSUPPORTED).  Returns PA_OK or a
  * negative pa_status; run-to-run results are bitwise deterministic.

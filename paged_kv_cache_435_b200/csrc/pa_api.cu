@@ -130,6 +130,27 @@ size_t workspace_bytes_for(int num_seqs, int num_heads, int num_kv_heads,
                         max_partitions).total;
 }
 
+// Shared-prefix call, after the split scratch: the group pass's pieces of
+// split items, piece_o [S][Hkv][32][D], piece_ml [S][Hkv][32][2] (S = groups
+// + CTAs per kv head, groups bounded by the sequences), and the items'
+// arrival counters [groups][Hkv].
+struct PieceLayout {
+    size_t o, ml, count, total;
+    int slots;
+};
+
+PieceLayout piece_layout(size_t base, int num_seqs, int num_kv_heads, int head_size) {
+    PieceLayout L{};
+    L.slots = num_seqs + multi_row_ctas_per_head(num_kv_heads);
+    const size_t rows = (size_t)L.slots * num_kv_heads * kMultiRowTile;
+    size_t off = align256(base);
+    L.o = off;     off = align256(off + rows * head_size * 4);
+    L.ml = off;    off = align256(off + rows * 2 * 4);
+    L.count = off; off = align256(off + (size_t)num_seqs * num_kv_heads * 4);
+    L.total = off;
+    return L;
+}
+
 // Point the decode parameters at the split scratch inside `ws`.
 void assign_split(DecodeParams& p, unsigned char* ws, const SplitLayout& L) {
     p.max_range_workers = L.range_workers;
@@ -408,8 +429,9 @@ size_t pa_shared_prefix_workspace_size(int num_seqs, int num_heads,
                                               head_size, block_size,
                                               max_context_len, partition_size);
     if (part <= 0 || num_heads <= 0 || head_size <= 0) return 0;
-    return pa::workspace_bytes_for(num_seqs, num_heads, num_kv_heads, head_size,
-                                   pa::num_partitions(max_context_len, part));
+    const size_t split = pa::workspace_bytes_for(num_seqs, num_heads, num_kv_heads, head_size,
+                                                 pa::num_partitions(max_context_len, part));
+    return pa::piece_layout(split, num_seqs, num_kv_heads, head_size).total;
 }
 
 int pa_decode_attention_shared_prefix(
@@ -456,10 +478,9 @@ int pa_decode_attention_shared_prefix(
     if (np > pa::kMaxGridYZ) return PA_ERR_INVALID_ARG;
     const pa::SplitLayout lay =
         pa::split_layout(num_seqs, num_heads, num_kv_heads, head_size, np);
-    if (lay.total > 0) {
-        if (!workspace || workspace_bytes < lay.total) return PA_ERR_WORKSPACE;
-        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PA_ERR_INVALID_ARG;
-    }
+    const pa::PieceLayout plan = pa::piece_layout(lay.total, num_seqs, num_kv_heads, head_size);
+    if (!workspace || workspace_bytes < plan.total) return PA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PA_ERR_INVALID_ARG;
     unsigned char* ws = static_cast<unsigned char*>(workspace);
     const int G = num_heads / num_kv_heads;
     // A group cannot hold more than num_seqs sequences: the bound changes
@@ -493,6 +514,12 @@ int pa_decode_attention_shared_prefix(
         r.scale_log2 = pa::log2e_scale(scale);
         if ((long long)num_groups * r.tiles * num_kv_heads > 0x7fffffffLL)
             return PA_ERR_UNSUPPORTED;
+        if (num_groups <= num_seqs) {  // the piece region holds this many units
+            r.piece_o = reinterpret_cast<float*>(ws + plan.o);
+            r.piece_ml = reinterpret_cast<float*>(ws + plan.ml);
+            r.piece_count = reinterpret_cast<int32_t*>(ws + plan.count);
+            r.piece_slots = plan.slots;
+        }
     }
 
     pa::DecodeParams p{};
@@ -517,6 +544,10 @@ int pa_decode_attention_shared_prefix(
     p.block_size = block_size;
     p.has_groups = num_groups > 0;
     p.groups = groups;
+    if (r.piece_count != nullptr) {
+        p.zero_ints = r.piece_count;
+        p.zero_count = (long long)num_groups * num_kv_heads;
+    }
     // The per-sequence pass first: it attends the sequences outside every
     // group and has little to do when every sequence is grouped; the group
     // pass, launched behind it, writes the other outputs.

@@ -297,6 +297,13 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
     pdl_wait();
     pdl_launch_dependents();
 
+    if (p.zero_count > 0) {
+        // Each CTA clears a contiguous share.
+        const long long ctas = (long long)gridDim.x * gridDim.y * gridDim.z;
+        const long long me = ((long long)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+        const long long z0 = p.zero_count * me / ctas, z1 = p.zero_count * (me + 1) / ctas;
+        for (long long z = z0 + threadIdx.x; z < z1; z += kThreads) p.zero_ints[z] = 0;
+    }
     Range rg{0, 0, 1, 0};
     uint32_t* grouped_bits = reinterpret_cast<uint32_t*>(smem + C::kGroupedOff);
     if (kPersist && kSkip) {

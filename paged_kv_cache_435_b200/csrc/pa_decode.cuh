@@ -56,6 +56,10 @@ struct DecodeParams {
     // classify a sequence with the same functions (pa_cascade.cuh).
     bool has_groups;
     CascadeGroups groups;
+    // Ints the partition kernel zeroes before anything else reads them (the
+    // group pass's arrival counters, which it reads only after this grid).
+    int32_t* zero_ints;
+    long long zero_count;
 };
 
 // scale * log2(e): logits are kept in the log2 domain (exp2f).

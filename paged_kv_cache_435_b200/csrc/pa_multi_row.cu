@@ -44,14 +44,20 @@
 //              every unit is one item (a bitonic sort across the warp), else
 //              the items whose cumulative weight starts in their share; all
 //              heads walk the batch in the same order, so the head slices of
-//              a block are read together.  For each item it works out the
-//              token range, block-table rows, each row's visible tokens and
-//              output row into a 4-slot shared-memory ring and copies the Q
-//              rows (cp.async), so no other warp waits on a global load at an
-//              item boundary.
-// Online softmax with a lazy reference: an item's rows start from the logit
-// of the item's first token (every row sees it, so each row's sum is at
-// least 1), which thread 0 publishes through shared memory.  Every chunk,
+//              a block are read together.  In the group pass, when one item
+//              alone is longer than 1.5 CTA shares, the items are instead cut
+//              into pieces at 128-token chunk boundaries so that every CTA of
+//              the head gets an even share; a piece writes its rows' partial
+//              (reference, sum, normalised O) and the last piece of an item to
+//              finish merges them into the output.  For each item or piece
+//              it works out the token range, block-table rows, each row's
+//              visible tokens and output row into a 4-slot shared-memory ring
+//              and copies the Q rows (cp.async), so no other warp waits on a
+//              global load at an item boundary.
+// Online softmax with a lazy reference: each row starts from the logit of its
+// first visible token of the item or piece (so its sum is at least 1),
+// published through shared memory by the thread that owns that token in the
+// chunk that holds it; until then the row's tokens are all masked.  Every chunk,
 // one barrier-reduction over the 4 warps (bar.red.popc) asks whether any
 // row's logit exceeds its reference by more than 2^24 (weights stay below
 // 2^24, far from fp32 overflow, and the split of P keeps its relative
@@ -67,7 +73,6 @@
 // barrier, and TMEM is released on every exit path.
 #include <cuda.h>
 
-#include <cfloat>
 #include <cstdint>
 #include <mutex>
 
@@ -104,19 +109,36 @@ constexpr int kCountSortMaxWeight = 2048;
 // One published item: what every role needs, and the per-row results the
 // epilogue writes out.
 struct ItemSlot {
-    int table_seq, g, range_end, nch;   // nch < 0: no further items
+    int table_seq, g, range_end, nch;   // nch: one past the last chunk of this
+                                        // piece (< 0: no further items)
+    int c0;                             // first chunk of this piece
+    int piece;                          // -1: the whole item (writes the
+                                        // output); else its partial's slot
+    int unit, item_n;                   // split item: group, its chunks
+    int item_a, axis_len;               // split item: first position, axis
+                                        // length (see the split deal)
+    int nref;                           // entries of refc / refm
+    uint32_t live_rows;                 // rows that exist (bit r: row r)
+    float m_fin[32], l_fin[32];         // rows: reference and sum at the end
+    float ref[32];                      // rows: logit at the first visible token
+    int first[32];                      // rows: first visible token of the
+                                        // piece (-1: none)
+    int refc[32];                       // chunks holding first tokens, rising,
+    uint32_t refm[32];                  // and the rows whose first token each holds
     int min_lim, nmem, shared_r16, P;   // smallest row limit; members (group
                                         // mode); end of the shared region
                                         // rounded to 16; prefix length
+    int arrived, pad_[3];               // pieces counted before this one
     int lim[32];                        // rows: last visible shared token
-    int tail_lo[32], tail_hi[32];       // rows: their member's tail [lo, hi)
+    int mem_tend[32];                   // members: end of the unpadded tail
+    uint32_t mem_rows[32];              // members: their rows (bit r: row r)
     int mem_seq[32];                    // members: sequence
     int mem_v[32], mem_vend[32];        // members: tail pieces [v, vend)
     long long row[32];                  // q / out row of each row (-1: none)
     float red_l[32][4];                 // per-warp partial row sums
     float inv_l[32];                    // 1 / row sum (0 for an empty row)
 };
-static_assert(sizeof(ItemSlot) == 1696, "slot layout");
+static_assert(sizeof(ItemSlot) == 2512 && sizeof(ItemSlot) % 16 == 0, "slot layout");
 
 constexpr int kSlotOff = kCmaxOff + 512;
 constexpr int kBarOff = kSlotOff + kSlots * (int)sizeof(ItemSlot);
@@ -128,7 +150,6 @@ constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16;
 constexpr uint32_t kTmemCols = 256;       // S0 | S1 | O0 (hi, lo) | O1 (hi, lo)
 constexpr uint32_t kTmemO = 64;           // first O column
 constexpr float kRescaleThreshold = 24.f;  // log2 units
-constexpr float kNoMax = -FLT_MAX;        // reference of a row with no token yet
 
 static_assert((kCountSortMaxWeight + 1 + 256) * 4 <= 2 * kPBytes,
               "the scheduler's counting sort fits in the P buffers");
@@ -454,8 +475,11 @@ __device__ __forceinline__ void query_unit_work(const MultiRowParams& p, int L, 
     w = (L + kTok - 1) / kTok + 1;
 }
 
+// Group mode also returns, for a one-tile group, its item's exact chunk
+// count (as row_item computes it), else 0.
 __device__ __forceinline__ void unit_work(const MultiRowParams& p, int u,
-                                          bool report_errors, int& tiles, int& w) {
+                                          bool report_errors, int& tiles, int& w, int& nch) {
+    nch = 0;
     if (!p.shared_prefix_mode) {
         const int L = clamp_len(p, u, report_errors);
         const int k = clamp_queries(p, u, L, report_errors);
@@ -469,17 +493,27 @@ __device__ __forceinline__ void unit_work(const MultiRowParams& p, int u,
         const int mpt = kN / p.group;
         tiles = P > 0 ? (members + mpt - 1) / mpt : 0;
         long long tails = 0;
+        int shared_end = 0;
         if (P > 0)
             for (int s0 = a; s0 < a + members; s0 += 8) {  // 8 loads in flight
                 int Ls[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
-                    Ls[e] = s0 + e < a + members ? clamp_len(p, s0 + e, report_errors) : P;
+                    Ls[e] = s0 + e < a + members ? clamp_len(p, s0 + e, report_errors) : -1;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) tails += round16(Ls[e] - min(P, Ls[e]));
+                for (int e = 0; e < 8; ++e)
+                    if (Ls[e] >= 0) {
+                        tails += round16(Ls[e] - min(P, Ls[e]));
+                        shared_end = max(shared_end, min(P, Ls[e]));
+                    }
             }
         const long long per_tile = tiles > 0 ? tails / tiles : 0;
         w = (int)((P + per_tile + kTok - 1) / kTok) + 1;
+        if (tiles == 1) {
+            const long long range_end =
+                tails > 0 ? round16(shared_end) + tails : (long long)shared_end;
+            nch = (int)((range_end + kTok - 1) / kTok);
+        }
     }
     tiles = min(tiles, p.tiles);
 }
@@ -512,6 +546,34 @@ __device__ void row_of(const MultiRowParams& p, const RowItem& it, int r, int& l
         lim = min(it.P, Lm) - 1;
         row = (long long)s * Hq + it.g * G + r % G;
     }
+}
+
+// Split deal of the shared-prefix group pass.  Per kv head the items (one
+// per group, one tile each) lie end to end on an axis in group order: item
+// u takes positions [a, a + n + 1), the first for its fixed cost, then one
+// per 128-token chunk (chunk c at a + 1 + c).  CTA j of the head's `per`
+// owns positions [B(j), B(j + 1)), B(j) = floor(j T / per), T the axis
+// length, and attends the chunks whose positions it owns: a piece of an item
+// is a run of chunks with one owner.  The piece at an item's first chunk
+// writes its partial to slot u; a piece that starts at chunk c >= 1 does so
+// only where a CTA's range starts (B(j) = a + 1 + c), and takes slot
+// units + j.
+// The deal keeps (T + 1) * per within int, so these products do not overflow.
+__device__ __forceinline__ int axis_bound(int T, int per, int j) { return j * T / per; }
+
+// Calls f(j) for every CTA j whose range starts inside item (a, n) at
+// chunk 1 .. n - 1 (each such piece's slot is units + j); CTAs with empty
+// ranges own nothing and are skipped.
+template <typename F>
+__device__ __forceinline__ void for_each_inner_piece(int a, int n, int T, int per, F&& f) {
+    if (n <= 1 || T <= 0) return;
+    // B(j) in [a + 2, a + n].
+    int jlo = ((a + 2) * per + T - 1) / T;
+    int jhi = ((a + n + 1) * per + T - 1) / T - 1;
+    if (jlo < 1) jlo = 1;
+    if (jhi > per - 1) jhi = per - 1;
+    for (int j = jlo; j <= jhi; ++j)
+        if (axis_bound(T, per, j + 1) > axis_bound(T, per, j)) f(j);
 }
 
 template <int BS>
@@ -591,14 +653,25 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
     if (warp == 7) {
         // -------------------------------------------------------- scheduler
         int live = 0;
-        // Publish item idx (idx < 0: the end marker); false on abort.
-        auto publish = [&](int idx) -> bool {
+        // A split item's piece: chunks [c0, c1) of the item at position a
+        // of an axis of length T (see the split deal); slot -1 for the whole.
+        struct Piece {
+            int c0, c1, slot, n, a, T;
+        };
+        // Publish item idx (idx < 0: the end marker), whole or one piece of
+        // it; false on abort.
+        auto publish = [&](int idx, const Piece& pc) -> bool {
             const bool end = idx < 0;
             RowItem it;
             it.unit = -1;
             if (!end) {
                 it = row_item(p, idx, false);
                 if (it.unit < 0) return true;
+            }
+            if (!end && pc.slot >= 0 &&
+                (pc.n != it.nch || pc.c0 < 0 || pc.c1 <= pc.c0 || pc.c1 > it.nch)) {
+                if (lane == 0) report(p.error_flags, PA_DEVERR_INTERNAL);
+                return true;
             }
             const int s = live % kSlots;
             bool good = true;
@@ -645,19 +718,75 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 if (lane >= o) incl += t;
             }
             mv = shared_r16 + incl - mpad;
+            // Member lane's rows are lane * G .. lane * G + G - 1 (those that exist).
+            const uint32_t live_rows = __ballot_sync(0xffffffffu, row >= 0);
+            const int G = p.group;
             S.mem_seq[lane] = mseq;
             S.mem_v[lane] = mv;
             S.mem_vend[lane] = mv + mpad;
-            const int my_m = row >= 0 && p.shared_prefix_mode ? lane / p.group : 0;
+            S.mem_tend[lane] = mv + mt;
+            S.mem_rows[lane] = (p.shared_prefix_mode && lane < it.nmem && lane * G < 32)
+                                   ? (((1u << G) - 1u) << (lane * G)) & live_rows
+                                   : 0u;
+            const int my_m = row >= 0 && p.shared_prefix_mode ? lane / G : 0;
             const int t_lo = __shfl_sync(0xffffffffu, mv, my_m);
             const int t_len = __shfl_sync(0xffffffffu, mt, my_m);
-            S.tail_lo[lane] = row >= 0 && p.shared_prefix_mode ? t_lo : 0;
-            S.tail_hi[lane] = row >= 0 && p.shared_prefix_mode ? t_lo + t_len : 0;
+            const int tail_lo = row >= 0 && p.shared_prefix_mode ? t_lo : 0;
+            const int tail_hi = row >= 0 && p.shared_prefix_mode ? t_lo + t_len : 0;
+            // This piece's chunks.  The deal took a split item's count from
+            // the same lengths; a piece that does not fit its item is an
+            // internal error and is not streamed.
+            const bool split = pc.slot >= 0;
+            const int c0 = split ? pc.c0 : 0;
+            const int c1 = split ? pc.c1 : it.nch;
+            // Row lane's first visible token in the piece: the piece's first
+            // token if the row sees it (shared region, or every token up to
+            // its limit in multi-query mode), else the first token of its own
+            // tail inside the piece.
+            int first = -1;
+            if (row >= 0) {
+                const int t0 = c0 * kTok;
+                if (t0 <= lim) {
+                    first = t0;
+                } else if (tail_hi > tail_lo) {
+                    const int f = max(t0, tail_lo);
+                    if (f < tail_hi && f < c1 * kTok) first = f;
+                }
+            }
+            S.first[lane] = first;
+            // The chunks that hold first tokens, rising, each with its rows:
+            // entry k in lane k.
+            const int fc = first >= 0 ? first / kTok : 0x7fffffff;
+            int nref = 0, last = -1, refc = 0;
+            uint32_t refm = 0;
+            for (;;) {
+                int cm = fc > last ? fc : 0x7fffffff;
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) cm = min(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+                if (cm == 0x7fffffff) break;
+                const uint32_t m = __ballot_sync(0xffffffffu, fc == cm);
+                if (lane == nref) {
+                    refc = cm;
+                    refm = m;
+                }
+                ++nref;
+                last = cm;
+            }
+            S.refc[lane] = refc;
+            S.refm[lane] = refm;
             if (lane == 0) {
                 S.table_seq = it.table_seq;
                 S.g = it.g;
                 S.range_end = it.range_end;
-                S.nch = it.nch;
+                S.nch = c1;
+                S.c0 = c0;
+                S.piece = split ? pc.slot : -1;
+                S.unit = it.unit;
+                S.item_n = split ? pc.n : it.nch;  // the deal's count (pieces)
+                S.item_a = pc.a;
+                S.axis_len = pc.T;
+                S.nref = nref;
+                S.live_rows = live_rows;
                 S.min_lim = ml;
                 S.nmem = p.shared_prefix_mode ? it.nmem : 0;
                 S.shared_r16 = shared_r16;
@@ -679,6 +808,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             ++live;
             return true;
         };
+        const Piece kWhole = {0, 0, -1, 0, 0, 0};
 
         // Deal by work.  CTA b serves kv head g = b % Hkv as the j-th of the
         // head's per_head CTAs.  The head's items are ordered (unit, tile);
@@ -695,6 +825,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
         const int per_head = gridDim.x / Hkv;
         constexpr int kUnitRounds = 8;
         int tl[kUnitRounds], w[kUnitRounds];
+        int nc[kUnitRounds];  // group mode, one-tile groups: exact chunk counts
         auto gather = [&](int base, bool report_errors) {
             if (!p.shared_prefix_mode) {
                 // Every round's lengths first: the error reports below are
@@ -713,6 +844,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 for (int k = 0; k < kUnitRounds; ++k) {
                     tl[k] = 0;
                     w[k] = 0;
+                    nc[k] = 0;
                     if (base + k * 32 + lane < p.num_units)
                         query_unit_work(p, Lr[k], q1[k] - q0[k], report_errors, tl[k], w[k]);
                 }
@@ -723,7 +855,8 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 const int u = base + k * 32 + lane;
                 tl[k] = 0;
                 w[k] = 0;
-                if (u < p.num_units) unit_work(p, u, report_errors, tl[k], w[k]);
+                nc[k] = 0;
+                if (u < p.num_units) unit_work(p, u, report_errors, tl[k], w[k], nc[k]);
             }
         };
         long long T = 0;
@@ -753,7 +886,69 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1)
             max_weight = max(max_weight, __shfl_xor_sync(0xffffffffu, max_weight, o));
-        if (lpt && p.num_units <= 32) {
+        // Split deal (group mode with a piece region, every group one item):
+        // the head's items on the position axis described above
+        // for_each_inner_piece, in group order; this CTA attends the chunks
+        // whose positions it owns.
+        // Split only when one item alone exceeds 1.5 times a CTA's even
+        // share: whole items dealt longest first balance to within about one
+        // item, and a piece costs its partial write, reference barriers and
+        // a share of the merge.
+        long long Tl = 0;  // the split deal's axis length
+        int wmax = 0;      // its longest item
+#pragma unroll
+        for (int k = 0; k < kUnitRounds; ++k) {
+            Tl += nc[k] > 0 ? nc[k] + 1 : 0;
+            wmax = max(wmax, nc[k] > 0 ? nc[k] + 1 : 0);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            Tl += __shfl_xor_sync(0xffffffffu, Tl, o);
+            wmax = max(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
+        }
+        const bool split_deal = lpt && p.shared_prefix_mode && p.piece_o != nullptr &&
+                                (long long)p.num_units + per_head <= p.piece_slots &&
+                                (Tl + 1) * per_head <= 0x7fffffffLL &&
+                                2LL * wmax * per_head > 3LL * Tl;
+        if (split_deal) {
+            const int Ta = (int)Tl;
+            const int A = axis_bound(Ta, per_head, j);
+            const int Bd = axis_bound(Ta, per_head, j + 1);
+            int run = 0;  // first position of this round's units
+            for (int k = 0; k < kUnitRounds && !stopped && run < Bd; ++k) {
+                int n = 0;
+#pragma unroll
+                for (int e = 0; e < kUnitRounds; ++e)
+                    if (e == k) n = nc[e];
+                const int wgt = n > 0 ? n + 1 : 0;
+                int incl = wgt;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += t;
+                }
+                const int a = run + incl - wgt;
+                const int c0 = min(max(A - a - 1, 0), n);
+                const int c1 = min(max(Bd - a - 1, 0), n);
+                unsigned todo = __ballot_sync(0xffffffffu, n > 0 && c1 > c0);
+                while (todo != 0 && !stopped) {
+                    const int i = __ffs(todo) - 1;
+                    todo &= todo - 1;
+                    Piece pc;
+                    pc.c0 = __shfl_sync(0xffffffffu, c0, i);
+                    pc.c1 = __shfl_sync(0xffffffffu, c1, i);
+                    pc.n = __shfl_sync(0xffffffffu, n, i);
+                    pc.a = __shfl_sync(0xffffffffu, a, i);
+                    pc.T = Ta;
+                    const int u = k * 32 + i;
+                    pc.slot = (pc.c0 == 0 && pc.c1 == pc.n) ? -1
+                              : pc.c0 == 0                  ? u
+                                                            : p.num_units + j;
+                    if (!publish((u * p.tiles) * Hkv + g, pc)) stopped = true;
+                }
+                run += __shfl_sync(0xffffffffu, incl, 31);
+            }
+        } else if (lpt && p.num_units <= 32) {
             // One key per lane (unit = lane): a 15-stage bitonic sort across
             // the warp, descending; the sorted key at position pos is in
             // lane pos.
@@ -776,7 +971,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 if (pos >= live_units) break;
                 const long long kk = __shfl_sync(0xffffffffu, k1, pos);
                 const int u = (int)(0xFFFFFFFFu - (uint32_t)(kk & 0xFFFFFFFFll));
-                if (!publish((u * p.tiles) * Hkv + g)) stopped = true;
+                if (!publish((u * p.tiles) * Hkv + g, kWhole)) stopped = true;
             }
         } else if (lpt && max_weight <= kCountSortMaxWeight) {
             // Counting sort by weight, heavier first and lower unit first on
@@ -839,7 +1034,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                     if (e == (r >> 5)) own = mine[e];
                 const int u = __shfl_sync(0xffffffffu, own, r & 31);
                 if (u < 0) break;
-                if (!publish((u * p.tiles) * Hkv + g)) stopped = true;
+                if (!publish((u * p.tiles) * Hkv + g, kWhole)) stopped = true;
             }
         } else if (lpt) {
             // Weights too large for the counting sort: bitonic sort of
@@ -877,7 +1072,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                     if (e == (pos & 7)) mine = key[e];
                 const long long kk = __shfl_sync(0xffffffffu, mine, pos >> 3);
                 const int u = (int)(0xFFFFFFFFu - (uint32_t)(kk & 0xFFFFFFFFll));
-                if (!publish((u * p.tiles) * Hkv + g)) stopped = true;
+                if (!publish((u * p.tiles) * Hkv + g, kWhole)) stopped = true;
             }
         }
         long long pos = 0;  // start of the current batch of 32 units
@@ -909,13 +1104,13 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                     for (int t = 0; t < ti && !stopped; ++t) {
                         const long long q = us + (long long)t * wi;
                         if (q < lo || q >= hi) continue;
-                        if (!publish(((base + i) * p.tiles + t) * Hkv + g)) stopped = true;
+                        if (!publish(((base + i) * p.tiles + t) * Hkv + g, kWhole)) stopped = true;
                     }
                 }
             }
             pos += total;
         }
-        if (!stopped) (void)publish(-1);
+        if (!stopped) (void)publish(-1, kWhole);
     } else if (warp == 4 || warp == 5) {
         // ------------------------------------------------ K / V producers
         const bool is_v = warp == 5;
@@ -935,12 +1130,13 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             const ItemSlot& SL = slots[sl];
             const int nch = SL.nch;
             if (nch < 0) break;
+            const int c0 = SL.c0;
             const int g = SL.g;
             const int range_end = SL.range_end;
             const int shared_r16 = SL.shared_r16;
             int win = -1;  // lane l: slot of 16-token piece l of chunks c..c+3
-            for (int c = 0; c < nch; ++c) {
-                if ((c & 3) == 0) {
+            for (int c = c0; c < nch; ++c) {
+                if (((c - c0) & 3) == 0) {
                     // Virtual token v0: shared (the group's table), or a
                     // member's tail (that member's table, after the prefix).
                     const int v0 = (c * 8 + lane) * 16;
@@ -981,7 +1177,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                     ok = false;
                     break;
                 }
-                const int sl16 = __shfl_sync(0xffffffffu, win, (c & 3) * 8 + (lane & 7));
+                const int sl16 = __shfl_sync(0xffffffffu, win, ((c - c0) & 3) * 8 + (lane & 7));
                 const bool mine = lane < 8 && sl16 >= 0;
                 const uint32_t pieces = __popc(__ballot_sync(0xffffffffu, mine));
                 if (lane == 0) mbar_arrive_expect_tx(&full[stage], pieces * 2 * 2048);
@@ -1063,8 +1259,9 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             }
             const int nch = slots[sl].nch;
             if (nch < 0) break;
+            const int c0 = slots[sl].c0;
             const uint64_t qd = q_desc0 + (uint64_t)(((item & 1) * kQBytes) >> 4);
-            for (int c = 0; c < nch; ++c, ++n) {
+            for (int c = c0; c < nch; ++c, ++n) {
                 bool good = true;
                 if (lane == 0) {
                     good = wait_bar(&k_full[n % kKStages], (n / kKStages) & 1);
@@ -1104,7 +1301,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 Pending pn;
                 pn.n = n;
                 pn.item = item;
-                pn.first = c == 0;
+                pn.first = c == c0;
                 pn.last = c == nch - 1;
                 if (npend == 0) pend0 = pn; else pend1 = pn;
                 ++npend;
@@ -1132,14 +1329,97 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 const float4 v = *reinterpret_cast<const float4*>(S.red_l[lane]);
                 const float l = (v.x + v.y) + (v.z + v.w);
                 S.inv_l[lane] = l > 0.f ? 1.f / l : 0.f;
+                S.l_fin[lane] = l;
+            }
+        };
+        // Merge of a split item's pieces into its output rows (thread = d),
+        // by the piece that arrived last: per row, the pieces' normalised O
+        // weighted by l_i 2^(m_i - m) / sum_j l_j 2^(m_j - m), m the largest
+        // reference among pieces with l > 0.  Warp 0 (lane = row) forms the
+        // weights of up to four pieces at a time in cmax; then every thread
+        // gathers its column of those pieces, all rows at once.  The pieces
+        // were written by other CTAs of this grid: read through L2.  Called
+        // by all four warps between barriers (cmax is free there).
+        auto merge_pieces = [&](const ItemSlot& S) {
+            const int Hkv = p.num_kv_heads;
+            const int per = gridDim.x / Hkv;
+            // Slot of the k-th piece: the item's own, then the inner ones.
+            auto slot_of = [&](int k) {
+                if (k == 0) return S.unit;
+                int found = -1, i = 0;
+                for_each_inner_piece(S.item_a, S.item_n, S.axis_len, per, [&](int jj) {
+                    if (++i == k) found = p.num_units + jj;
+                });
+                return found;
+            };
+            int npieces = 1;
+            for_each_inner_piece(S.item_a, S.item_n, S.axis_len, per, [&](int) { ++npieces; });
+            const float2* ml = reinterpret_cast<const float2*>(p.piece_ml);
+            // Row totals (warp 0): largest reference and weight sum.
+            float M = -INFINITY, Lsum = 0.f;
+            if (warp == 0) {
+                for (int k = 0; k < npieces; ++k) {
+                    const float2 v = __ldcg(ml + ((size_t)slot_of(k) * Hkv + S.g) * kN + lane);
+                    if (!(v.y > 0.f)) continue;
+                    if (v.x > M) {
+                        Lsum *= exp2f(M - v.x);
+                        M = v.x;
+                    }
+                    Lsum += v.y * exp2f(v.x - M);
+                }
+            }
+            float acc[32];
+#pragma unroll
+            for (int r = 0; r < 32; ++r) acc[r] = 0.f;
+            for (int k0 = 0; k0 < npieces; k0 += 4) {
+                const int kn = min(4, npieces - k0);
+                if (warp == 0) {
+                    for (int q = 0; q < 4; ++q) {
+                        float w = 0.f;
+                        if (q < kn) {
+                            const float2 v =
+                                __ldcg(ml + ((size_t)slot_of(k0 + q) * Hkv + S.g) * kN + lane);
+                            w = (v.y > 0.f && Lsum > 0.f) ? v.y * exp2f(v.x - M) / Lsum : 0.f;
+                        }
+                        cmax[q * 32 + lane] = w;
+                    }
+                }
+                softmax_sync();
+                for (int q = 0; q < kn; ++q) {
+                    const float* po =
+                        p.piece_o + ((size_t)slot_of(k0 + q) * Hkv + S.g) * kN * kD + tid;
+                    float o[32];
+#pragma unroll
+                    for (int r = 0; r < 32; ++r) o[r] = __ldcg(po + (size_t)r * kD);
+#pragma unroll
+                    for (int r = 0; r < 32; r += 4) {
+                        const float4 w4 = *reinterpret_cast<const float4*>(cmax + q * 32 + r);
+                        acc[r] += w4.x * o[r];
+                        acc[r + 1] += w4.y * o[r + 1];
+                        acc[r + 2] += w4.z * o[r + 2];
+                        acc[r + 3] += w4.w * o[r + 3];
+                    }
+                }
+                softmax_sync();  // cmax is rewritten by the next batch
+            }
+#pragma unroll
+            for (int r = 0; r < 32; r += 2) {
+                const longlong2 rr = *reinterpret_cast<const longlong2*>(&S.row[r]);
+                if (rr.x >= 0) p.out[rr.x * kD + tid] = acc[r];
+                if (rr.y >= 0) p.out[rr.y * kD + tid] = acc[r + 1];
             }
         };
         // Epilogue of item i (slot sl): O^T (thread = d) / l into the output rows
-        // (one 4-byte store per row and thread; rows of one warp coalesce).
+        // (one 4-byte store per row and thread; rows of one warp coalesce).  A
+        // piece of a split item writes its partial instead and counts itself
+        // on the item's counter; the last to arrive merges the item.
         auto epilogue = [&](int i, int sl) {
-            const ItemSlot& S = slots[sl];
+            ItemSlot& S = slots[sl];
             const int ob = i & 1;
-            const bool okw = __all_sync(0xffffffffu, wait_bar(&o_full[ob], (i >> 1) & 1));
+            const bool piece = S.piece >= 0;
+            bool okw = __all_sync(0xffffffffu, wait_bar(&o_full[ob], (i >> 1) & 1));
+            // A piece's epilogue has barriers: the four warps agree first.
+            if (piece) okw = softmax_sync_count(!okw) == 0;
             if (!okw) {
                 fail = true;
                 return;
@@ -1151,26 +1431,62 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive_plain(&o_empty[ob]);
+            if (!piece) {
+#pragma unroll
+                for (int r = 0; r < 32; r += 4) {
+                    const float4 iv = *reinterpret_cast<const float4*>(&S.inv_l[r]);
+                    const longlong2 ra = *reinterpret_cast<const longlong2*>(&S.row[r]);
+                    const longlong2 rb = *reinterpret_cast<const longlong2*>(&S.row[r + 2]);
+                    const float inv[4] = {iv.x, iv.y, iv.z, iv.w};
+                    const long long row[4] = {ra.x, ra.y, rb.x, rb.y};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (row[e] >= 0)
+                            p.out[row[e] * kD + tid] =
+                                (__uint_as_float(o[r + e]) + __uint_as_float(olo[r + e])) *
+                                inv[e];
+                }
+                mbar_arrive_plain(&slot_free[sl]);
+                return;
+            }
+            const int Hkv = p.num_kv_heads;
+            const size_t base = ((size_t)S.piece * Hkv + S.g) * kN;
+            float* po = p.piece_o + base * kD + tid;
 #pragma unroll
             for (int r = 0; r < 32; r += 4) {
                 const float4 iv = *reinterpret_cast<const float4*>(&S.inv_l[r]);
-                const longlong2 ra = *reinterpret_cast<const longlong2*>(&S.row[r]);
-                const longlong2 rb = *reinterpret_cast<const longlong2*>(&S.row[r + 2]);
                 const float inv[4] = {iv.x, iv.y, iv.z, iv.w};
-                const long long row[4] = {ra.x, ra.y, rb.x, rb.y};
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
-                    if (row[e] >= 0)
-                        p.out[row[e] * kD + tid] =
-                            (__uint_as_float(o[r + e]) + __uint_as_float(olo[r + e])) * inv[e];
+                    po[(size_t)(r + e) * kD] =
+                        (__uint_as_float(o[r + e]) + __uint_as_float(olo[r + e])) * inv[e];
             }
+            if (tid < 32)
+                reinterpret_cast<float2*>(p.piece_ml)[base + tid] =
+                    make_float2(S.m_fin[tid], S.l_fin[tid]);
+            // Release the partial, count it, and acquire the others' if this
+            // piece is the last: the barrier orders every thread's stores
+            // before thread 0's fences and atomic.
+            softmax_sync();
+            if (tid == 0) {
+                __threadfence();
+                S.arrived = atomicAdd(&p.piece_count[(size_t)S.unit * Hkv + S.g], 1);
+                __threadfence();
+            }
+            softmax_sync();
+            int pieces = 1;
+            for_each_inner_piece(S.item_a, S.item_n, S.axis_len, gridDim.x / Hkv,
+                                 [&](int) { ++pieces; });
+            if (S.arrived == pieces - 1) merge_pieces(S);
             mbar_arrive_plain(&slot_free[sl]);
         };
 
+        // Reference and partial sum per row; a row keeps reference 0 until
+        // its first visible token (its tokens before that are masked).
         float m_ref[32], l_part[32];
 #pragma unroll
         for (int r = 0; r < 32; ++r) {
-            m_ref[r] = kNoMax;
+            m_ref[r] = 0.f;
             l_part[r] = 0.f;
         }
         int n = 0, item = 0;
@@ -1194,15 +1510,31 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             ItemSlot& S = slots[sl];
             const int nch = S.nch;
             if (nch < 0) break;
+            const int c0 = S.c0;
             if (prev >= 0) finish_sums(prev);
             const int min_lim = S.min_lim;
             const int ob = item & 1;
+            const uint32_t live_rows = S.live_rows;
+            const int nref = S.nref;
+            int kref = 0;  // next entry of the reference list
+            // Rows whose first visible token of the piece falls on this
+            // thread's column of some chunk.
+            uint32_t own = 0;
+#pragma unroll
+            for (int r = 0; r < 32; r += 4) {
+                const int4 f4 = *reinterpret_cast<const int4*>(&S.first[r]);
+                const int f[4] = {f4.x, f4.y, f4.z, f4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (f[e] >= 0 && (f[e] & (kTok - 1)) == tid) own |= 1u << (r + e);
+            }
 
-            for (int c = 0; c < nch; ++c, ++n) {
+            for (int c = c0; c < nch; ++c, ++n) {
                 const int sb = n & 1;
                 bool ok = !fail && __all_sync(0xffffffffu, wait_bar(&s_full[sb], (n >> 1) & 1));
                 float x[32];
                 bool dead = false;  // no row sees this thread's token
+                const int tok = c * kTok + tid;
                 if (ok) {
                     tc_fence_after();
                     uint32_t raw[32];
@@ -1212,49 +1544,74 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                     mbar_arrive_plain(&s_free[sb]);  // S(n+2) may overwrite the buffer
 #pragma unroll
                     for (int r = 0; r < 32; ++r) x[r] = __uint_as_float(raw[r]) * sl2;
-                    const int tok = c * kTok + tid;
                     if (c * kTok + kTok - 1 > min_lim) {
-                        // A row sees the shared tokens of its context and
-                        // its own tail (group mode).
-                        bool seen = false;
+                        // The rows that see this token: every row up to the
+                        // smallest limit; in the shared region (or in
+                        // multi-query mode) those whose limit reaches it;
+                        // past it, the rows of the one member whose tail
+                        // holds it (none on a tail's padding).
+                        uint32_t vis = live_rows;
+                        if (tok > min_lim) {
+                            if (tok < S.shared_r16) {
+                                vis = 0;
 #pragma unroll
-                        for (int r = 0; r < 32; r += 4) {
-                            const int4 lm = *reinterpret_cast<const int4*>(&S.lim[r]);
-                            const int4 lo = *reinterpret_cast<const int4*>(&S.tail_lo[r]);
-                            const int4 hi = *reinterpret_cast<const int4*>(&S.tail_hi[r]);
-                            const int l4[4] = {lm.x, lm.y, lm.z, lm.w};
-                            const int o4[4] = {lo.x, lo.y, lo.z, lo.w};
-                            const int h4[4] = {hi.x, hi.y, hi.z, hi.w};
+                                for (int r = 0; r < 32; r += 4) {
+                                    const int4 lm = *reinterpret_cast<const int4*>(&S.lim[r]);
+                                    vis |= (tok <= lm.x ? 1u : 0u) << r;
+                                    vis |= (tok <= lm.y ? 2u : 0u) << r;
+                                    vis |= (tok <= lm.z ? 4u : 0u) << r;
+                                    vis |= (tok <= lm.w ? 8u : 0u) << r;
+                                }
+                                vis &= live_rows;
+                            } else {
+                                // The last member whose tail starts at or
+                                // before tok (tails rise with the member):
+                                // a branch-free search over at most 32.
+                                const int nm = S.nmem;
+                                int lo = 0;
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const bool vis = tok <= l4[e] || (tok >= o4[e] && tok < h4[e]);
-                                if (!vis) x[r + e] = -INFINITY;
-                                seen = seen || vis;
+                                for (int step = 16; step >= 1; step >>= 1)
+                                    if (lo + step < nm && S.mem_v[lo + step] <= tok) lo += step;
+                                vis = (nm > 0 && S.mem_v[lo] <= tok && tok < S.mem_tend[lo])
+                                          ? S.mem_rows[lo]
+                                          : 0u;
                             }
                         }
-                        dead = !seen;
+#pragma unroll
+                        for (int r = 0; r < 32; ++r)
+                            if (!((vis >> r) & 1u)) x[r] = -INFINITY;
+                        dead = vis == 0;
                     }
                 } else {
 #pragma unroll
                     for (int r = 0; r < 32; ++r) x[r] = -INFINITY;
                 }
-                if (c == 0) {
-                    // References from the item's first token (thread 0).  The
-                    // previous readers of cmax passed the item barrier above.
-                    if (tid == 0) {
+                if (__builtin_expect(kref < nref && S.refc[kref] == c, 0)) {
+                    // Rows whose first visible token of the piece is in this
+                    // chunk take its logit as their reference, published by
+                    // the thread that owns the token (each row once a piece;
+                    // a row's earlier tokens were all masked, so its sum and
+                    // O^T row are still zero).
+                    const uint32_t rows = S.refm[kref];
+                    ++kref;
+                    const uint32_t mine = rows & own;
+                    if (mine != 0) {
 #pragma unroll
-                        for (int r = 0; r < 32; ++r) cmax[r] = x[r];
+                        for (int r = 0; r < 32; ++r)
+                            if ((mine >> r) & 1u) S.ref[r] = x[r];
                     }
                     softmax_sync();
 #pragma unroll
                     for (int r = 0; r < 32; r += 4) {
-                        const float4 c4 = *reinterpret_cast<const float4*>(cmax + r);
-                        const float c0[4] = {c4.x, c4.y, c4.z, c4.w};
+                        const float4 x4 = *reinterpret_cast<const float4*>(&S.ref[r]);
+                        const float rf[4] = {x4.x, x4.y, x4.z, x4.w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)  // -inf: a row that does not exist
-                            m_ref[r + e] = c0[e] > -INFINITY ? c0[e] : 0.f;
+                        for (int e = 0; e < 4; ++e)
+                            if ((rows >> (r + e)) & 1u)
+                                m_ref[r + e] = rf[e] > -INFINITY ? rf[e] : 0.f;
                     }
-                    // cmax is read again only after the vote barrier below.
+                    // Read before this chunk's vote barrier; the next writer
+                    // of a row's reference belongs to another item.
                 }
                 bool grow = false;
 #pragma unroll
@@ -1262,12 +1619,12 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 if (lane == 0 && aborted(abort_flag)) ok = false;
                 ok = __all_sync(0xffffffffu, ok);
                 const bool slow = softmax_sync_count(grow || !ok) != 0;
-                if (slow && softmax_sync_count(!ok) != 0) {
+                if (__builtin_expect(slow, 0) && softmax_sync_count(!ok) != 0) {
                     if (tid == 0) set_abort(abort_flag, p.error_flags);
                     stop = true;
                     break;
                 }
-                if (slow) {
+                if (__builtin_expect(slow, 0)) {
                     // Exact chunk max per row, then move the references.
                     float v[32];
 #pragma unroll
@@ -1286,7 +1643,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                         m_ref[r] = mn;
                         l_part[r] *= alpha[r];
                     }
-                    if (resc && c > 0) {
+                    if (resc && c > c0) {
                         // O^T must be stable: the previous PV has to be done.
                         const bool okp = __all_sync(
                             0xffffffffu, wait_bar(&pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1));
@@ -1351,7 +1708,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
 
                 // The previous item's epilogue, one chunk into this item when
                 // there is one: its last PV is then done, not just issued.
-                if (prev >= 0 && c == min(1, nch - 1)) {
+                if (__builtin_expect(prev >= 0 && c - c0 == min(1, nch - c0 - 1), 0)) {
                     epilogue(item - 1, prev);
                     prev = -1;
                 }
@@ -1363,9 +1720,13 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
 #pragma unroll
                 for (int r = 0; r < 32; ++r) v[r] = l_part[r];
                 S.red_l[lane][warp] = transpose_reduce<false>(v, lane);
+                if (tid == 0) {
+#pragma unroll
+                    for (int r = 0; r < 32; ++r) S.m_fin[r] = m_ref[r];
+                }
 #pragma unroll
                 for (int r = 0; r < 32; ++r) {
-                    m_ref[r] = kNoMax;
+                    m_ref[r] = 0.f;
                     l_part[r] = 0.f;
                 }
             }
@@ -1450,7 +1811,7 @@ cudaError_t mr_launch_typed(const MultiRowParams& p, cudaStream_t stream) {
     if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
     // One kv head per CTA, the same number of CTAs for every head (at least
     // one per head, at most one per item).
-    long long per_head = num_sms() / p.num_kv_heads;
+    long long per_head = multi_row_ctas_per_head(p.num_kv_heads);
     const long long head_items = (long long)p.num_units * p.tiles;
     if (per_head > head_items) per_head = head_items;
     if (per_head < 1) per_head = 1;
@@ -1472,6 +1833,11 @@ cudaError_t mr_launch_typed(const MultiRowParams& p, cudaStream_t stream) {
 }
 
 }  // namespace
+
+int multi_row_ctas_per_head(int num_kv_heads) {
+    const int n = num_sms() / (num_kv_heads > 0 ? num_kv_heads : 1);
+    return n > 0 ? n : 1;
+}
 
 cudaError_t launch_paged_multi_row(const MultiRowParams& p, cudaStream_t stream) {
     if (p.block_size == 16) return mr_launch_typed<16>(p, stream);

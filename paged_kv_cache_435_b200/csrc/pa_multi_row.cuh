@@ -35,6 +35,17 @@ struct MultiRowParams {
     int tiles;                       // 32-row tiles per sequence or group
     int num_units;                   // sequences or groups
     float scale_log2;                // scale * log2(e)
+    // Shared-prefix mode, optional (null: items are never split): a group's
+    // item may be split across CTAs inside its shared region.  A piece that
+    // does not cover the whole item writes its rows' (max, sum, normalised O)
+    // to slot `unit` (the piece at the item's start) or num_units + j (the
+    // piece CTA j of the head starts inside the item), and counts itself on
+    // the item's arrival counter (zeroed by the launch before this one); the
+    // last piece to arrive merges the item's pieces into the output.
+    float* piece_o;                  // fp32 [slots][Hkv][32][D]
+    float* piece_ml;                 // fp32 [slots][Hkv][32][2]
+    int32_t* piece_count;            // int32 [num_units][Hkv]
+    int piece_slots;                 // num_units + CTAs per kv head (at most)
 };
 
 // Rows handled per tile.
@@ -42,5 +53,8 @@ constexpr int kMultiRowTile = 32;
 
 // head_size 128 only; block_size 16 or 32.
 cudaError_t launch_paged_multi_row(const MultiRowParams& p, cudaStream_t stream);
+
+// CTAs per kv head the kernel launches at most on the current device.
+int multi_row_ctas_per_head(int num_kv_heads);
 
 }  // namespace pa

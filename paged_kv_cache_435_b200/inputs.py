@@ -56,6 +56,7 @@ class Workload:
     samples: int = 0
     prefix_tokens: int = 0
     tail_max: int = 0
+    first_prefix_tokens: int = 0      # prompt 0's prefix (0: prefix_tokens)
     # multi-query workloads: the last query_len tokens of each context are
     # the step's queries (0: decode, one query per sequence)
     query_len: int = 0
@@ -84,6 +85,13 @@ WORKLOADS = {
         description="32 prompts x 8 samples, 1024-token shared prefix "
                     "(64 blocks, refcount 8), CoW copy of prefix block 63 per "
                     "sample, tails U[0,256]; 32q/8kv, D=128, bs=16"),
+    "shared_prefix_skew": Workload(
+        "shared_prefix_skew", 8, 256, 32, 8, 128, 16, "shared",
+        prompts=32, samples=8, prefix_tokens=1024, tail_max=256,
+        first_prefix_tokens=32768,
+        description="as shared_prefix_cow, but prompt 0's prefix is 32768 "
+                    "tokens (2048 blocks shared by its 8 samples): one "
+                    "group's pass is several CTAs' share"),
     "long_skew_bs16": Workload(
         "long_skew_bs16", 5, 32, 32, 8, 128, 16, "skew:131072;64,1024",
         partition_size=512,
@@ -218,38 +226,44 @@ def build_shared_prefix_case(w: Workload, device="cpu",
     bs = w.block_size
     P, S = w.prompts, w.samples
     B = P * S
-    assert B == w.num_seqs and w.prefix_tokens % bs == 0
-    pblk = w.prefix_tokens // bs
+    first = w.first_prefix_tokens or w.prefix_tokens
+    assert B == w.num_seqs and w.prefix_tokens % bs == 0 and first % bs == 0
+    prefix = np.full(P, w.prefix_tokens, dtype=np.int64)
+    prefix[0] = first
+    pblks = prefix // bs
     tails = rng.integers(0, w.tail_max + 1, size=B).astype(np.int64)
-    lens = w.prefix_tokens + tails
+    lens = np.repeat(prefix, S) + tails
     tail_blocks = blocks_for(tails, bs)
-    need = P * pblk + B + int(tail_blocks.sum())
+    need = int(pblks.sum()) + B + int(tail_blocks.sum())
     NB = max(1, math.ceil(need * (1 + POOL_SLACK)))
     perm = rng.permutation(NB).astype(np.int32)
     cursor = 0
-    prompt_blocks = perm[cursor:cursor + P * pblk].reshape(P, pblk)
-    cursor += P * pblk
-    MB = pblk + int(tail_blocks.max())
+    prompt_blocks = []
+    for p in range(P):
+        prompt_blocks.append(perm[cursor:cursor + int(pblks[p])])
+        cursor += int(pblks[p])
+    MB = int(pblks.max()) + int(tail_blocks.max())
     tables = np.full((B, MB), -1, dtype=np.int32)
     pairs = np.zeros((B, 2), dtype=np.int64)
     for p in range(P):
+        pblk = int(pblks[p])
         for j in range(S):
             s = p * S + j
             tables[s, :pblk] = prompt_blocks[p]
             private = int(perm[cursor]); cursor += 1
-            pairs[s] = (prompt_blocks[p, pblk - 1], private)
+            pairs[s] = (prompt_blocks[p][pblk - 1], private)
             tables[s, pblk - 1] = private
             n = int(tail_blocks[s])
             tables[s, pblk:pblk + n] = perm[cursor:cursor + n]
             cursor += n
-    unique = P * (pblk - 1) * bs + B * bs + int(tails.sum())
+    unique = int(((pblks - 1) * bs).sum()) + B * bs + int(tails.sum())
     case = _finish(w, lens, tables, NB, pairs, device,
                    2000 + w.wid if seed is None else seed + 1, pool_device,
                    unique_tokens=unique)
     # The samples of a prompt share its blocks up to the copied last one.
     dev = torch.device(device)
     gs = (np.arange(P + 1) * S).astype(np.int32)
-    pl = np.full(P, (pblk - 1) * bs, dtype=np.int32)
+    pl = ((pblks - 1) * bs).astype(np.int32)
     return dataclasses.replace(case, group_start=torch.from_numpy(gs).to(dev),
                                prefix_lens=torch.from_numpy(pl).to(dev),
                                max_group_size=S)

@@ -217,11 +217,17 @@ def test_shared_prefix_host_validation(lib):
 
 
 def test_shared_prefix_workspace_grows_with_rows(lib):
-    # The shared-prefix call needs only the per-sequence pass's split scratch.
+    # The per-sequence pass's split scratch, then the group pass's pieces:
+    # (B + 148 / Hkv) slots x Hkv x 32 rows of D + 2 floats, and B x Hkv
+    # counters, each region 256-byte aligned (no device here: 148 SMs).
+    def a256(x):
+        return (x + 255) // 256 * 256
     for B in (8, 16):
         for part in (0, 64):
-            assert (nat.pa_shared_prefix_workspace_size(B, 32, 8, 128, 16, 1000, part) ==
-                    nat.pa_decode_workspace_size(B, 32, 8, 128, 16, 1000, part))
+            split = nat.pa_decode_workspace_size(B, 32, 8, 128, 16, 1000, part)
+            rows = (B + 148 // 8) * 8 * 32
+            want = a256(a256(a256(a256(split) + rows * 128 * 4) + rows * 2 * 4) + B * 8 * 4)
+            assert nat.pa_shared_prefix_workspace_size(B, 32, 8, 128, 16, 1000, part) == want
     a = nat.pa_shared_prefix_workspace_size(8, 32, 8, 128, 16, 1000)
     b = nat.pa_shared_prefix_workspace_size(16, 32, 8, 128, 16, 1000)
     assert b > a > 0

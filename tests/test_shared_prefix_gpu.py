@@ -55,11 +55,14 @@ def check(case, expect_flags=0, **kw):
     return assert_attn_close(out, reference(case), case.workload.name), out
 
 
-def test_parallel_sampling_workload():
+@pytest.mark.parametrize("name", ["shared_prefix_cow", "shared_prefix_skew"])
+def test_parallel_sampling_workload(name):
     """32 prompts x 8 samples (32q/8kv, D=128, bs=16): the copy-on-write step
-    and the new token's write run first; groups share 63 of the 64 prompt
-    blocks (the 64th is each sample's private copy)."""
-    case = inputs.make_case("shared_prefix_cow", device="cuda")
+    and the new token's write run first; groups share their prompt's blocks
+    but the last (each sample's private copy).  In the skewed batch prompt 0
+    has 32768 tokens, so its group's pass is cut into pieces across CTAs;
+    every output is compared."""
+    case = inputs.make_case(name, device="cuda")
     ek, ev = bits(case.k_cache), bits(case.v_cache)
     pa.pa_copy_blocks([case.k_cache], [case.v_cache], case.copy_pairs)
     pa.pa_reshape_and_cache(case.new_key, case.new_value, case.k_cache,
@@ -241,3 +244,39 @@ def test_more_than_768_sequences(partition_size):
     case = inputs.grouped_case(32, 8, 128, 16, lens, gs, pl, seed=800,
                                device="cuda")
     check(case, partition_size=partition_size)
+
+
+@pytest.mark.parametrize("Hq,Hkv,bs,scale", [(32, 8, 16, None), (32, 8, 16, 1.0),
+                                             (8, 8, 32, None)])
+def test_items_cut_across_ctas(Hq, Hkv, bs, scale):
+    """One group with long private tails among many short groups: the items
+    are dealt by chunks, so the long one is cut into pieces on several CTAs,
+    most of which start inside the tails, where a row's first visible token
+    lies chunks into the piece.  The group also holds a member shorter than
+    its prefix and one that ends exactly at it.  Scale 1.0 makes the logits
+    spread far beyond the rescale threshold.  The piece merge order is fixed,
+    so repeated calls are bitwise equal."""
+    import dataclasses
+    G = Hq // Hkv
+    members = 32 // G if G > 1 else 20
+    P0 = 4 * bs
+    rng = np.random.default_rng(Hq * 7 + bs)
+    tails = rng.integers(900, 1800, size=members)
+    tails[2] = -(P0 - 24)          # ends inside the prefix
+    tails[3] = 0                   # ends exactly at the prefix
+    tails[5] = 17
+    lens = list(P0 + tails)
+    gs, pl = [0, members], [P0]
+    for i in range(20):
+        lens += list(bs + rng.integers(0, 60, size=2))
+        gs.append(gs[-1] + 2)
+        pl.append(bs)
+    lens += [700, 5]               # outside every group
+    case = inputs.grouped_case(Hq, Hkv, 128, bs, lens, gs, pl, seed=Hq + bs + 5,
+                               device="cuda")
+    if scale is not None:
+        case = dataclasses.replace(case, scale_override=scale)
+    (_, _), a = check(case)
+    b = run(case)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
