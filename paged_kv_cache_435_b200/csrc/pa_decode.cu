@@ -891,15 +891,56 @@ paged_decode_reduce_kernel(const DecodeParams p) {
         p.out[((int64_t)s * p.num_heads + h) * D + d] = combined_column<D>(sm, M, d) / den;
 }
 
-// Range-worker grid: a persistent grid over work items (sequence, query
-// head, slice of kMergeRows candidate rows).  A sequence's candidate rows
-// are its partition slots, then the range boundaries strictly inside it
-// (live when the boundary is no partition start and is the last worker
-// starting there).  Each CTA scans the published slice counts into a work
-// list; an item merges its slice in one round; a sequence with one slice is
-// written at once, otherwise each slice writes its (max, sum, normalised O)
-// and the last of the sequence's slices to arrive (an arrival counter the
-// partition kernel zeroed) merges them.  No CTA waits on another.
+// Candidate rows of a split sequence for one query head: its partition
+// slots, then the range boundaries strictly inside it (live when the
+// boundary is no partition start and is the last worker starting there).
+// Loads rows i0 + u * step (u < kReduceUnroll, those below total) in one
+// round and folds them into a.
+template <int D>
+__device__ __forceinline__ void fold_candidates(const DecodeParams& p, MergeAcc<D>& a, int i0,
+                                                int step, int total, int nslot, int b_lo, int xs,
+                                                int q, int nw, int64_t slot_base,
+                                                int64_t st_base, int lane) {
+    constexpr int V = D / 32;
+    const int32_t* E = p.worker_bounds;
+    float mv[kReduceUnroll], lv[kReduceUnroll], vals[kReduceUnroll][V];
+    int e0[kReduceUnroll], e1[kReduceUnroll];
+    bool live[kReduceUnroll], in_slots[kReduceUnroll];
+#pragma unroll
+    for (int u = 0; u < kReduceUnroll; ++u) {
+        const int i = i0 + u * step;
+        const bool ok = i < total;
+        in_slots[u] = i < nslot;
+        const int b = min(max(b_lo + i - nslot, 0), nw - 1);
+        const int64_t r = in_slots[u] ? slot_base + i : st_base + b;
+        e0[u] = (ok && !in_slots[u]) ? E[b] : 0;
+        e1[u] = (ok && !in_slots[u]) ? E[b + 1] : 0;
+        mv[u] = ok ? (in_slots[u] ? p.tmp_m : p.st_m)[r] : -INFINITY;
+        lv[u] = ok ? (in_slots[u] ? p.tmp_l : p.st_l)[r] : 0.f;
+        load_row<D>((in_slots[u] ? p.tmp_o : p.st_o) + r * D + lane * V, ok, vals[u]);
+        live[u] = ok;
+    }
+#pragma unroll
+    for (int u = 0; u < kReduceUnroll; ++u)
+        live[u] = live[u] && (in_slots[u] || ((e0[u] - xs) % q != 0 && e1[u] > e0[u]));
+    a.fold(mv, lv, vals, live);
+}
+
+// A split sequence with at most this many candidate rows is merged by one
+// warp; longer ones by CTAs, kMergeRows rows per slice.
+constexpr int kWarpMergeMax = 2 * kReduceUnroll;
+
+// Range-worker grid: a persistent grid over the split sequences.  Each CTA
+// scans the published chunk prefix into two work lists.  Long sequences
+// (more than kWarpMergeMax candidate rows) are merged by CTA items
+// (sequence, query head, slice of kMergeRows rows), one round per slice: a
+// sequence with one slice is written at once, otherwise each slice writes
+// its (max, sum, normalised O) and the last of the sequence's slices to
+// arrive (an arrival counter the partition kernel zeroed) merges them.
+// Short ones (most split sequences: two or three pieces) are merged whole by
+// one warp per (sequence, query head), in one or two rounds with no CTA
+// barrier.  A CTA takes its long items first, so the slices that gate a
+// second level are done early.  No CTA waits on another.
 template <int D>
 __global__ void __launch_bounds__(kReduceWarps * 32, 2)
 paged_decode_merge_kernel(const DecodeParams p) {
@@ -907,25 +948,28 @@ paged_decode_merge_kernel(const DecodeParams p) {
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int Hq = p.num_heads;
-    // Per sequence, computed once by the CTA: merge slices (as a prefix over
-    // sequences: the work list), partition slots, first boundary candidate,
-    // candidate count and first chunk.
-    __shared__ int work[kMaxPersistSeqs + 1];
+    // Per sequence, computed once by the CTA: CTA slices and warp items (as
+    // prefixes over sequences: the work lists), partition slots, first
+    // boundary candidate, candidate count and first chunk.
+    __shared__ int work[kMaxPersistSeqs + 1], work_w[kMaxPersistSeqs + 1];
     __shared__ int g_nslot[kMaxPersistSeqs], g_blo[kMaxPersistSeqs];
     __shared__ int g_total[kMaxPersistSeqs], g_xs[kMaxPersistSeqs];
+    __shared__ int wsum[2][kReduceWarps];
     __shared__ MergeSmem<D> sm;
     __shared__ int is_last;
     pdl_wait();  // the partials come from the grid launched just before
 
     const long long T = p.chunk_prefix[p.num_seqs];
-    const long long nw = p.range_workers;
+    const int nw = p.range_workers;
     const int q = p.partition_size / kChunk;
-    const int32_t* E = p.worker_bounds;
-    int running = 0;
-    if (threadIdx.x == 0) work[0] = 0;
+    int running = 0, running_w = 0;
+    if (threadIdx.x == 0) {
+        work[0] = 0;
+        work_w[0] = 0;
+    }
     for (int base = 0; base < p.num_seqs; base += kReduceWarps * 32) {
         const int s = base + threadIdx.x;
-        int v = 0;
+        int v = 0, vw = 0;
         if (s < p.num_seqs) {
             const long long xs = p.chunk_prefix[s];
             const long long cs = p.chunk_prefix[s + 1] - xs;
@@ -933,11 +977,14 @@ paged_decode_merge_kernel(const DecodeParams p) {
             if (cs > 0) {
                 nslot = (int)((cs + q - 1) / q);
                 const long long lo = max(1LL, ((xs + 1) * nw + T - 1) / T);
-                const long long hi = min(nw - 1, ((xs + cs) * nw + T - 1) / T - 1);
+                const long long hi = min((long long)nw - 1, ((xs + cs) * nw + T - 1) / T - 1);
                 b_lo = (int)lo;
                 ncand = hi >= lo ? (int)(hi - lo + 1) : 0;
                 // Two slots, or one slot and a boundary inside: split.
-                if (nslot >= 2 || ncand >= 1) v = (nslot + ncand + kMergeRows - 1) / kMergeRows;
+                if (nslot >= 2 || ncand >= 1) {
+                    if (nslot + ncand <= kWarpMergeMax) vw = 1;
+                    else v = (nslot + ncand + kMergeRows - 1) / kMergeRows;
+                }
             }
             g_nslot[s] = nslot;
             g_blo[s] = b_lo;
@@ -947,60 +994,56 @@ paged_decode_merge_kernel(const DecodeParams p) {
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int t = __shfl_up_sync(0xffffffffu, v, o);
-            if (lane >= o) v += t;
+            const int tw = __shfl_up_sync(0xffffffffu, vw, o);
+            if (lane >= o) {
+                v += t;
+                vw += tw;
+            }
         }
-        if (lane == 31) sm.m[warp] = __int_as_float(v);
+        if (lane == 31) {
+            wsum[0][warp] = v;
+            wsum[1][warp] = vw;
+        }
         __syncthreads();
-        int before = running;
-        for (int w = 0; w < warp; ++w) before += __float_as_int(sm.m[w]);
-        if (s < p.num_seqs) work[s + 1] = before + v;
-        for (int w = 0; w < kReduceWarps; ++w) running += __float_as_int(sm.m[w]);
+        int before = running, before_w = running_w;
+        for (int w = 0; w < warp; ++w) {
+            before += wsum[0][w];
+            before_w += wsum[1][w];
+        }
+        if (s < p.num_seqs) {
+            work[s + 1] = before + v;
+            work_w[s + 1] = before_w + vw;
+        }
+        for (int w = 0; w < kReduceWarps; ++w) {
+            running += wsum[0][w];
+            running_w += wsum[1][w];
+        }
         __syncthreads();
     }
     const int total_items = running * Hq;
+    // Largest s with list[s] <= k.
+    auto seq_of = [&](const int* list, int k) {
+        int lo = 0, hi = p.num_seqs - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (list[mid] <= k) lo = mid; else hi = mid - 1;
+        }
+        return lo;
+    };
 
     for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
         const int h = item % Hq;
         const int gsl = item / Hq;
-        int lo = 0, hi = p.num_seqs - 1;  // largest s with work[s] <= gsl
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (work[mid] <= gsl) lo = mid; else hi = mid - 1;
-        }
-        const int s = lo;
+        const int s = seq_of(work, gsl);
         const int sl = gsl - work[s];
         const int nsl = work[s + 1] - work[s];
-        const int nslot = g_nslot[s], b_lo = g_blo[s], total = g_total[s];
-        const int xs = g_xs[s];
         const int64_t slot_base = ((int64_t)s * Hq + h) * p.max_partitions;
         const int64_t st_base = (int64_t)h * p.max_range_workers;
 
         // First level: candidate rows [sl * kMergeRows, +kMergeRows), one round.
         MergeAcc<D> a;
-        {
-            float mv[kReduceUnroll], lv[kReduceUnroll], vals[kReduceUnroll][V];
-            int e0[kReduceUnroll], e1[kReduceUnroll];
-            bool live[kReduceUnroll], in_slots[kReduceUnroll];
-#pragma unroll
-            for (int u = 0; u < kReduceUnroll; ++u) {
-                const int i = sl * kMergeRows + warp + u * kReduceWarps;
-                const bool ok = i < total;
-                in_slots[u] = i < nslot;
-                const int b = min(max(b_lo + i - nslot, 0), (int)nw - 1);
-                const int64_t r = in_slots[u] ? slot_base + i : st_base + b;
-                e0[u] = (ok && !in_slots[u]) ? E[b] : 0;
-                e1[u] = (ok && !in_slots[u]) ? E[b + 1] : 0;
-                mv[u] = ok ? (in_slots[u] ? p.tmp_m : p.st_m)[r] : -INFINITY;
-                lv[u] = ok ? (in_slots[u] ? p.tmp_l : p.st_l)[r] : 0.f;
-                load_row<D>((in_slots[u] ? p.tmp_o : p.st_o) + r * D + lane * V, ok, vals[u]);
-                live[u] = ok;
-            }
-#pragma unroll
-            for (int u = 0; u < kReduceUnroll; ++u)
-                live[u] = live[u] && (in_slots[u] ||
-                                      ((e0[u] - xs) % q != 0 && e1[u] > e0[u]));
-            a.fold(mv, lv, vals, live);
-        }
+        fold_candidates<D>(p, a, sl * kMergeRows + warp, kReduceWarps, g_total[s], g_nslot[s],
+                           g_blo[s], g_xs[s], q, nw, slot_base, st_base, lane);
         float M, den;
         combine_warps<D>(a, sm, M, den);
         float* out_row = p.out + ((int64_t)s * Hq + h) * D;
@@ -1048,6 +1091,25 @@ paged_decode_merge_kernel(const DecodeParams p) {
         for (int d = threadIdx.x; d < D; d += kReduceWarps * 32)
             out_row[d] = combined_column<D>(sm, M, d) / den;
         __syncthreads();
+    }
+
+    // Short split sequences: one warp per (sequence, query head), no barrier.
+    const int total_w = running_w * Hq;
+    for (int it = blockIdx.x * kReduceWarps + warp; it < total_w;
+         it += gridDim.x * kReduceWarps) {
+        const int h = it % Hq;
+        const int s = seq_of(work_w, it / Hq);
+        const int total = g_total[s];
+        const int64_t slot_base = ((int64_t)s * Hq + h) * p.max_partitions;
+        const int64_t st_base = (int64_t)h * p.max_range_workers;
+        MergeAcc<D> a;
+        for (int i0 = 0; i0 < total; i0 += kReduceUnroll)
+            fold_candidates<D>(p, a, i0, 1, total, g_nslot[s], g_blo[s], g_xs[s], q, nw,
+                               slot_base, st_base, lane);
+        float* out_row = p.out + ((int64_t)s * Hq + h) * D + lane * V;
+        const float inv = a.den > 0.f ? 1.f / a.den : 0.f;
+#pragma unroll
+        for (int v = 0; v < V; ++v) out_row[v] = a.acc[v] * inv;
     }
 }
 
