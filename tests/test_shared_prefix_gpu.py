@@ -280,3 +280,26 @@ def test_items_cut_across_ctas(Hq, Hkv, bs, scale):
     b = run(case)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+def test_cut_items_with_invalid_group_and_empty_member():
+    """G = 8 (four members per 32-row tile).  A dominant group whose pass is
+    cut into pieces holds an empty member (context 0: no visible token in
+    any piece, output 0) and a member shorter than the prefix; an invalid
+    group (prefix not a multiple of the block size) falls back to the
+    per-sequence pass and is flagged; twenty small groups and two lone
+    sequences fill the batch."""
+    bs, P0 = 16, 160
+    lens = [P0 + 1500, 0, 100, P0 + 1777]              # group 0 (dominant)
+    lens += [300, 320]                                  # group 1 (made invalid below)
+    gs, pl = [0, 4, 6], [P0, 48]
+    rng = np.random.default_rng(64)
+    for i in range(20):
+        lens += list(bs + rng.integers(0, 40, size=2))
+        gs.append(gs[-1] + 2)
+        pl.append(bs)
+    lens += [900, 3]
+    case = inputs.grouped_case(64, 8, 128, bs, lens, gs, pl, seed=64, device="cuda")
+    bad = torch.tensor([P0, 40] + pl[2:], dtype=torch.int32)   # 40: not whole blocks
+    (_, _), out = check(case, expect_flags=pa.PA_DEVERR_PREFIX, prefix_lens=bad)
+    assert torch.count_nonzero(out[1]).item() == 0
