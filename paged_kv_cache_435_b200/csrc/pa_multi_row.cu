@@ -144,8 +144,8 @@ constexpr int kSlotOff = kCmaxOff + 512;
 constexpr int kBarOff = kSlotOff + kSlots * (int)sizeof(ItemSlot);
 // barriers: k_full[KS] k_empty[KS] v_full[VS] v_empty[VS] s_full[2] s_free[2]
 //           p_full[2] pv_done[2] o_full[2] o_empty[2] q_empty[2] item_ready[4]
-//           slot_free[4] drain
-constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 15 + 2 * kSlots;
+//           slot_free[4] drain item_meta[4]
+constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 15 + 3 * kSlots;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16;
 constexpr uint32_t kTmemCols = 256;       // S0 | S1 | O0 (hi, lo) | O1 (hi, lo)
 constexpr uint32_t kTmemO = 64;           // first O column
@@ -597,6 +597,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
     uint64_t* item_ready = q_empty + 2;
     uint64_t* slot_free = item_ready + kSlots;
     uint64_t* drain = slot_free + kSlots;
+    uint64_t* item_meta = drain + 1;  // the slot's fields (producers); item_ready adds Q
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
     int* abort_flag = reinterpret_cast<int*>(smem + kBarOff + kNumBars * 8 + 4);
     float* cmax = reinterpret_cast<float*>(smem + kCmaxOff);
@@ -632,6 +633,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
         }
         for (int i = 0; i < kSlots; ++i) {
             mbar_init(&item_ready[i], 32);
+            mbar_init(&item_meta[i], 32);
             mbar_init(&slot_free[i], 128);
         }
         mbar_init(drain, 1);
@@ -688,6 +690,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             ItemSlot& S = slots[s];
             if (end) {
                 if (lane == 0) S.nch = -1;
+                mbar_arrive_plain(&item_meta[s]);
                 mbar_arrive_plain(&item_ready[s]);
                 return true;
             }
@@ -791,7 +794,13 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 S.nmem = p.shared_prefix_mode ? it.nmem : 0;
                 S.shared_r16 = shared_r16;
                 S.P = p.shared_prefix_mode ? it.P : 0;
+                // The producers' first block-table read, on its way to L2.
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(
+                    p.block_tables + (int64_t)it.table_seq * p.max_blocks_per_seq +
+                    (c0 * kTok) / BS));
             }
+            // The producers need the fields only; the MMA warp also the Q rows.
+            mbar_arrive_plain(&item_meta[s]);
             // Q^T row `lane` (K-major, 128-byte swizzle; zeros for a missing row).
             const uint32_t qb = smem_u32(smem + kQOff + (live & 1) * kQBytes);
             const unsigned char* src =
@@ -1123,7 +1132,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
         bool ok = true;
         for (int item = 0; ok; ++item) {
             const int sl = item % kSlots;
-            if (!__all_sync(0xffffffffu, wait_bar(&item_ready[sl], (item / kSlots) & 1))) {
+            if (!__all_sync(0xffffffffu, wait_bar(&item_meta[sl], (item / kSlots) & 1))) {
                 if (lane == 0) set_abort(abort_flag, p.error_flags);
                 break;
             }
