@@ -36,8 +36,9 @@ struct MultiRowParams {
     int num_units;                   // sequences or groups
     float scale_log2;                // scale * log2(e)
     // Shared-prefix mode, optional (null: items are never split): a group's
-    // item may be split across CTAs inside its shared region.  A piece that
-    // does not cover the whole item writes its rows' (max, sum, normalised O)
+    // item may be cut at 128-token chunk boundaries into pieces on several
+    // CTAs.  A piece that does not cover the whole item writes its rows'
+    // (reference, sum, normalised O)
     // to slot `unit` (the piece at the item's start) or num_units + j (the
     // piece CTA j of the head starts inside the item), and counts itself on
     // the item's arrival counter (zeroed by the launch before this one); the
