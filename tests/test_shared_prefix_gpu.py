@@ -303,3 +303,22 @@ def test_cut_items_with_invalid_group_and_empty_member():
     bad = torch.tensor([P0, 40] + pl[2:], dtype=torch.int32)   # 40: not whole blocks
     (_, _), out = check(case, expect_flags=pa.PA_DEVERR_PREFIX, prefix_lens=bad)
     assert torch.count_nonzero(out[1]).item() == 0
+
+
+@pytest.mark.parametrize("Hkv", [1, 2, 4])
+def test_cut_items_fewer_kv_heads(Hkv):
+    """The split deal with 148, 74 and 37 CTAs per kv head (G = 4): one group
+    with long tails among thirty short groups, so its pass is cut into many
+    pieces, most of them inside the tails."""
+    G, bs, P0 = 4, 16, 64
+    rng = np.random.default_rng(100 + Hkv)
+    lens = list(P0 + rng.integers(800, 2400, size=8))
+    gs, pl = [0, 8], [P0]
+    for i in range(30):
+        lens += list(bs + rng.integers(0, 50, size=2))
+        gs.append(gs[-1] + 2)
+        pl.append(bs)
+    lens += [333]
+    case = inputs.grouped_case(G * Hkv, Hkv, 128, bs, lens, gs, pl, seed=200 + Hkv,
+                               device="cuda")
+    check(case)
