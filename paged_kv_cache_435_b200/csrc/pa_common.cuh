@@ -116,6 +116,20 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     return pol;
 }
 
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;"
+                 : "=l"(pol));
+    return pol;
+}
+
+// 8-byte store with an L2 eviction-priority hint.
+__device__ __forceinline__ void st_global_f2_hint(float* ptr, float a, float b, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;" ::"l"(ptr), "f"(a),
+                 "f"(b), "l"(pol)
+                 : "memory");
+}
+
 // ------------------------------------------- programmatic dependent launch
 // Wait until the grids this launch depends on have completed and their
 // memory is visible (no-op when the launch carries no programmatic edge).

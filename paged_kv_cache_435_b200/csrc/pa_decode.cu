@@ -659,10 +659,20 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                     dst = p.st_o + pidx * D;
                 }
                 const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+                if (it.kind == kWhole) {
 #pragma unroll
-                for (int j = 0; j < D / 8; ++j)
-                    *reinterpret_cast<float2*>(dst + 8 * j + qc) =
-                        make_float2((o[j][0] + o[j][2]) * inv, (o[j][1] + o[j][3]) * inv);
+                    for (int j = 0; j < D / 8; ++j)
+                        *reinterpret_cast<float2*>(dst + 8 * j + qc) =
+                            make_float2((o[j][0] + o[j][2]) * inv, (o[j][1] + o[j][3]) * inv);
+                } else {
+                    // A partial: kept in L2 for the merge kernel, which reads
+                    // it right after this grid while the KV stream evicts.
+                    const uint64_t keep = l2_policy_evict_last();
+#pragma unroll
+                    for (int j = 0; j < D / 8; ++j)
+                        st_global_f2_hint(dst + 8 * j + qc, (o[j][0] + o[j][2]) * inv,
+                                          (o[j][1] + o[j][3]) * inv, keep);
+                }
                 if (it.kind != kWhole && (lane & 3) == 0) {
                     float* dm = it.kind == kSlot ? p.tmp_m : p.st_m;
                     float* dl = it.kind == kSlot ? p.tmp_l : p.st_l;
