@@ -62,6 +62,28 @@ def test_shared_prefix_workload_structure():
     assert (case.lens_np >= 64 * bs).all() and (case.lens_np <= 64 * bs + 256).all()
 
 
+def test_skewed_shared_prefix_workload_structure():
+    """Prompt 0 shares 2047 blocks (its last block is each sample's copy);
+    the other prompts as in the uniform workload; unique tokens count every
+    shared block once."""
+    case = inputs.make_case("shared_prefix_skew")
+    w = case.workload
+    bs = w.block_size
+    gs = case.group_start.numpy()
+    pl = case.prefix_lens.numpy()
+    assert pl[0] == 2047 * bs and (pl[1:] == 63 * bs).all()
+    rows = case.tables_np[gs[0]:gs[1]]
+    assert (rows[:, :2047] == rows[0, :2047]).all()
+    assert len(set(rows[:, 2047].tolist())) == 8
+    assert (case.lens_np[:8] >= 2048 * bs).all() and (case.lens_np[8:] < 2048 * bs).all()
+    # Every distinct (block, offset) position read: each group's shared
+    # blocks once, every sample's copied block and tail.
+    tails = case.lens_np - np.repeat(np.where(np.arange(32) == 0, 2048, 64) * bs, 8)
+    assert case.unique_tokens == int(pl.sum()) + w.num_seqs * bs + int(tails.sum())
+    # The uniform workload's draws are unchanged by the skewed one's field.
+    assert inputs.make_case("shared_prefix_cow").unique_tokens == 69927
+
+
 def test_multi_query_case_places_queries_at_the_end():
     lens, qlens = [40, 300, 7], [8, 128, 7]
     case = inputs.multi_query_case(3, 16, 4, 64, 16, lens, qlens, seed=3)
