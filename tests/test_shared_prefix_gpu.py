@@ -322,3 +322,39 @@ def test_cut_items_fewer_kv_heads(Hkv):
     case = inputs.grouped_case(G * Hkv, Hkv, 128, bs, lens, gs, pl, seed=200 + Hkv,
                                device="cuda")
     check(case)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_grouped_batches(seed):
+    """Randomised grouped batches: G in 1..8 with 1, 2, 4 or 8 kv heads,
+    block size 16 or 32, groups of random size (one 32-row tile each) with
+    prefixes of 0..40 blocks and tails of 0..1500 tokens, lone sequences
+    between them, and in most seeds one group whose pass dominates (a long
+    prefix or long tails), which takes the split deal.  Every output is
+    compared with the oracle."""
+    rng = np.random.default_rng(4000 + seed)
+    Hkv = int(rng.choice([1, 2, 4, 8]))
+    G = int(rng.integers(1, 9))
+    bs = int(rng.choice([16, 32]))
+    mpt = 32 // G if G > 1 else 16
+    lens, gs, pl = [], [], []
+    for gi in range(int(rng.integers(5, 30))):
+        if rng.random() < 0.2:
+            lens.append(int(rng.integers(0, 900)))        # a lone sequence
+        m = int(rng.integers(1, mpt + 1))
+        P = int(rng.integers(0, 41)) * bs
+        dominant = gi == 0 and seed % 3 != 2
+        tails = rng.integers(0, 2500 if dominant else 300, size=m)
+        if dominant and seed % 2 == 0:
+            P = int(rng.integers(150, 400)) * bs          # a long shared prefix
+        start = len(lens)
+        lens += [int(P + t) for t in tails]
+        if rng.random() < 0.3 and m > 1:
+            lens[start + 1] = int(rng.integers(0, P + 1))  # ends inside the prefix
+        gs.append(start)
+        pl.append(P)
+    gs.append(len(lens))
+    lens.append(int(rng.integers(1, 500)))               # one after the last group
+    case = inputs.grouped_case(G * Hkv, Hkv, 128, bs, lens, gs, pl, seed=5000 + seed,
+                               device="cuda")
+    check(case)
