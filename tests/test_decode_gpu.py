@@ -204,3 +204,25 @@ def test_workspace_too_small_is_rejected_before_launch():
                                case.scale, partition_size=64, workspace=ws)
     assert e.value.status == pa.PA_ERR_WORKSPACE
     assert pa.pa_launch_count() == n0
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_random_split_batches(seed):
+    """Randomised long-context batches on the persistent split path: a few
+    long sequences (so their merge runs as CTA slices, more than 16 candidate
+    rows) among many short ones that straddle worker boundaries (merged
+    whole by one warp each), with random head shapes, head size, block size
+    and a forced partition size.  Every output is compared with the oracle."""
+    rng = np.random.default_rng(6000 + seed)
+    Hkv = int(rng.choice([1, 2, 4, 8]))
+    G = int(rng.choice([1, 2, 4, 8]))
+    D = int(rng.choice([64, 128]))
+    bs = int(rng.choice([16, 32]))
+    part = int(rng.choice([128, 256, 512]))
+    n_long = int(rng.integers(1, 4))
+    lens = list(rng.integers(8000, 40000, size=n_long)) + \
+        list(rng.integers(0, 1200, size=int(rng.integers(20, 200))))
+    rng.shuffle(lens)
+    case = inputs.custom_case(len(lens), G * Hkv, Hkv, D, bs, lens, seed=7000 + seed,
+                              device="cuda")
+    run_and_check(case, partition_size=part)
