@@ -1704,11 +1704,14 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                     // as late as possible so the wait rarely blocks.
                     const int vs = n % kVStages;
                     if (!wait_bar(&v_full[vs], (n / kVStages) & 1)) fail = true;
+                    // Rows are 128 bytes apart: thread t starts at 16-byte
+                    // column t % 8 so that eight lanes cover all banks.
                     unsigned char* vr = smem + kVOff + vs * kStageBytes + tid * 128;
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        *reinterpret_cast<uint4*>(vr + j * 16) = make_uint4(0, 0, 0, 0);
-                        *reinterpret_cast<uint4*>(vr + kHalf + j * 16) = make_uint4(0, 0, 0, 0);
+                        const int col = ((j + tid) & 7) * 16;
+                        *reinterpret_cast<uint4*>(vr + col) = make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4*>(vr + kHalf + col) = make_uint4(0, 0, 0, 0);
                     }
                 }
                 fence_proxy_async_smem();

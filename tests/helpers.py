@@ -84,3 +84,34 @@ def oracle_attention(case, k_bits, v_bits, seqs=None):
     return oracle.paged_decode_attention(q, k_bits, v_bits, tables, lens,
                                          case.scale,
                                          case.workload.num_kv_heads)
+
+
+# Bit patterns a never-written bf16 slot may hold: NaN, +inf, -inf, -NaN.
+_POISON = np.array([0x7FC0, 0x7F80, 0xFF80, 0xFFC1], dtype=np.uint16)
+
+
+def poison_unwritten_slots(case, extra_live=()):
+    """Fill every K and V slot that no sequence's context covers (the rows
+    past the last token of each last block, blocks no table reaches) with
+    NaN and infinities.  A kernel must never let such a slot reach an
+    output: the attention of a sequence depends on its first L tokens only.
+    `extra_live`: further (sequence, length) pairs whose tokens stay as they
+    are.  Returns the number of poisoned slots."""
+    bs = case.workload.block_size
+    NB = case.k_cache.shape[0]
+    live = np.zeros(NB * bs, dtype=bool)
+    pairs = list(zip(range(len(case.lens_np)), case.lens_np)) + list(extra_live)
+    for s, L in pairs:
+        L = int(L)
+        if L <= 0:
+            continue
+        t = np.arange(L)
+        ids = case.tables_np[s, t // bs].astype(np.int64)
+        live[ids * bs + t % bs] = True
+    dead = np.nonzero(~live)[0]
+    pattern = torch.from_numpy(_POISON[dead % 4].view(np.int16).copy())
+    idx = torch.from_numpy(dead)
+    for pool in (case.k_cache, case.v_cache):
+        flat = pool.view(NB * bs, -1).view(torch.int16)
+        flat[idx.to(pool.device)] = pattern.to(pool.device)[:, None]
+    return int(dead.size)
