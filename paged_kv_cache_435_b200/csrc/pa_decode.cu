@@ -320,6 +320,18 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
             for (int s = a; s < b; ++s) atomicOr(&grouped_bits[s >> 5], 1u << (s & 31));
         }
         __syncthreads();
+        if (!kWarpRanges) {
+            // Every sequence answered by the group pass: nothing to stream
+            // and no output to write (no merge follows without a split).
+            bool any = false;
+            for (int w = threadIdx.x; w < (p.num_seqs + 31) / 32; w += kThreads) {
+                const uint32_t mine = w == (p.num_seqs - 1) / 32 && (p.num_seqs & 31)
+                                          ? (1u << (p.num_seqs & 31)) - 1u
+                                          : 0xffffffffu;
+                any = any || (grouped_bits[w] & mine) != mine;
+            }
+            if (__syncthreads_or(any) == 0) return;
+        }
     }
     if (kPersist) {
         // X[s] = 16-token chunks of sequences 0..s-1 (block-wide scan).  The
