@@ -358,3 +358,33 @@ def test_random_grouped_batches(seed):
     case = inputs.grouped_case(G * Hkv, Hkv, 128, bs, lens, gs, pl, seed=5000 + seed,
                                device="cuda")
     check(case)
+
+
+@pytest.mark.parametrize("lone_last", [False, True])
+def test_every_sequence_grouped_ragged_batch(lone_last):
+    """37 sequences (the grouped bitmap's last word is partial), G = 4: every
+    sequence in a valid group, one of them empty, so the per-sequence pass
+    has nothing to answer; with `lone_last` the 37th sequence is outside
+    every group and that pass must attend it."""
+    G, Hkv, bs = 4, 8, 16
+    rng = np.random.default_rng(37 + lone_last)
+    lens, gs, pl = [], [], []
+    while len(lens) < 37:
+        m = min(int(rng.integers(1, 9)), 37 - len(lens))
+        P = int(rng.integers(1, 20)) * bs
+        gs.append(len(lens))
+        pl.append(P)
+        lens += [int(P + t) for t in rng.integers(0, 300, size=m)]
+    lens[5] = 0                                              # an empty member
+    if lone_last:
+        if gs[-1] == 36:                                     # the last group is that one sequence
+            gs.pop()
+            pl.pop()
+        lens[36] = 901
+        gs.append(36)
+    else:
+        gs.append(37)
+    case = inputs.grouped_case(G * Hkv, Hkv, 128, bs, lens, gs, pl, seed=370 + lone_last,
+                               device="cuda")
+    (_, _), out = check(case)
+    assert torch.count_nonzero(out[5]).item() == 0
