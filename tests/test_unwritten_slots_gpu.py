@@ -27,15 +27,17 @@ def _need_gpu():
 RAGGED = [1, 15, 17, 31, 33, 100, 257, 1000, 0, 2, 4095, 130]
 
 
-@pytest.mark.parametrize("Hq,Hkv,bs,partition", [
-    (32, 32, 16, 0),       # MHA, whole sequences
-    (64, 8, 16, 0),        # GQA 8
-    (64, 8, 32, 512),      # forced split + merge
-    (16, 2, 16, 64),       # many partitions per sequence
+@pytest.mark.parametrize("Hq,Hkv,D,bs,partition", [
+    (32, 32, 128, 16, 0),      # MHA, whole sequences
+    (64, 8, 128, 16, 0),       # GQA 8
+    (64, 8, 128, 32, 512),     # forced split + merge
+    (16, 2, 128, 16, 64),      # many partitions per sequence
+    (16, 4, 64, 16, 0),        # head size 64
+    (16, 4, 64, 32, 128),      # head size 64, split
 ])
-def test_decode_ignores_unwritten_slots(Hq, Hkv, bs, partition):
-    case = inputs.custom_case(len(RAGGED), Hq, Hkv, 128, bs, RAGGED,
-                              seed=7000 + Hq + bs + partition, device="cuda")
+def test_decode_ignores_unwritten_slots(Hq, Hkv, D, bs, partition):
+    case = inputs.custom_case(len(RAGGED), Hq, Hkv, D, bs, RAGGED,
+                              seed=7000 + Hq + D + bs + partition, device="cuda")
     assert poison_unwritten_slots(case) > 0
     flags = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = gpu_step(case, partition_size=partition, error_flags=flags,
@@ -53,9 +55,20 @@ def test_decode_ignores_unwritten_slots(Hq, Hkv, bs, partition):
     (24, 8, 16, [129, 127, 1000, 2], [11, 16, 3, 2]),            # G = 3
 ])
 def test_multi_query_ignores_unwritten_slots(monkeypatch, kernel, Hq, Hkv, bs, lens, qlens):
+    run_multi_query(monkeypatch, kernel, Hq, Hkv, 128, bs, lens, qlens)
+
+
+@pytest.mark.parametrize("bs", [16, 32])
+def test_multi_query_head64_ignores_unwritten_slots(monkeypatch, bs):
+    """Head size 64 runs on the mma.sync kernel."""
+    run_multi_query(monkeypatch, "mma", 16, 4, 64, bs, [300, 65, 129, 31, 1000],
+                    [5, 3, 8, 31, 64])
+
+
+def run_multi_query(monkeypatch, kernel, Hq, Hkv, D, bs, lens, qlens):
     monkeypatch.setenv("PA_MULTI_QUERY_KERNEL", kernel)
-    case = inputs.multi_query_case(len(lens), Hq, Hkv, 128, bs, lens, qlens,
-                                   seed=7100 + sum(lens) + Hq, device="cuda")
+    case = inputs.multi_query_case(len(lens), Hq, Hkv, D, bs, lens, qlens,
+                                   seed=7100 + sum(lens) + Hq + D, device="cuda")
     assert poison_unwritten_slots(case) > 0
     flags = torch.zeros(1, dtype=torch.int32, device="cuda")
     pa.pa_reshape_and_cache(case.new_key, case.new_value, case.k_cache,
