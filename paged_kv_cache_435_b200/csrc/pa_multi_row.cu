@@ -51,13 +51,13 @@
 //              (reference, sum, normalised O) and the last piece of an item to
 //              finish merges them into the output.  For each item or piece
 //              it works out the token range, block-table rows, each row's
-//              visible tokens and output row into a 4-slot shared-memory ring
-//              and copies the Q rows (cp.async), so no other warp waits on a
-//              global load at an item boundary.
-// Online softmax with a lazy reference: each row starts from the logit of its
-// first visible token of the item or piece (so its sum is at least 1),
-// published through shared memory by the thread that owns that token in the
-// chunk that holds it; until then the row's tokens are all masked.  Every chunk,
+//              visible tokens, output row and reference into a 4-slot
+//              shared-memory ring and copies the Q rows (cp.async), so no
+//              other warp waits on a global load at an item boundary.
+// Online softmax with a lazy reference: each row starts from its logit at
+// its first visible token of the item or piece (so its sum is at least 1),
+// which the scheduler computes (q . k of that token's K row) when it
+// publishes the item; the row's tokens before that one are masked.  Every chunk,
 // one barrier-reduction over the 4 warps (bar.red.popc) asks whether any
 // row's logit exceeds its reference by more than 2^24 (weights stay below
 // 2^24, far from fp32 overflow, and the split of P keeps its relative
@@ -117,14 +117,11 @@ struct ItemSlot {
     int unit, item_n;                   // split item: group, its chunks
     int item_a, axis_len;               // split item: first position, axis
                                         // length (see the split deal)
-    int nref;                           // entries of refc / refm
+    int pad0_;
     uint32_t live_rows;                 // rows that exist (bit r: row r)
     float m_fin[32], l_fin[32];         // rows: reference and sum at the end
     float ref[32];                      // rows: logit at the first visible token
-    int first[32];                      // rows: first visible token of the
-                                        // piece (-1: none)
-    int refc[32];                       // chunks holding first tokens, rising,
-    uint32_t refm[32];                  // and the rows whose first token each holds
+                                        // of the piece (0: none), the scheduler's
     int min_lim, nmem, shared_r16, P;   // smallest row limit; members (group
                                         // mode); end of the shared region
                                         // rounded to 16; prefix length
@@ -138,14 +135,14 @@ struct ItemSlot {
     float red_l[32][4];                 // per-warp partial row sums
     float inv_l[32];                    // 1 / row sum (0 for an empty row)
 };
-static_assert(sizeof(ItemSlot) == 2512 && sizeof(ItemSlot) % 16 == 0, "slot layout");
+static_assert(sizeof(ItemSlot) == 2128 && sizeof(ItemSlot) % 16 == 0, "slot layout");
 
 constexpr int kSlotOff = kCmaxOff + 512;
 constexpr int kBarOff = kSlotOff + kSlots * (int)sizeof(ItemSlot);
 // barriers: k_full[KS] k_empty[KS] v_full[VS] v_empty[VS] s_full[2] s_free[2]
 //           p_full[2] pv_done[2] o_full[2] o_empty[2] q_empty[2] item_ready[4]
-//           slot_free[4] drain item_meta[4]
-constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 15 + 3 * kSlots;
+//           slot_free[4] drain item_meta[4] item_refs[4]
+constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 15 + 4 * kSlots;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16;
 constexpr uint32_t kTmemCols = 256;       // S0 | S1 | O0 (hi, lo) | O1 (hi, lo)
 constexpr uint32_t kTmemO = 64;           // first O column
@@ -598,6 +595,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
     uint64_t* slot_free = item_ready + kSlots;
     uint64_t* drain = slot_free + kSlots;
     uint64_t* item_meta = drain + 1;  // the slot's fields (producers); item_ready adds Q
+    uint64_t* item_refs = item_meta + kSlots;  // and the rows' references (softmax)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
     int* abort_flag = reinterpret_cast<int*>(smem + kBarOff + kNumBars * 8 + 4);
     float* cmax = reinterpret_cast<float*>(smem + kCmaxOff);
@@ -634,6 +632,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
         for (int i = 0; i < kSlots; ++i) {
             mbar_init(&item_ready[i], 32);
             mbar_init(&item_meta[i], 32);
+            mbar_init(&item_refs[i], 32);
             mbar_init(&slot_free[i], 128);
         }
         mbar_init(drain, 1);
@@ -692,6 +691,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 if (lane == 0) S.nch = -1;
                 mbar_arrive_plain(&item_meta[s]);
                 mbar_arrive_plain(&item_ready[s]);
+                mbar_arrive_plain(&item_refs[s]);
                 return true;
             }
             int lim;
@@ -756,27 +756,18 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                     if (f < tail_hi && f < c1 * kTok) first = f;
                 }
             }
-            S.first[lane] = first;
-            // The chunks that hold first tokens, rising, each with its rows:
-            // entry k in lane k.
-            const int fc = first >= 0 ? first / kTok : 0x7fffffff;
-            int nref = 0, last = -1, refc = 0;
-            uint32_t refm = 0;
-            for (;;) {
-                int cm = fc > last ? fc : 0x7fffffff;
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) cm = min(cm, __shfl_xor_sync(0xffffffffu, cm, o));
-                if (cm == 0x7fffffff) break;
-                const uint32_t m = __ballot_sync(0xffffffffu, fc == cm);
-                if (lane == nref) {
-                    refc = cm;
-                    refm = m;
-                }
-                ++nref;
-                last = cm;
+            // Row lane's reference is its logit at that token: the token's
+            // block id (the shared region from the group's table, a tail from
+            // its member's, as the producers map it) is loaded now and used
+            // after the Q copy is under way.
+            const int m_seq = __shfl_sync(0xffffffffu, mseq, my_m);
+            int ref_id = 0, ref_tok = 0;
+            if (first >= 0) {
+                const bool in_shared = first < shared_r16;
+                const int seq = in_shared ? it.table_seq : m_seq;
+                ref_tok = in_shared ? first : it.P + (first - t_lo);
+                ref_id = p.block_tables[(int64_t)seq * p.max_blocks_per_seq + ref_tok / BS];
             }
-            S.refc[lane] = refc;
-            S.refm[lane] = refm;
             if (lane == 0) {
                 S.table_seq = it.table_seq;
                 S.g = it.g;
@@ -788,7 +779,6 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 S.item_n = split ? pc.n : it.nch;  // the deal's count (pieces)
                 S.item_a = pc.a;
                 S.axis_len = pc.T;
-                S.nref = nref;
                 S.live_rows = live_rows;
                 S.min_lim = ml;
                 S.nmem = p.shared_prefix_mode ? it.nmem : 0;
@@ -811,9 +801,46 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 cp_async_16(qb + (c16 >> 3) * kQHalf + lane * 128 +
                                 (((c16 & 7) ^ (lane & 7)) << 4),
                             src + c16 * 16, nbytes);
+            const uint16_t* krow = nullptr;
+            if (first >= 0) {
+                if (ref_id < 0 || ref_id >= p.num_blocks) {
+                    report(p.error_flags, PA_DEVERR_BLOCK_ID);
+                    ref_id = 0;
+                }
+                krow = p.k_cache +
+                       ((int64_t)(ref_id * BS + ref_tok % BS) * p.num_kv_heads + it.g) * kD;
+            }
             cp_async_wait_all();
             fence_proxy_async_smem();
             mbar_arrive_plain(&item_ready[s]);
+            // The reference: q . k in fp32 (bf16 products are exact), in the
+            // softmax's log2 units.  Any value near the row's logits serves
+            // (it only shifts the exponent; the softmax's growth check covers
+            // a row whose logits rise far above it); the token's own weight
+            // is then ~1, so the row's sum never underflows.
+            float ref = 0.f;
+            if (krow != nullptr) {
+                const unsigned char* qrow = smem + kQOff + (live & 1) * kQBytes + lane * 128;
+                float acc = 0.f;
+#pragma unroll 4
+                for (int c16 = 0; c16 < 16; ++c16) {
+                    const uint4 qv = *reinterpret_cast<const uint4*>(
+                        qrow + (c16 >> 3) * kQHalf + (((c16 & 7) ^ (lane & 7)) << 4));
+                    const uint4 kv = __ldg(reinterpret_cast<const uint4*>(krow + c16 * 8));
+                    const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+                    const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        acc = fmaf(__uint_as_float(qw[e] << 16), __uint_as_float(kw[e] << 16), acc);
+                        acc = fmaf(__uint_as_float(qw[e] & 0xffff0000u),
+                                   __uint_as_float(kw[e] & 0xffff0000u), acc);
+                    }
+                }
+                ref = acc * p.scale_log2;
+                if (!(ref > -INFINITY)) ref = 0.f;  // an overflowed or NaN product
+            }
+            S.ref[lane] = ref;
+            mbar_arrive_plain(&item_refs[s]);
             ++live;
             return true;
         };
@@ -901,8 +928,8 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
         // whose positions it owns.
         // Split only when one item alone exceeds 1.5 times a CTA's even
         // share: whole items dealt longest first balance to within about one
-        // item, and a piece costs its partial write, reference barriers and
-        // a share of the merge.
+        // item, and a piece costs its partial write and a share of the
+        // merge.
         long long Tl = 0;  // the split deal's axis length
         int wmax = 0;      // its longest item
 #pragma unroll
@@ -1490,8 +1517,9 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             mbar_arrive_plain(&slot_free[sl]);
         };
 
-        // Reference and partial sum per row; a row keeps reference 0 until
-        // its first visible token (its tokens before that are masked).
+        // Reference and partial sum per row; the reference starts as the
+        // row's logit at its first visible token of the item (the
+        // scheduler's; its tokens before that are masked).
         float m_ref[32], l_part[32];
 #pragma unroll
         for (int r = 0; r < 32; ++r) {
@@ -1507,7 +1535,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
 
         for (;; ++item) {
             const int sl = item % kSlots;
-            const bool okw = wait_bar(&item_ready[sl], (item / kSlots) & 1);
+            const bool okw = wait_bar(&item_refs[sl], (item / kSlots) & 1);
             // One barrier per item: the four warps agree on stopping, and the
             // previous item's partial sums are visible.
             const bool bad = !okw || fail || (tid == 0 && aborted(abort_flag));
@@ -1524,18 +1552,13 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
             const int min_lim = S.min_lim;
             const int ob = item & 1;
             const uint32_t live_rows = S.live_rows;
-            const int nref = S.nref;
-            int kref = 0;  // next entry of the reference list
-            // Rows whose first visible token of the piece falls on this
-            // thread's column of some chunk.
-            uint32_t own = 0;
 #pragma unroll
             for (int r = 0; r < 32; r += 4) {
-                const int4 f4 = *reinterpret_cast<const int4*>(&S.first[r]);
-                const int f[4] = {f4.x, f4.y, f4.z, f4.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    if (f[e] >= 0 && (f[e] & (kTok - 1)) == tid) own |= 1u << (r + e);
+                const float4 r4 = *reinterpret_cast<const float4*>(&S.ref[r]);
+                m_ref[r] = r4.x;
+                m_ref[r + 1] = r4.y;
+                m_ref[r + 2] = r4.z;
+                m_ref[r + 3] = r4.w;
             }
 
             for (int c = c0; c < nch; ++c, ++n) {
@@ -1594,33 +1617,6 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                 } else {
 #pragma unroll
                     for (int r = 0; r < 32; ++r) x[r] = -INFINITY;
-                }
-                if (__builtin_expect(kref < nref && S.refc[kref] == c, 0)) {
-                    // Rows whose first visible token of the piece is in this
-                    // chunk take its logit as their reference, published by
-                    // the thread that owns the token (each row once a piece;
-                    // a row's earlier tokens were all masked, so its sum and
-                    // O^T row are still zero).
-                    const uint32_t rows = S.refm[kref];
-                    ++kref;
-                    const uint32_t mine = rows & own;
-                    if (mine != 0) {
-#pragma unroll
-                        for (int r = 0; r < 32; ++r)
-                            if ((mine >> r) & 1u) S.ref[r] = x[r];
-                    }
-                    softmax_sync();
-#pragma unroll
-                    for (int r = 0; r < 32; r += 4) {
-                        const float4 x4 = *reinterpret_cast<const float4*>(&S.ref[r]);
-                        const float rf[4] = {x4.x, x4.y, x4.z, x4.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            if ((rows >> (r + e)) & 1u)
-                                m_ref[r + e] = rf[e] > -INFINITY ? rf[e] : 0.f;
-                    }
-                    // Read before this chunk's vote barrier; the next writer
-                    // of a row's reference belongs to another item.
                 }
                 bool grow = false;
 #pragma unroll
@@ -1737,10 +1733,7 @@ paged_multi_row_kernel(const __grid_constant__ CUtensorMap tm_k,
                     for (int r = 0; r < 32; ++r) S.m_fin[r] = m_ref[r];
                 }
 #pragma unroll
-                for (int r = 0; r < 32; ++r) {
-                    m_ref[r] = 0.f;
-                    l_part[r] = 0.f;
-                }
+                for (int r = 0; r < 32; ++r) l_part[r] = 0.f;
             }
             prev = sl;
         }
