@@ -168,3 +168,30 @@ def test_multi_row_kernel_long_context(monkeypatch):
     case = inputs.multi_query_case(3, 16, 2, 128, 16, [131072, 300, 17],
                                    [4, 4, 4], seed=131, device="cuda")
     check(case)
+
+
+@pytest.mark.parametrize("kernel", ["rows", "tc", "mma"])
+def test_bad_first_block_id_sets_flag_without_fault(monkeypatch, kernel):
+    """Sequence 1's first block id is out of range: every row of it has its
+    first visible token there (the 32-row kernel's scheduler reads that K
+    row for the row's reference).  The flag is set, nothing faults, and the
+    other sequences' outputs stay exact."""
+    monkeypatch.setenv("PA_MULTI_QUERY_KERNEL", kernel)
+    case = inputs.multi_query_case(3, 32, 8, 128, 16, [300, 200, 129], [4, 4, 4],
+                                   seed=77, device="cuda")
+    ek, ev = bits(case.k_cache), bits(case.v_cache)
+    case.block_tables[1, 0] = case.k_cache.shape[0] + 3      # out of range
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = gpu_mq(case, flags)
+    torch.cuda.synchronize()
+    assert int(flags.item()) & pa.PA_DEVERR_BLOCK_ID
+    oracle.reshape_and_cache(case.new_key.cpu(), case.new_value.cpu(), ek, ev,
+                             case.slot_mapping.cpu().numpy())
+    tables = case.tables_np.copy()
+    qsl = case.query_start_loc.cpu().numpy()
+    ref = oracle.paged_multi_query_attention(
+        case.q.cpu(), ek, ev, tables, case.lens_np.astype(np.int32), qsl,
+        case.scale, case.workload.num_kv_heads)
+    for s in (0, 2):
+        a, b = int(qsl[s]), int(qsl[s + 1])
+        assert_attn_close(out[a:b], ref[a:b], f"seq {s} beside a bad table ({kernel})")
