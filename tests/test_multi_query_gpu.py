@@ -195,3 +195,17 @@ def test_bad_first_block_id_sets_flag_without_fault(monkeypatch, kernel):
     for s in (0, 2):
         a, b = int(qsl[s]), int(qsl[s + 1])
         assert_attn_close(out[a:b], ref[a:b], f"seq {s} beside a bad table ({kernel})")
+
+
+@pytest.mark.parametrize("scale", [1.0, 4.0])
+def test_multi_row_kernel_large_logits(monkeypatch, scale):
+    """Scale 1 and 4 instead of 1/sqrt(D): logits of tens to hundreds (log2
+    units), a sharply peaked softmax.  The 32-row kernel's reference (each
+    row's logit at its first token, summed by the scheduler apart from the
+    tensor core's S) and its growth check must keep every row exact."""
+    monkeypatch.setenv("PA_MULTI_QUERY_KERNEL", "rows")
+    case = inputs.multi_query_case(4, 64, 8, 128, 16, [300, 1000, 17, 2049],
+                                   [4, 4, 4, 4], seed=4100 + int(scale), device="cuda")
+    case.scale_override = scale
+    (_, _), out = check(case)
+    assert torch.isfinite(out).all()

@@ -388,3 +388,22 @@ def test_every_sequence_grouped_ragged_batch(lone_last):
                                device="cuda")
     (_, _), out = check(case)
     assert torch.count_nonzero(out[5]).item() == 0
+
+
+@pytest.mark.parametrize("scale", [1.0, 4.0])
+def test_large_logits_grouped_batch(scale):
+    """Scale 1 and 4: sharply peaked rows through the group pass, whole and
+    cut into pieces (one long group), against the oracle."""
+    G, Hkv, bs, P0 = 4, 2, 16, 64
+    rng = np.random.default_rng(4200 + int(scale))
+    lens = list(P0 + rng.integers(800, 2400, size=8))
+    gs, pl = [0, 8], [P0]
+    for i in range(12):
+        lens += list(bs + rng.integers(0, 50, size=2))
+        gs.append(gs[-1] + 2)
+        pl.append(bs)
+    case = inputs.grouped_case(G * Hkv, Hkv, 128, bs, lens, gs, pl, seed=4300 + int(scale),
+                               device="cuda")
+    case.scale_override = scale
+    (_, _), out = check(case)
+    assert torch.isfinite(out).all()
