@@ -321,9 +321,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
         }
         __syncthreads();
         if (!kWarpRanges) {
-            // When the group pass answers every sequence, this CTA has
-            // nothing to stream and no output to write (and without a split
-            // no merge follows): it returns before the scan.
+            // Every sequence answered by the group pass: nothing to stream
+            // and no output to write (no merge follows without a split).
             bool any = false;
             for (int w = threadIdx.x; w < (p.num_seqs + 31) / 32; w += kThreads) {
                 const uint32_t mine = w == (p.num_seqs - 1) / 32 && (p.num_seqs & 31)
